@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Benchmark of the fused decode FFN half-layer ("mono" kernel) on B200.
+
+One step = one fused MoE layer-step of the chosen workload (all rows, every
+stage of the layer, n_layers persistent launches).  Inputs are seeded and
+synthetic; the weights are generated on the device and packed before timing.
+L2 is flushed (512 MiB write) before every timed step, and four hc_in sets
+rotate so the routed experts change from step to step.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs per fused MoE layer-step and achieved HBM GB/s (% of peak), rows=1..8"
+UNIT = "us/layer-step"
+FLUSH_BYTES = 512 << 20
+N_INPUT_SETS = 4
+KERNEL_SOURCES = ["moe_decode_layer_sm_b200/csrc/mono_ffn.cu", "moe_decode_layer_sm_b200/csrc/mono_ffn_kernel.cuh",
+                  "moe_decode_layer_sm_b200/csrc/ptx.cuh"]
+
+
+def kernel_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def workload(name):
+    from synth import configs as C
+    return C.BY_NAME[name]
+
+
+def wl_config(wl, extra=None):
+    cfg = {"workload": wl.name, "rows": wl.rows, "hidden": wl.hidden, "hc_streams": wl.hc,
+           "routed_experts": wl.n_routed, "top_k": wl.top_k, "shared_experts": 1, "inter": wl.inter,
+           "layers_per_step": wl.n_layers, "expert_format": wl.w_dtype, "hc_format": wl.hc_dtype,
+           "l2": "flushed before every timed step (512 MiB write)",
+           "inputs": f"{N_INPUT_SETS} rotating seeded hc_in sets"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def dtype_of(wl):
+    return {"f32": "f32", "bf16": "bf16", "fp8": "fp8e4m3", "mxfp4": "mxfp4"}[wl.w_dtype]
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mono_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ CPU baseline --
+
+def cpu_oracle_sample(wl, budget_s=12.0):
+    """Time the CPU oracle (as it stands) on one full layer-step of the
+    workload's first input set; weights of the touched experts are generated
+    before the clock starts.  Repeats while the budget lasts."""
+    from oracle import oracle as O
+    from synth import synth as S
+    hc = S.cpu_hc_in(wl)
+    lws = []
+    x = hc
+    for l in range(wl.n_layers):
+        dense = S.cpu_dense(wl, l)
+        t = O.route(wl, O.LayerWeights(wl, dense, {}), x)
+        slots = sorted(set(int(e) for e in t.idx.ravel()) | {wl.n_routed})
+        lw = O.LayerWeights(wl, dense, {e: S.cpu_expert(wl, l, e) for e in slots})
+        lws.append(lw)
+        if l + 1 < wl.n_layers:
+            x, _ = O.layer(wl, lw, x)
+    times = []
+    t_end = time.time() + budget_s
+    while time.time() < t_end or not times:
+        t0 = time.perf_counter()
+        if wl.n_layers == 1:
+            O.layer(wl, lws[0], hc)
+        else:
+            O.chain(wl, lws, hc, deferred=True)
+        times.append(time.perf_counter() - t0)
+        if len(times) >= 5:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    us = statistics.median(times) * 1e6 / wl.n_layers
+    return {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(times)} full layer-step(s) of {wl.name} ({wl.rows} rows, {wl.n_layers} layer(s)), "
+                      f"median; touched experts generated before timing"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workload(args.config)
+    # bounded: the whole --steps K --warmup W run stays within a few minutes
+    budget = min(20.0, max(5.0, 60.0 / max(1, args.steps + args.warmup)))
+    cb = cpu_oracle_sample(wl, budget_s=budget)
+    line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": cb["value"] / 1000.0, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+            "config": wl_config(wl, {"parallelism": "single host process"}), "impl": "reference",
+            "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- GPU path --
+
+TRACE_NAMES = ["start", "mix published", "mix totals seen", "n ready", "logits published", "lists ready",
+               "shared gate/up done", "routed gate/up done", "activations seen", "down done", "end",
+               "producer saw lists", "producer issued all"]
+
+
+def print_trace(plan, wl, sets, out, flush):
+    """One extra traced step: stage timestamps relative to the earliest CTA
+    start, min / median / max over CTAs (µs), to stderr."""
+    import torch
+    info = plan.info()
+    G = info["grid"]
+    buf = torch.zeros(wl.n_layers * G * 16, dtype=torch.int64, device="cuda")
+    plan.set_trace(buf)
+    flush.zero_()
+    plan.step(wl.rows, sets[0], out)
+    torch.cuda.synchronize()
+    plan.set_trace(None)
+    t = buf.view(wl.n_layers, G, 16).cpu().numpy().astype("float64")
+    for l in range(wl.n_layers):
+        t0 = t[l, :, 0].min()
+        print(f"layer {l}: stage times in us from the first CTA start (min / median / max over CTAs)", file=sys.stderr)
+        for i, nm in enumerate(TRACE_NAMES):
+            col = t[l, :, i]
+            col = col[col > 0]
+            if len(col) == 0:
+                continue
+            d = (col - t0) / 1000.0
+            print(f"  {i:2d} {nm:22s} {d.min():9.2f} {statistics.median(d):9.2f} {d.max():9.2f}  (n={len(col)})",
+                  file=sys.stderr)
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from moe_decode_layer_sm_b200 import Plan
+    from synth import synth as S
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = workload(args.config)
+    if args.routed:
+        wl = wl.with_(name=f"{wl.name}-e{args.routed}", n_routed=args.routed)
+    plan = Plan.for_workload(wl, device=local)
+    info = plan.info()
+    for l in range(wl.n_layers):
+        d = S.gpu_dense(wl, l)
+        ex = S.gpu_experts(wl, l)
+        plan.pack(l, d["mix_w"], d["norm_w"], d["router_w"], d["router_bias"], ex["gate"][0], ex["up"][0],
+                  ex["down"][0], ex["gate"][1], ex["up"][1], ex["down"][1])
+        torch.cuda.synchronize()
+        del ex, d
+        torch.cuda.empty_cache()
+    # input sets: seeds differ per set and per rank (independent replicas)
+    sets = [S.gpu_hc_in(wl.with_(seed=wl.seed + 1000 * i + 7919 * rank)) for i in range(N_INPUT_SETS)]
+    out = torch.empty_like(sets[0])
+    idx_taps = [torch.zeros((wl.rows, wl.top_k), dtype=torch.int32, device="cuda") for _ in range(wl.n_layers)]
+    for l in range(wl.n_layers):
+        plan.set_taps(l, idx=idx_taps[l])
+    # unique experts touched per input set (for the byte count)
+    uniq = []
+    for i in range(N_INPUT_SETS):
+        plan.step(wl.rows, sets[i], out)
+        rc, st = plan.query_error()
+        if rc != 0:
+            raise SystemExit(f"device error {rc} stage {st.stage}")
+        uniq.append([len(set(t.cpu().numpy().ravel().tolist())) for t in idx_taps])
+    hc_bytes = wl.rows * wl.hc * wl.hidden * (2 if wl.hc_dtype == "bf16" else 4)
+    bytes_per_set = [sum(info["dense_bytes"] + (u + 1) * info["expert_bytes"] + 2 * hc_bytes for u in us)
+                     for us in uniq]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    for k in range(args.warmup):
+        flush.zero_()
+        plan.step(wl.rows, sets[k % N_INPUT_SETS], out)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        ev[k][0].record(stream)
+        plan.step(wl.rows, sets[k % N_INPUT_SETS], out)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+
+    # end to end through the host-buffer entry point: H2D of the step's hc_in
+    # from pinned memory, the step, D2H of the result, per step
+    host_in = [s.cpu().pin_memory() for s in sets]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    KE = min(K, args.e2e_steps)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KE)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(KE):
+        flush.zero_()
+        ev2[k][0].record(stream)
+        plan.step_host(wl.rows, host_in[k % N_INPUT_SETS], host_out)
+        ev2[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = [a.elapsed_time(b) for a, b in ev2]
+    clk = clocks.stop()
+    if args.trace:
+        print_trace(plan, wl, sets, out, flush)
+    rc, st = plan.query_error()
+    if rc != 0:
+        raise SystemExit(f"device error {rc} stage {st.stage}")
+
+    tot_ms = sum(step_ms)
+    tot_e2e = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms, tot_e2e], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, tot_e2e = t.tolist()
+    us_per_step = tot_ms * 1000.0 / K
+    value = us_per_step / wl.n_layers / world       # whole job: layer-steps of all ranks per unit time
+    mean_bytes = sum(bytes_per_set[k % N_INPUT_SETS] for k in range(K)) / K
+    achieved = mean_bytes / (tot_ms / 1000.0 / K) / 1e9
+    pk, pk_kind = peaks()
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", f"traffic_{wl.name}.json")
+    if os.path.exists(tr_path):
+        tr = json.load(open(tr_path))
+        if tr.get("kernel_sha") == kernel_sha():
+            traffic = tr.get("dram_bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": tot_ms / K, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_of(wl), "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
+        "config": wl_config(wl, {"parallelism": "replicas" if world > 1 else "single GPU"}),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "peak_kind": f"{pk_kind} HBM copy", "frac_of_8tbs_nominal": achieved / 8000.0,
+                     "algorithmic_bytes_per_step": mean_bytes,
+                     "unique_routed_experts_per_layer": statistics.mean(x for us in uniq for x in us)},
+        "e2e": {"value": tot_e2e * 1000.0 / KE / wl.n_layers / world, "unit": UNIT, "h2d_bytes_per_step": hc_bytes,
+                "d2h_bytes_per_step": hc_bytes},
+        "gpu_launches": K * wl.n_layers,
+        "clocks": clk,
+        "step_us_p10_p50_p90": [float(np.percentile(step_ms, q)) * 1000.0 for q in (10, 50, 90)],
+        "plan": {k: info[k] for k in ("grid", "threads", "smem_bytes", "ring_stages", "ring_slot_bytes")},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(wl)
+    plan.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="mono", choices=["mono", "reference"])
+    ap.add_argument("--config", default="v41flash-bf16-r1")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--routed", type=int, default=0, help="override the routed-expert count (small profiling cases)")
+    ap.add_argument("--trace", action="store_true", help="print per-stage device timestamps (stderr) after the run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,586 @@
+// Host side of libmonoffn: the C ABI declared in include/mono_ffn.h — plan
+// validation and allocation, the one-time weight repack, the per-step
+// launches and the device error word.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "mono_ffn.h"
+#include "mono_ffn_kernel.cuh"
+
+using namespace mono;
+
+namespace {
+
+thread_local std::string g_plan_error;
+
+struct LayerSlot {
+  float* mix_w = nullptr;
+  void* norm_w = nullptr;
+  float* router_t = nullptr;
+  float* bias = nullptr;
+  uint8_t* gu = nullptr;
+  uint8_t* dn = nullptr;
+  bool packed = false;
+  Taps taps{};
+};
+
+}  // namespace
+
+struct mono_ffn_plan_s {
+  mono_ffn_config cfg{};
+  int wt = 0;
+  int G = 0, nst = 0, slot_bytes = 0, regA_bytes = 0, ymax = 0, mix_ctas = 0, smem = 0;
+  int gu_kc = 0, gu_nk = 0, gu_rc = 0, dn_kc = 0, dn_nk = 0, dn_rc = 0;
+  long long gu_estride = 0, dn_estride = 0;
+  std::vector<LayerSlot> layers;
+  float* mix_part = nullptr;
+  float* logits = nullptr;
+  float* act = nullptr;
+  std::vector<float*> pend;
+  void* xbuf[2] = {nullptr, nullptr};
+  SyncBlock* sync = nullptr;
+  ErrBlock* err = nullptr;
+  void* stage_in = nullptr;
+  void* stage_out = nullptr;
+  int64_t packed_bytes = 0, scratch_bytes = 0;
+  int fault_cta = -1;
+  unsigned long long* trace = nullptr;
+  std::string last_error;
+};
+
+namespace {
+
+int elem_bits(int dt) { return dt == MONO_F32 ? 32 : dt == MONO_BF16 ? 16 : dt == MONO_FP8E4M3_B128 ? 8 : 4; }
+int block_of(int dt) { return dt == MONO_FP8E4M3_B128 ? 128 : dt == MONO_MXFP4 ? 32 : 0; }
+int unit_elems(int dt) { return 128 / elem_bits(dt); }   // elements per 16 bytes
+
+// largest chunk <= target that divides K and keeps whole 16-byte units and scale blocks
+int pick_kc(int dt, int K, int target) {
+  int step = std::max(unit_elems(dt), block_of(dt));
+  for (int kc = std::min(target, K) / step * step; kc >= step; kc -= step)
+    if (K % kc == 0) return kc;
+  return 0;
+}
+
+int code_bytes(int dt, int kc) { return (int)((long long)kc * elem_bits(dt) / 8); }
+int scale_bytes(int dt, int kc) {
+  if (dt == MONO_FP8E4M3_B128) return kc / 128 * 4;
+  if (dt == MONO_MXFP4) return kc / 32;
+  return 0;
+}
+int chunk_bytes(int dt, int kc) { return (int)align_up((size_t)code_bytes(dt, kc) + scale_bytes(dt, kc), 16); }
+
+int fail(mono_ffn_plan_t* p, int code, const std::string& msg) {
+  if (p) p->last_error = msg;
+  else g_plan_error = msg;
+  return code;
+}
+
+int cuda_fail(mono_ffn_plan_t* p, cudaError_t e, const char* what) {
+  return fail(p, MONO_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+template <int WT>
+void* kernel_ptr() {
+  return reinterpret_cast<void*>(&mono_ffn_layer_kernel<WT>);
+}
+
+void* kernel_for(int wt) {
+  switch (wt) {
+    case W_F32: return kernel_ptr<W_F32>();
+    case W_BF16: return kernel_ptr<W_BF16>();
+    case W_FP8: return kernel_ptr<W_FP8>();
+    default: return kernel_ptr<W_FP4>();
+  }
+}
+
+// ------------------------------------------------------------ pack kernels --
+
+// Cut every [rows][in] matrix row into nk chunks of kc elements, each chunk
+// followed by its block scales and padded to rc bytes; chunk (row, k) lands at
+// dst + (row * nk + k) * item + sub.
+__global__ void pack_rows_kernel(const uint8_t* codes, const uint8_t* scales, uint8_t* dst, long long rows,
+                                 int nk, int cb, int sb, int rc, int item, int sub, int vec) {
+  const long long nitems = rows * nk;
+  const int lane = threadIdx.x & 31;
+  long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (; w < nitems; w += nw) {
+    const long long row = w / nk;
+    const int k = (int)(w % nk);
+    const uint8_t* src = codes + row * (long long)cb * nk + (long long)k * cb;
+    uint8_t* d = dst + (row * nk + k) * (long long)item + sub;
+    if (vec) {
+      for (int i = lane; i < cb / 16; i += 32)
+        reinterpret_cast<uint4*>(d)[i] = reinterpret_cast<const uint4*>(src)[i];
+    } else {
+      for (int i = lane; i < cb; i += 32) d[i] = src[i];
+    }
+    if (sb) {
+      const uint8_t* ss = scales + row * (long long)sb * nk + (long long)k * sb;
+      for (int i = lane; i < sb; i += 32) d[cb + i] = ss[i];
+    }
+    for (int i = cb + sb + lane; i < rc; i += 32) d[i] = 0;
+  }
+}
+
+__global__ void transpose_f32_kernel(const float* src, float* dst, int rows, int cols) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int r = r0 + i, cc = c0 + threadIdx.x;
+    if (r < rows && cc < cols) tile[i][threadIdx.x] = src[(size_t)r * cols + cc];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int cc = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && cc < cols) dst[(size_t)cc * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+int pack_matrix(mono_ffn_plan_t* p, const void* codes, const void* scales, uint8_t* dst, long long rows, int in,
+                int kc, int nk, int rc, int item, int sub, cudaStream_t st) {
+  const int dt = p->cfg.expert_dtype;
+  const int cb = code_bytes(dt, kc), sb = scale_bytes(dt, kc);
+  if (sb && !scales) return fail(p, MONO_ERR_INVALID_ARG, "pack: block scales are required for this expert format");
+  (void)in;
+  const int vec = ((uintptr_t)codes % 16 == 0) && (cb % 16 == 0);
+  long long warps = rows * nk;
+  long long blocks = std::min<long long>((warps + 7) / 8, 148LL * 32);
+  pack_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>((const uint8_t*)codes, (const uint8_t*)scales, dst, rows, nk, cb,
+                                                     sb, rc, item, sub, vec);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? 0 : cuda_fail(p, e, "pack kernel launch");
+}
+
+template <typename T>
+int dalloc(mono_ffn_plan_t* p, T** ptr, size_t bytes, int64_t* acct) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc((void**)ptr, bytes);
+  if (e != cudaSuccess) return fail(p, MONO_ERR_OOM, std::string("cudaMalloc of ") + std::to_string(bytes) + " bytes: " +
+                                                         cudaGetErrorString(e));
+  *acct += (int64_t)bytes;
+  return 0;
+}
+
+}  // namespace
+
+// ================================================================ the C ABI
+
+extern "C" int mono_ffn_abi_version(void) { return 1; }
+
+extern "C" const char* mono_ffn_last_error(const mono_ffn_plan_t* plan) {
+  return plan ? plan->last_error.c_str() : g_plan_error.c_str();
+}
+
+extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
+  if (!p) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->cfg.device);
+  for (auto& l : p->layers) {
+    cudaFree(l.mix_w);
+    cudaFree(l.norm_w);
+    cudaFree(l.router_t);
+    cudaFree(l.bias);
+    cudaFree(l.gu);
+    cudaFree(l.dn);
+  }
+  for (float* q : p->pend) cudaFree(q);
+  cudaFree(p->mix_part);
+  cudaFree(p->logits);
+  cudaFree(p->act);
+  cudaFree(p->xbuf[0]);
+  cudaFree(p->xbuf[1]);
+  cudaFree(p->sync);
+  cudaFree(p->err);
+  cudaFree(p->stage_in);
+  cudaFree(p->stage_out);
+  cudaSetDevice(prev);
+  delete p;
+}
+
+extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** out) {
+  g_plan_error.clear();
+  if (!cfg_in || !out) return fail(nullptr, MONO_ERR_INVALID_ARG, "plan: NULL argument");
+  *out = nullptr;
+  mono_ffn_config cfg = *cfg_in;
+  if (cfg.wait_timeout_us == 0) cfg.wait_timeout_us = 250000;
+  std::string why;
+  auto need = [&](bool ok, const std::string& m) {
+    if (!ok) why += m + "\n";
+  };
+  const int dt = cfg.expert_dtype;
+  need(cfg.hc == kS, "hc must be 4");
+  need(cfg.hidden > 0 && cfg.inter > 0, "hidden and inter must be positive");
+  need(cfg.n_routed >= 1 && cfg.n_routed <= kMaxE, "n_routed must be in [1, 1024]");
+  need(cfg.top_k >= 1 && cfg.top_k <= std::min(cfg.n_routed, kMaxK), "top_k must be in [1, min(n_routed, 16)]");
+  need(cfg.max_rows >= 1 && cfg.max_rows <= kMaxR, "max_rows must be in [1, 8]");
+  need(cfg.n_layers >= 1, "n_layers must be >= 1");
+  need(cfg.hc_dtype == MONO_F32 || cfg.hc_dtype == MONO_BF16, "hc_dtype must be F32 or BF16");
+  need(cfg.norm_dtype == MONO_F32 || cfg.norm_dtype == MONO_BF16, "norm_dtype must be F32 or BF16");
+  need(dt >= MONO_F32 && dt <= MONO_MXFP4, "expert_dtype unknown");
+  need(!(cfg.hc_dtype == MONO_BF16 && !cfg.round_bf16), "bf16 residual streams need round_bf16 = 1");
+  need(cfg.sinkhorn_iters >= 0, "sinkhorn_iters must be >= 0");
+  if (dt >= MONO_F32 && dt <= MONO_MXFP4 && cfg.hidden > 0 && cfg.inter > 0) {
+    const int m = std::max(unit_elems(dt), block_of(dt));
+    need(cfg.hidden % m == 0, "hidden must be a multiple of " + std::to_string(m) + " for this expert format");
+    need(cfg.inter % m == 0, "inter must be a multiple of " + std::to_string(m) + " for this expert format");
+    need(cfg.hidden % 8 == 0 && cfg.inter % 8 == 0, "hidden and inter must be multiples of 8");
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) why += "no CUDA device\n";
+  else if (cfg.device < 0 || cfg.device >= ndev) why += "device ordinal out of range\n";
+  if (!why.empty()) return fail(nullptr, MONO_ERR_INVALID_ARG, why);
+
+  cudaDeviceProp prop{};
+  cudaGetDeviceProperties(&prop, cfg.device);
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(nullptr, MONO_ERR_UNSUPPORTED_ARCH,
+                "device " + std::to_string(cfg.device) + " is sm_" + std::to_string(prop.major) +
+                    std::to_string(prop.minor) + "; this library is built for sm_100a only");
+  if (!prop.cooperativeLaunch) return fail(nullptr, MONO_ERR_NOT_CORESIDENT, "device lacks cooperative launch");
+
+  mono_ffn_plan_t* p = new mono_ffn_plan_s();
+  p->cfg = cfg;
+  p->wt = dt;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(cfg.device);
+  const int H = cfg.hidden, I = cfg.inter, E = cfg.n_routed, K = cfg.top_k, RM = cfg.max_rows;
+
+  // chunking of the packed rows
+  const int gu_target = dt == MONO_F32 ? 256 : dt == MONO_BF16 ? 512 : 1024;
+  const int dn_target = dt == MONO_F32 ? 512 : dt == MONO_BF16 ? 1024 : 2048;
+  p->gu_kc = pick_kc(dt, H, gu_target);
+  p->dn_kc = pick_kc(dt, I, dn_target);
+  p->gu_nk = H / p->gu_kc;
+  p->dn_nk = I / p->dn_kc;
+  p->gu_rc = chunk_bytes(dt, p->gu_kc);
+  p->dn_rc = chunk_bytes(dt, p->dn_kc);
+  p->gu_estride = (long long)I * p->gu_nk * 2 * p->gu_rc;
+  p->dn_estride = (long long)H * p->dn_nk * p->dn_rc;
+  p->slot_bytes = (int)align_up((size_t)std::max(kCW * 2 * p->gu_rc, kCW * p->dn_rc), 128);
+
+  // grid and shared memory
+  // grid: one CTA per SM, a multiple of 4 (the mix partials are read as float4 per output)
+  p->G = cfg.grid > 0 ? std::min(cfg.grid, prop.multiProcessorCount) : prop.multiProcessorCount;
+  p->G = std::max(4, p->G / 4 * 4);
+  p->mix_ctas = p->G;
+  p->ymax = (H + p->G - 1) / p->G;
+  // region A holds, in turn: the mix_w and hc slices of A2, the mix partials,
+  // n [R][H], and the activation rows of the down projections (two halves
+  // of at least one row each, for the prefetch of the next expert)
+  size_t regA = std::max<size_t>((size_t)RM * H * (cfg.round_bf16 ? 2 : 4), (size_t)RM * I * 4);
+  regA = std::max<size_t>(regA, (size_t)2 * I * 4 + 256);
+  regA = std::max<size_t>(regA, ((size_t)kS * p->ymax * kMixC + (size_t)RM * kS * p->ymax) * 4);
+  regA = std::max<size_t>(regA, (size_t)p->G * kMixP * 4);
+  p->regA_bytes = (int)align_up(regA, 128);
+  const int smem_max = prop.sharedMemPerBlockOptin;
+  SmemLayout L0(0, p->slot_bytes, p->regA_bytes, p->ymax);
+  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16;
+  p->nst = (int)std::min<long long>(16, room / p->slot_bytes);
+  if (p->nst < 2) {
+    std::string m = "shared memory: " + std::to_string(smem_max) + " bytes leave room for " + std::to_string(p->nst) +
+                    " ring stages of " + std::to_string(p->slot_bytes) + " bytes (need 2)";
+    mono_ffn_destroy(p);
+    cudaSetDevice(prev);
+    return fail(nullptr, MONO_ERR_INVALID_ARG, m);
+  }
+  p->smem = (int)SmemLayout(p->nst, p->slot_bytes, p->regA_bytes, p->ymax).total;
+  void* kfn = kernel_for(dt);
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
+  int occ = 0;
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kfn, kThreads, p->smem);
+  if (e != cudaSuccess || occ < 1) {
+    std::string m = std::string("persistent grid cannot be co-resident: ") +
+                    (e != cudaSuccess ? cudaGetErrorString(e) : "occupancy 0");
+    mono_ffn_destroy(p);
+    cudaSetDevice(prev);
+    return fail(nullptr, MONO_ERR_NOT_CORESIDENT, m);
+  }
+
+  // storage
+  int rc = 0;
+  const size_t hc_elem = cfg.hc_dtype == MONO_BF16 ? 2 : 4;
+  const size_t norm_elem = cfg.norm_dtype == MONO_BF16 ? 2 : 4;
+  p->layers.resize(cfg.n_layers);
+  for (auto& l : p->layers) {
+    if (!rc) rc = dalloc(p, &l.mix_w, (size_t)kS * H * kMixC * 4, &p->packed_bytes);
+    if (!rc) rc = dalloc(p, &l.norm_w, (size_t)H * norm_elem, &p->packed_bytes);
+    if (!rc) rc = dalloc(p, &l.router_t, (size_t)E * H * 4, &p->packed_bytes);
+    if (!rc) rc = dalloc(p, &l.bias, (size_t)E * 4, &p->packed_bytes);
+    if (!rc) rc = dalloc(p, &l.gu, (size_t)(E + 1) * p->gu_estride, &p->packed_bytes);
+    if (!rc) rc = dalloc(p, &l.dn, (size_t)(E + 1) * p->dn_estride, &p->packed_bytes);
+  }
+  if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->act, (size_t)RM * (K + 1) * I * 4, &p->scratch_bytes);
+  p->pend.assign(cfg.n_layers, nullptr);
+  for (int l = 0; l + 1 < cfg.n_layers && !rc; ++l)
+    rc = dalloc(p, &p->pend[l], (size_t)RM * (kS + kS * kS + H) * 4, &p->scratch_bytes);
+  if (cfg.n_layers > 1) {
+    if (!rc) rc = dalloc(p, &p->xbuf[0], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
+    if (!rc) rc = dalloc(p, &p->xbuf[1], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
+  }
+  if (!rc) rc = dalloc(p, &p->sync, sizeof(SyncBlock) * cfg.n_layers, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->err, sizeof(ErrBlock), &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->stage_in, (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->stage_out, (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
+  if (!rc) {
+    cudaMemset(p->sync, 0, sizeof(SyncBlock) * cfg.n_layers);
+    cudaMemset(p->err, 0, sizeof(ErrBlock));
+    cudaMemset(p->act, 0, (size_t)RM * (K + 1) * I * 4);
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) rc = cuda_fail(p, e, "plan setup");
+  }
+  if (rc) {
+    std::string m = p->last_error;
+    mono_ffn_destroy(p);
+    cudaSetDevice(prev);
+    return fail(nullptr, rc, m);
+  }
+  cudaSetDevice(prev);
+  *out = p;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_ffn_layer_weights* w, void* stream) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "pack: NULL plan");
+  if (!w || layer < 0 || layer >= p->cfg.n_layers) return fail(p, MONO_ERR_INVALID_ARG, "pack: bad layer or weights");
+  std::string why;
+  if (!w->mix_w) why += "mix_w is NULL\n";
+  if (!w->norm_w) why += "norm_w is NULL\n";
+  if (!w->router_w) why += "router_w is NULL\n";
+  if (!w->router_bias) why += "router_bias is NULL\n";
+  if (!w->w_gate || !w->w_up || !w->w_down) why += "expert weights are NULL\n";
+  if (!why.empty()) return fail(p, MONO_ERR_INVALID_ARG, why);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->cfg.device);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int H = p->cfg.hidden, I = p->cfg.inter, E = p->cfg.n_routed;
+  LayerSlot& l = p->layers[layer];
+  const size_t norm_elem = p->cfg.norm_dtype == MONO_BF16 ? 2 : 4;
+  cudaMemcpyAsync(l.mix_w, w->mix_w, (size_t)kS * H * kMixC * 4, cudaMemcpyDeviceToDevice, st);
+  cudaMemcpyAsync(l.norm_w, w->norm_w, (size_t)H * norm_elem, cudaMemcpyDeviceToDevice, st);
+  cudaMemcpyAsync(l.bias, w->router_bias, (size_t)E * 4, cudaMemcpyDeviceToDevice, st);
+  transpose_f32_kernel<<<dim3((E + 31) / 32, (H + 31) / 32), dim3(32, 8), 0, st>>>(w->router_w, l.router_t, H, E);
+  int rc = 0;
+  // gate and up share an item: [gate chunk | up chunk]
+  rc = pack_matrix(p, w->w_gate, w->s_gate, l.gu, (long long)(E + 1) * I, H, p->gu_kc, p->gu_nk, p->gu_rc,
+                   2 * p->gu_rc, 0, st);
+  if (!rc)
+    rc = pack_matrix(p, w->w_up, w->s_up, l.gu, (long long)(E + 1) * I, H, p->gu_kc, p->gu_nk, p->gu_rc, 2 * p->gu_rc,
+                     p->gu_rc, st);
+  if (!rc)
+    rc = pack_matrix(p, w->w_down, w->s_down, l.dn, (long long)(E + 1) * H, I, p->dn_kc, p->dn_nk, p->dn_rc, p->dn_rc,
+                     0, st);
+  cudaError_t e = cudaGetLastError();
+  cudaSetDevice(prev);
+  if (rc) return rc;
+  if (e != cudaSuccess) return cuda_fail(p, e, "pack");
+  l.packed = true;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_set_taps(mono_ffn_plan_t* p, int layer, const mono_ffn_taps* t) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "set_taps: NULL plan");
+  if (layer < 0 || layer >= p->cfg.n_layers) return fail(p, MONO_ERR_INVALID_ARG, "set_taps: bad layer");
+  Taps& d = p->layers[layer].taps;
+  if (!t) {
+    d = Taps{};
+    return MONO_OK;
+  }
+  d.mix = t->mix;
+  d.pre = t->pre;
+  d.post = t->post;
+  d.comb = t->comb;
+  d.n = t->n;
+  d.logits = t->logits;
+  d.idx = t->idx;
+  d.w = t->w;
+  d.y = t->y;
+  d.x = t->x;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, void* hc_out, void* stream) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "step: NULL plan");
+  if (rows == 0) return MONO_OK;
+  if (rows < 0 || rows > p->cfg.max_rows)
+    return fail(p, MONO_ERR_INVALID_ARG, "step: rows " + std::to_string(rows) + " outside [0, max_rows = " +
+                                             std::to_string(p->cfg.max_rows) + "]");
+  if (!hc_in || !hc_out) return fail(p, MONO_ERR_INVALID_ARG, "step: NULL hc_in or hc_out");
+  const size_t hc_bytes = (size_t)rows * kS * p->cfg.hidden * (p->cfg.hc_dtype == MONO_BF16 ? 2 : 4);
+  {
+    const char* a = (const char*)hc_in;
+    const char* b = (const char*)hc_out;
+    if (a < b + hc_bytes && b < a + hc_bytes) return fail(p, MONO_ERR_INVALID_ARG, "step: hc_in and hc_out overlap");
+  }
+  for (int l = 0; l < p->cfg.n_layers; ++l)
+    if (!p->layers[l].packed)
+      return fail(p, MONO_ERR_NOT_PACKED, "step: layer " + std::to_string(l) + " has no packed weights");
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != p->cfg.device) cudaSetDevice(p->cfg.device);
+  const int L = p->cfg.n_layers;
+  void* kfn = kernel_for(p->wt);
+  cudaError_t e = cudaSuccess;
+  for (int l = 0; l < L && e == cudaSuccess; ++l) {
+    const LayerSlot& ls = p->layers[l];
+    Params prm{};
+    prm.H = p->cfg.hidden;
+    prm.I = p->cfg.inter;
+    prm.E = p->cfg.n_routed;
+    prm.K = p->cfg.top_k;
+    prm.R = rows;
+    prm.G = p->G;
+    prm.layer = l;
+    prm.first = l == 0;
+    prm.last = l == L - 1;
+    prm.mix_ctas = p->mix_ctas;
+    prm.hc_bf16 = p->cfg.hc_dtype == MONO_BF16;
+    prm.norm_bf16 = p->cfg.norm_dtype == MONO_BF16;
+    prm.round_bf16 = p->cfg.round_bf16 != 0;
+    prm.rms_eps = p->cfg.rms_eps;
+    prm.pre_eps = p->cfg.pre_eps;
+    prm.post_mult = p->cfg.post_mult;
+    prm.route_scale = p->cfg.route_scale;
+    prm.denom_clamp = p->cfg.denom_clamp;
+    prm.sink_iters = p->cfg.sinkhorn_iters;
+    prm.x_prev = l <= 1 ? hc_in : p->xbuf[(l - 1) % 2];
+    prm.xbuf = l == 0 ? nullptr : p->xbuf[l % 2];
+    prm.hc_out = hc_out;
+    prm.pend_in = l > 0 ? p->pend[l - 1] : nullptr;
+    prm.pend_out = l + 1 < L ? p->pend[l] : nullptr;
+    prm.mix_w = ls.mix_w;
+    prm.norm_w = ls.norm_w;
+    prm.router_t = ls.router_t;
+    prm.bias = ls.bias;
+    prm.gu = ls.gu;
+    prm.dn = ls.dn;
+    prm.gu_kc = p->gu_kc;
+    prm.gu_nk = p->gu_nk;
+    prm.gu_rc = p->gu_rc;
+    prm.dn_kc = p->dn_kc;
+    prm.dn_nk = p->dn_nk;
+    prm.dn_rc = p->dn_rc;
+    prm.gu_estride = p->gu_estride;
+    prm.dn_estride = p->dn_estride;
+    prm.mix_part = p->mix_part;
+    prm.logits = p->logits;
+    prm.act = p->act;
+    prm.sync = p->sync + l;
+    prm.err = p->err;
+    prm.taps = ls.taps;
+    prm.nst = p->nst;
+    prm.slot_bytes = p->slot_bytes;
+    prm.regA_bytes = p->regA_bytes;
+    prm.ymax = p->ymax;
+    prm.timeout_ns = (unsigned long long)p->cfg.wait_timeout_us * 1000ull;
+    prm.fault_cta = p->fault_cta;
+    prm.trace = p->trace ? p->trace + (size_t)l * p->G * kTracePoints : nullptr;
+
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(p->G);
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = p->smem;
+    lc.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    void* args[] = {&prm};
+    e = cudaLaunchKernelExC(&lc, kfn, args);
+  }
+  if (prev != p->cfg.device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(p, e, "step launch");
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_step_host(mono_ffn_plan_t* p, int rows, const void* hc_in_host, void* hc_out_host,
+                                  void* stream) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "step_host: NULL plan");
+  if (rows == 0) return MONO_OK;
+  if (rows < 0 || rows > p->cfg.max_rows) return fail(p, MONO_ERR_INVALID_ARG, "step_host: rows out of range");
+  if (!hc_in_host || !hc_out_host) return fail(p, MONO_ERR_INVALID_ARG, "step_host: NULL buffer");
+  const size_t bytes = (size_t)rows * kS * p->cfg.hidden * (p->cfg.hc_dtype == MONO_BF16 ? 2 : 4);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->cfg.device);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(p->stage_in, hc_in_host, bytes, cudaMemcpyHostToDevice, st);
+  int rc = e == cudaSuccess ? mono_ffn_step(p, rows, p->stage_in, p->stage_out, stream) : cuda_fail(p, e, "H2D");
+  if (!rc) {
+    e = cudaMemcpyAsync(hc_out_host, p->stage_out, bytes, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) rc = cuda_fail(p, e, "D2H");
+  }
+  cudaSetDevice(prev);
+  return rc;
+}
+
+extern "C" int mono_ffn_query_error(mono_ffn_plan_t* p, mono_ffn_status* st) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "query_error: NULL plan");
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->cfg.device);
+  ErrBlock eb{};
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&eb, p->err, sizeof(eb), cudaMemcpyDeviceToHost);
+  int rc = MONO_OK;
+  if (e != cudaSuccess) {
+    rc = cuda_fail(p, e, "query_error");
+  } else if (eb.code || eb.abort) {
+    rc = eb.code == 7u ? MONO_ERR_DEVICE_TIMEOUT : MONO_ERR_DEVICE_ABORTED;
+    p->last_error = "device wait failed: stage " + std::to_string(eb.stage) + ", cta " + std::to_string(eb.cta) +
+                    ", layer " + std::to_string(eb.layer);
+    // reset the sync state so the next step starts clean
+    cudaMemset(p->sync, 0, sizeof(SyncBlock) * p->cfg.n_layers);
+    cudaMemset(p->err, 0, sizeof(ErrBlock));
+    cudaDeviceSynchronize();
+  }
+  if (st) {
+    st->code = rc == MONO_ERR_DEVICE_TIMEOUT || rc == MONO_ERR_DEVICE_ABORTED ? rc : 0;
+    st->stage = (int)eb.stage;
+    st->cta = (int)eb.cta;
+    st->layer = (int)eb.layer;
+  }
+  cudaSetDevice(prev);
+  return rc;
+}
+
+extern "C" int mono_ffn_get_info(const mono_ffn_plan_t* p, mono_ffn_info* info) {
+  if (!p || !info) return MONO_ERR_INVALID_ARG;
+  const int H = p->cfg.hidden, E = p->cfg.n_routed;
+  info->grid = p->G;
+  info->threads = kThreads;
+  info->smem_bytes = p->smem;
+  info->ring_stages = p->nst;
+  info->ring_slot_bytes = p->slot_bytes;
+  info->expert_bytes = p->gu_estride + p->dn_estride;
+  info->dense_bytes = (int64_t)kS * H * kMixC * 4 + (int64_t)E * H * 4 + (int64_t)E * 4 +
+                      (int64_t)H * (p->cfg.norm_dtype == MONO_BF16 ? 2 : 4);
+  info->packed_bytes = p->packed_bytes;
+  info->scratch_bytes = p->scratch_bytes;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_set_trace(mono_ffn_plan_t* p, unsigned long long* buf) {
+  if (!p) return MONO_ERR_INVALID_ARG;
+  p->trace = buf;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* p, int cta) {
+  if (!p) return MONO_ERR_INVALID_ARG;
+  p->fault_cta = cta;
+  return MONO_OK;
+}

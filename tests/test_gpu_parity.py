@@ -1,0 +1,186 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same
+seeded inputs, at sizes the oracle finishes in seconds: several weight-ring
+tiles per CTA, a ragged tail of items, every rows count 1..8, the all-zero
+tie rounds, FP8 and MXFP4 experts, and a 4-layer chain."""
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from synth import configs as C
+from synth import synth as S
+from tests.gpu_harness import GpuRun, compare_out, oracle_rows, raw_hc, routing_ok, select_weights
+from tests.oracle_helpers import all_experts
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    import __graft_entry__
+    __graft_entry__.build()
+
+
+def _check_layer(wl, run, rows, layer=0, hc_in=None, dense=None):
+    """Compare every tap and the output of `rows` with the oracle."""
+    want, t = oracle_rows(wl, rows, layer=layer, hc_in=hc_in, dense=dense)
+    got = run.out_host()[rows]
+    idx = run.tap(layer, "idx")[rows]
+    exempt = []
+    for i in range(len(rows)):
+        ok, ex = routing_ok(idx[i], t.idx[i], t.sel[i], wl.top_k)
+        assert ok, f"row {rows[i]}: gpu {idx[i]} oracle {t.idx[i]}"
+        if ex:
+            exempt.append(i)
+    keep = [i for i in range(len(rows)) if i not in exempt]
+    tol_mix = 1e-4
+    assert np.allclose(run.tap(layer, "mix")[rows], t.mix, rtol=tol_mix, atol=tol_mix)
+    assert np.allclose(run.tap(layer, "pre")[rows], t.pre, rtol=1e-5, atol=1e-6)
+    assert np.allclose(run.tap(layer, "comb")[rows], t.comb.reshape(len(rows), 16), rtol=1e-4, atol=1e-5)
+    # the router matvec, checked on the kernel's own n (a bf16 rounding flip in
+    # n moves a logit by ~1e-4, so n itself is compared with the bf16 tolerance)
+    d = S.cpu_dense(wl, layer) if dense is None else dense
+    n_gpu = run.tap(layer, "n")[rows].astype(np.float64)
+    lg_want = n_gpu @ d["router_w"].astype(np.float64)
+    assert np.allclose(run.tap(layer, "logits")[rows], lg_want, rtol=1e-4, atol=1e-5)
+    # the select math on the kernel's own logits and selection, then the
+    # weights against the oracle's (which see the oracle's n)
+    w = run.tap(layer, "w")[rows]
+    w_own = select_weights(wl, run.tap(layer, "logits")[rows], idx, None)
+    assert np.allclose(w, w_own, rtol=2e-6, atol=1e-7)
+    wtol = 1e-5 if not wl.round_bf16 else 1e-3
+    assert np.allclose(w[keep], t.w[keep], rtol=wtol, atol=wtol * 1e-1)
+    if keep:
+        compare_out(wl, run.tap(layer, "n")[rows][keep], t.n[keep], "n")
+        compare_out(wl, run.tap(layer, "y")[rows][keep], t.y[keep], "y")
+        if wl.n_layers == 1:
+            compare_out(wl, got[keep], want[keep], "hc_out")
+    return t
+
+
+def test_tiny_fp32_all_rows():
+    wl = C.TINY_FP32
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, [0])
+    run.close()
+
+
+@pytest.mark.parametrize("rows", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_tiny_fp32_rows_sweep(rows):
+    wl = C.TINY_FP32.with_(rows=rows, seed=100 + rows)
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(rows)))
+    run.close()
+
+
+def test_rows_zero_is_noop_and_rows_above_max_refused():
+    import torch
+
+    from moe_decode_layer_sm_b200 import MonoError
+    wl = C.TINY_FP32.with_(rows=2)
+    run = GpuRun(wl)
+    run.out.fill_(7.0)
+    run.plan.step(0, run.hc, run.out)
+    torch.cuda.synchronize()
+    assert bool((run.out == 7.0).all())
+    with pytest.raises(MonoError):
+        run.plan.step(3, run.hc, run.out)
+    run.close()
+
+
+@pytest.mark.parametrize("bias", ["zero", "four-levels"])
+def test_zero_input_tie_rounds(bias):
+    import torch
+    wl = C.TINY_FP32.with_(rows=2)
+    d = S.cpu_dense(wl, 0)
+    if bias == "zero":
+        b = np.zeros_like(d["router_bias"])
+    else:
+        levels = np.array([-0.075, -0.025, 0.025, 0.075], np.float32)
+        b = levels[np.minimum(3, np.floor((d["router_bias"] + 0.1) / 0.05).astype(int))]
+    hc = torch.zeros((2, 4, wl.hidden), dtype=torch.float32, device="cuda")
+    run = GpuRun(wl, dense_override=lambda l: {"router_bias": b}, hc_in=hc)
+    run.step()
+    d["router_bias"] = b
+    t = _check_layer(wl, run, [0, 1], hc_in=np.zeros((2, 4, wl.hidden), np.float32), dense=d)
+    order = sorted(range(wl.n_routed), key=lambda e: (-b[e], e))
+    assert run.tap(0, "idx").tolist() == [order[:wl.top_k]] * 2 == t.idx.tolist()
+    assert np.all(run.out_host() == 0.0)
+    run.close()
+
+
+@pytest.mark.parametrize("rows", [1, 3, 8])
+def test_scaled_bf16(rows):
+    wl = C.scaled(C.FLASH_BF16_R8, rows=rows, seed=200 + rows)
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(rows)))
+    # a second step on the same plan (epoch-tagged counters, no reset) gives the same bytes
+    first = run.out_host().copy()
+    run.step()
+    assert np.array_equal(first, run.out_host())
+    run.close()
+
+
+def test_scaled_fp8_rows4():
+    wl = C.scaled(C.FLASH_FP8_R4, seed=301)
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
+def test_scaled_mxfp4_single_layer():
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=401)
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
+@pytest.mark.parametrize("wdt", ["bf16", "mxfp4"])
+def test_scaled_chain_four_layers(wdt):
+    """Each layer of the chain checked on the residual streams the kernel
+    materialised for it (x tap): routing exact (near-tie exemption), y and the
+    next layer's streams within tolerance, and the final output.  Then the
+    whole chain against the oracle's own chain."""
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, w_dtype=wdt, seed=402)
+    run = GpuRun(wl)
+    got = run.step()
+    lws = [O.LayerWeights(wl, S.cpu_dense(wl, l), all_experts(wl, l)) for l in range(wl.n_layers)]
+    assert np.array_equal(run.tap(0, "x"), O.decode_hc(wl, S.cpu_hc_in(wl)))
+    for l, lw in enumerate(lws):
+        x_gpu = raw_hc(wl, run.tap(l, "x"))
+        out, t = O.layer(wl, lw, x_gpu)
+        keep = []
+        for r in range(wl.rows):
+            ok, ex = routing_ok(run.tap(l, "idx")[r], t.idx[r], t.sel[r], wl.top_k)
+            assert ok, f"layer {l} row {r}: gpu {run.tap(l, 'idx')[r]} oracle {t.idx[r]}"
+            if not ex:
+                keep.append(r)
+        compare_out(wl, run.tap(l, "y")[keep], t.y[keep], f"layer {l} y")
+        nxt = run.tap(l + 1, "x") if l + 1 < wl.n_layers else got
+        compare_out(wl, nxt[keep], O.decode_hc(wl, out)[keep], f"layer {l} expand")
+    # the whole chain against the oracle's chain: rows whose routing never
+    # met a near tie along the way
+    want = O.decode_hc(wl, O.chain(wl, lws, S.cpu_hc_in(wl), deferred=True))
+    compare_out(wl, got, want, "chain hc_out", allow_rows_off=2)
+    run.close()
+
+
+def test_device_timeout_is_reported_and_recovers():
+    """A CTA withholds its router-logits arrival: every other CTA's bounded
+    wait expires, the step reports DEVICE_TIMEOUT, and the next step on the
+    same plan is correct again."""
+    wl = C.TINY_FP32.with_(rows=1)
+    run = GpuRun(wl, wait_timeout_us=20000)
+    run.plan.debug_skip_arrival(3)
+    run.plan.step(1, run.hc, run.out)
+    rc, st = run.plan.query_error()
+    assert rc == -7 and st.stage == 2   # the root cause: the router-logits counter
+    run.plan.debug_skip_arrival(-1)
+    run.step()
+    _check_layer(wl, run, [0])
+    run.close()

@@ -56,9 +56,10 @@ def test_device_build_writes_host_bytes(wdt):
         host = S.cpu_expert(wl, 1, slot)
         for nm in ("gate", "up", "down"):
             q, s = dev[nm]
-            qh = q[slot].cpu().numpy()
-            if qh.dtype != host[nm][0].dtype:
-                qh = qh.view(host[nm][0].dtype) if wdt != "bf16" else q[slot].view(torch.int16).cpu().numpy().view(np.uint16)
+            if wdt == "bf16":
+                qh = q[slot].view(torch.int16).cpu().numpy().view(np.uint16)
+            else:
+                qh = q[slot].cpu().numpy().view(host[nm][0].dtype)
             assert np.array_equal(qh, host[nm][0])
             if s is not None:
                 assert np.array_equal(s[slot].cpu().numpy(), host[nm][1])
