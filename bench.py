@@ -27,7 +27,8 @@ METRIC = "µs per fused MoE layer-step and achieved HBM GB/s (% of peak), rows=1
 UNIT = "us/layer-step"
 FLUSH_BYTES = 512 << 20
 N_INPUT_SETS = 4
-KERNEL_SOURCES = ["moe_decode_layer_sm_b200/csrc/mono_ffn.cu", "moe_decode_layer_sm_b200/csrc/mono_ffn_kernel.cuh",
+KERNEL_SOURCES = ["moe_decode_layer_sm_b200/csrc/mono_ffn.cu", "moe_decode_layer_sm_b200/csrc/common.cuh",
+                  "moe_decode_layer_sm_b200/csrc/cc_kernel.cuh", "moe_decode_layer_sm_b200/csrc/tc_kernel.cuh",
                   "moe_decode_layer_sm_b200/csrc/ptx.cuh"]
 
 

@@ -7,7 +7,8 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "mono_ffn.cu")
-DEPS = [SRC, os.path.join(PKG, "csrc", "mono_ffn_kernel.cuh"), os.path.join(PKG, "csrc", "ptx.cuh"),
+DEPS = [SRC, os.path.join(PKG, "csrc", "common.cuh"), os.path.join(PKG, "csrc", "cc_kernel.cuh"),
+        os.path.join(PKG, "csrc", "tc_kernel.cuh"), os.path.join(PKG, "csrc", "ptx.cuh"),
         os.path.join(ROOT, "include", "mono_ffn.h")]
 SO = os.path.join(PKG, "libmonoffn.so")
 

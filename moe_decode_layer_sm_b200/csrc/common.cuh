@@ -1,0 +1,845 @@
+// Device code shared by the two persistent "mono" kernels (one launch runs the
+// whole FFN half-layer): constants, the per-CTA control block, bounded waits,
+// the prologue (hyper-connection mix, collapse + weighted RMSNorm, router
+// logits, top-k and work lists) and the tail (routed + shared sum, expand).
+//
+// Warp roles inside a CTA (384 threads, both kernels):
+//   warps 0-7    compute: prologue, then the expert phase of the kernel, tail
+//   warp  8      producer: 1-D TMA bulk copies of packed weight chunks into
+//                the shared-memory ring (mbarrier complete_tx)
+//   warp  9      tensor-core issuer (tcgen05.mma) in the tensor-core kernel
+//   warps 10-11  control: Sinkhorn, the canonical top-k, the expert lists
+//
+// Grid-wide dependencies are epoch-tagged counters in global memory (no reset
+// between steps): a CTA publishes with a release-add and waits with acquire
+// loads until the counter reaches (epoch + 1) * contributors.  Every wait is
+// bounded by the plan's timeout; on expiry the CTA records an error word,
+// raises the abort flag and runs the rest of its control flow without waiting
+// (so every named barrier is still reached), then returns.
+#pragma once
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace mono {
+
+constexpr int kS = 4;         // hyper-connection streams
+constexpr int kMixC = 24;     // 2S + S*S
+constexpr int kMixP = 25;     // mix columns + the square sum
+constexpr int kMaxR = 8;
+constexpr int kMaxK = 16;
+constexpr int kMaxU = kMaxR * kMaxK;
+constexpr int kMaxE = 1024;
+constexpr int kCW = 8;        // compute warps (also the items of a CUDA-core ring stage)
+constexpr int kProdWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kCtlWarp0 = 10;
+constexpr int kCtlWarps = 2;
+constexpr int kThreads = 12 * 32;                      // 384: 12 warps leave 168 registers a thread
+constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
+// named barriers: prologue (compute + control), compute, control, epilogue
+// warps 0-3, builder warps 4-7, end (epilogue warps + the issuer warp)
+constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarBld = 5, kBarEnd = 6;
+constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
+
+enum WType { W_F32 = 0, W_BF16 = 1, W_FP8 = 2, W_FP4 = 3 };
+
+struct SyncBlock {   // one per layer slot, 64 bytes
+  uint32_t epoch, cnt_mix, cnt_logit, cnt_act, cnt_done, cnt_y, pad[10];
+};
+struct ErrBlock {
+  uint32_t abort, code, stage, cta, layer, pad[11];
+};
+
+struct Taps {
+  float *mix, *pre, *post, *comb, *n, *logits;
+  int* idx;
+  float *w, *y, *x;
+};
+
+struct Params {
+  int H, I, E, K, R, G;
+  int layer, first, last;
+  int mix_ctas;
+  int hc_bf16, norm_bf16, round_bf16;
+  float rms_eps, pre_eps, post_mult, route_scale, denom_clamp;
+  int sink_iters;
+  // residual streams
+  const void* x_prev;   // first: this layer's X (hc_in); else the previous layer's X
+  void* xbuf;           // this layer's X when not first (written by the mix CTAs)
+  void* hc_out;         // written when last
+  const float* pend_in; // previous layer's pending post [R][4] | comb [R][16] | y [R][H]
+  float* pend_out;      // this layer's pending state (when not last)
+  // packed weights
+  const float* mix_w;
+  const void* norm_w;
+  const float* router_t;   // [E][H]
+  const float* bias;
+  // CUDA-core kernel: gu [E+1][I][gu_nk][gate|up][gu_rc], dn [E+1][H][dn_nk][dn_rc]
+  //   (row chunks of kc elements with their block scales);
+  // tensor-core kernel: gu [E+1][I/128][H/8][16][gate|up][8][8],
+  //   dn [E+1][H/128][I/8][16][8][8] (blocks of 128 output rows made of bf16
+  //   core matrices of 8 rows x 8 contraction elements)
+  const uint8_t* gu;
+  const uint8_t* dn;
+  int gu_kc, gu_nk, gu_rc;
+  int dn_kc, dn_nk, dn_rc;
+  long long gu_estride, dn_estride;
+  // scratch
+  float* mix_part;   // [R*25][G] output-major partials of the mix
+  float* logits;     // [R][E]
+  float* act;        // [R][K+1][I]
+  float* yp;         // tensor-core kernel: [R][K+1][H] weighted expert outputs
+  float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks
+  float* dpart;      // tensor-core kernel: [G][2][128][16] partial down tiles
+  uint32_t* gcnt;    // tensor-core kernel: [R*K+2][I/128] arrivals per split gate/up block (0 between launches)
+  uint32_t* dcnt;    // tensor-core kernel: [R*K+2][H/128] arrivals per split down block
+  SyncBlock* sync;
+  ErrBlock* err;
+  Taps taps;
+  int nst, slot_bytes, regA_bytes, ymax;
+  unsigned long long timeout_ns;
+  int fault_cta;
+  unsigned long long* trace;   // optional [G][kTracePoints] globaltimer stamps
+};
+
+constexpr int kTracePoints = 16;
+// stage timestamps (one writer per point and CTA)
+__device__ __forceinline__ void trace(const Params& p, int point, bool who = true) {
+  if (p.trace && who) p.trace[blockIdx.x * kTracePoints + point] = globaltimer();
+}
+
+// per-CTA control block in shared memory
+struct Ctl {
+  volatile int dead;
+  volatile int lists_ready;
+  uint32_t epoch;
+  volatile int nu;              // unique routed experts (control warps' copy)
+  int nu_comp;                  // the compute warps' agreed copy
+  float smix[kMaxR][kMixP];     // mix partial totals, then the scaled mix
+  float pre[kMaxR][kS], post[kMaxR][kS], comb[kMaxR][kS * kS];
+  float inv[kMaxR];
+  float sq[kCW][kMaxR];
+  float sq2[kCW][kMaxR];
+  uint32_t bm[kMaxE / 32];      // selected-expert bitmap
+  int nu_ctl;
+  int idx[kMaxR][kMaxK];
+  float wt[kMaxR][kMaxK];
+  int ulist[kMaxU];
+  uint32_t umask[kMaxU];
+  signed char uslot[kMaxU][kMaxR];
+  float red[kPreThreads * 2];
+  // tensor-core kernel
+  uint32_t tmem_base;
+  volatile int n_ready;         // n is in shared memory (B operand of gate/up)
+  volatile int bld_seq;         // activation B operands built so far
+  volatile int mma_seq;         // activation B operands released by the issuer
+  uint64_t accfull[2], accempty[2], drain;
+  volatile int bcast;           // epilogue: "this CTA completes the block"
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// dynamic shared memory layout
+struct SmemLayout {
+  size_t bars, ctl, ys, regA, ring, total;
+  __host__ __device__ SmemLayout(int nst, int slot_bytes, int regA_bytes, int ymax) {
+    bars = 0;
+    ctl = align_up(bars + 2 * 8 * (size_t)nst, 128);
+    ys = align_up(ctl + sizeof(Ctl), 128);
+    regA = align_up(ys + sizeof(float) * kMaxR * (size_t)ymax, 128);
+    ring = align_up(regA + (size_t)regA_bytes, 1024);
+    total = ring + (size_t)nst * slot_bytes + kRingGuard;
+  }
+};
+
+// ------------------------------------------------------------ bounded waits --
+
+__device__ __forceinline__ void record_error(const Params& p, Ctl* c, uint32_t code, uint32_t stage) {
+  if (atomicCAS(&p.err->code, 0u, code) == 0u) {
+    p.err->stage = stage;
+    p.err->cta = blockIdx.x;
+    p.err->layer = p.layer;
+  }
+  atomicExch(&p.err->abort, 1u);
+  c->dead = 1;
+}
+
+// wait until *cnt >= target (wrap-safe); false when dead or timed out
+__device__ bool wait_count(const Params& p, Ctl* c, const uint32_t* cnt, uint32_t target, uint32_t stage) {
+  volatile int* dead = &c->dead;
+  uint64_t t0 = globaltimer();
+  uint32_t ns = 32;
+  while (true) {
+    if (*dead) return false;
+    uint32_t v = ld_acquire(cnt);
+    if ((int32_t)(v - target) >= 0) return true;
+    if (ld_relaxed(&p.err->abort)) {
+      c->dead = 1;
+      return false;
+    }
+    if (globaltimer() - t0 > p.timeout_ns) {
+      record_error(p, c, 7u, stage);   // MONO_ERR_DEVICE_TIMEOUT (negated on the host)
+      return false;
+    }
+    __nanosleep(ns);
+    if (ns < 256) ns <<= 1;
+  }
+}
+
+__device__ bool wait_bar(const Params& p, Ctl* c, uint64_t* bar, uint32_t parity) {
+  volatile int* dead = &c->dead;
+  if (mbar_test(bar, parity)) return true;
+  uint64_t t0 = globaltimer();
+  while (true) {
+    if (*dead) return false;
+    if (mbar_test(bar, parity)) return true;
+    if (globaltimer() - t0 > 2 * p.timeout_ns) {   // downstream of the grid-wide waits
+      record_error(p, c, 7u, 5u);
+      return false;
+    }
+    __nanosleep(20);
+  }
+}
+
+__device__ bool wait_flag(const Params& p, Ctl* c, volatile int* flag) {
+  volatile int* dead = &c->dead;
+  uint64_t t0 = globaltimer();
+  while (true) {
+    if (*flag) return true;
+    if (*dead) return false;
+    if (globaltimer() - t0 > 2 * p.timeout_ns) {   // downstream of the grid-wide waits
+      record_error(p, c, 7u, 3u);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+// --------------------------------------------------------------- helpers --
+
+__device__ __forceinline__ float load_x(const void* base, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+__device__ __forceinline__ float load_x_cg(const void* base, size_t i, int bf16) {
+  if (bf16) {
+    unsigned short b = __ldcg(reinterpret_cast<const unsigned short*>(base) + i);
+    return __uint_as_float((uint32_t)b << 16);
+  }
+  return __ldcg(reinterpret_cast<const float*>(base) + i);
+}
+__device__ __forceinline__ void store_x(void* base, size_t i, float v, int bf16) {
+  if (bf16) reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(base)[i] = v;
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// ordered key of a float for a max-reduction (larger float -> larger key)
+__device__ __forceinline__ uint32_t ord_key(float x) {
+  x = x + 0.0f;   // -0 -> +0
+  uint32_t b = __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+template <int WT> struct WFmt;
+template <> struct WFmt<W_F32> { static constexpr int EPU = 4; };
+template <> struct WFmt<W_BF16> { static constexpr int EPU = 8; };
+template <> struct WFmt<W_FP8> { static constexpr int EPU = 16; };
+template <> struct WFmt<W_FP4> { static constexpr int EPU = 32; };
+
+// scale of weight unit u (16 bytes) of a row chunk that holds kc elements
+template <int WT>
+__device__ __forceinline__ float unit_scale(const uint8_t* chunk, int kc, int u) {
+  if (WT == W_FP8) return reinterpret_cast<const float*>(chunk + kc)[u >> 3];       // 8 units per 128
+  if (WT == W_FP4) {
+    uint32_t e = chunk[kc / 2 + u];
+    return e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);             // 2^(e-127)
+  }
+  return 1.0f;
+}
+
+// load NE activation values (elements k .. k+NE-1) of a row as floats
+template <int NE, bool BF>
+__device__ __forceinline__ void load_vec(const void* row, int k, float* f) {
+  if (BF) {
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(row) + k;
+    if (NE % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < NE / 8; ++i) {
+        uint4 v = reinterpret_cast<const uint4*>(src)[i];
+        f[8 * i + 0] = bf16lo(v.x); f[8 * i + 1] = bf16hi(v.x);
+        f[8 * i + 2] = bf16lo(v.y); f[8 * i + 3] = bf16hi(v.y);
+        f[8 * i + 4] = bf16lo(v.z); f[8 * i + 5] = bf16hi(v.z);
+        f[8 * i + 6] = bf16lo(v.w); f[8 * i + 7] = bf16hi(v.w);
+      }
+    } else if (NE % 2 == 0) {
+#pragma unroll
+      for (int i = 0; i < NE / 2; ++i) {
+        uint32_t v = reinterpret_cast<const uint32_t*>(src)[i];
+        f[2 * i] = bf16lo(v);
+        f[2 * i + 1] = bf16hi(v);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NE; ++i) f[i] = __uint_as_float((uint32_t)src[i] << 16);
+    }
+  } else {
+    const float* src = reinterpret_cast<const float*>(row) + k;
+    if (NE % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < NE / 4; ++i) {
+        float4 v = reinterpret_cast<const float4*>(src)[i];
+        f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+      }
+    } else if (NE % 2 == 0) {
+#pragma unroll
+      for (int i = 0; i < NE / 2; ++i) {
+        float2 v = reinterpret_cast<const float2*>(src)[i];
+        f[2 * i] = v.x; f[2 * i + 1] = v.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NE; ++i) f[i] = src[i];
+    }
+  }
+}
+
+// 16-byte units in the code part of a row chunk of kc elements
+template <int WT> __device__ __forceinline__ int units_of(int kc) {
+  return WT == W_F32 ? kc / 4 : WT == W_BF16 ? kc / 8 : WT == W_FP8 ? kc / 16 : kc / 32;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// 8 consecutive activation values (bf16 or fp32 storage) at element i
+__device__ __forceinline__ void load_hc8(const void* base, size_t i, int bf16, float* f) {
+  if (bf16) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + i));
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+  } else {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i) + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+// 8 values to shared memory: bf16 (exact for values already rounded) or fp32
+__device__ __forceinline__ void store8(uint8_t* base, size_t i, bool bf, const float* f) {
+  if (bf) {
+    uint4 v;
+    v.x = pack_bf16x2(f[0], f[1]); v.y = pack_bf16x2(f[2], f[3]);
+    v.z = pack_bf16x2(f[4], f[5]); v.w = pack_bf16x2(f[6], f[7]);
+    reinterpret_cast<uint4*>(base + i * 2)[0] = v;
+  } else {
+    reinterpret_cast<float4*>(base + i * 4)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(base + i * 4)[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+__device__ __forceinline__ void load8(const uint8_t* base, size_t i, bool bf, float* f) {
+  if (bf) {
+    const uint4 v = reinterpret_cast<const uint4*>(base + i * 2)[0];
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+  } else {
+    const float4 a = reinterpret_cast<const float4*>(base + i * 4)[0];
+    const float4 b = reinterpret_cast<const float4*>(base + i * 4)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+}
+
+// Router select of one row by one warp: score = sqrt(softplus(logit)) in
+// fp32, sel = score + bias, canonical top-k by (sel desc, index asc) through
+// warp max / min reductions, then weight = score / max(sum, clamp) * scale
+// with each op rounded to fp32.  Lane l holds experts l + 32 q, q < NQ.
+template <int NQ>
+__device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
+  const int lane = threadIdx.x & 31;
+  const int E = p.E, K = p.K;
+  float score[NQ];
+  uint32_t key[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = lane + 32 * q;
+    score[q] = 0.f;
+    key[q] = 0u;
+    if (e < E) {
+      const float lg = c->dead ? 0.f : __ldcg(p.logits + (size_t)r * E + e);
+      if (blockIdx.x == 0 && p.taps.logits) p.taps.logits[(size_t)r * E + e] = lg;
+      const float sp = fmaxf(lg, 0.f) + log1pf(expf(-fabsf(lg)));
+      score[q] = sqrtf(sp);
+      key[q] = ord_key(score[q] + __ldg(p.bias + e));
+    }
+  }
+  uint32_t taken = 0u;
+  float ssum = 0.f;
+  for (int j = 0; j < K; ++j) {
+    uint32_t bk = 0u;
+    int be = 0x7FFFFFFF;
+    float bs = 0.f;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      if (!((taken >> q) & 1u) && key[q] > bk) {
+        bk = key[q];
+        be = lane + 32 * q;
+        bs = score[q];
+      }
+    }
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+    const int we = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(bk == wk ? be : 0x7FFFFFFF));
+    const int wl = we & 31;
+    if (we < E && wl == lane) taken |= 1u << (we >> 5);
+    const float ws = __shfl_sync(0xffffffffu, bs, wl);
+    if (lane == 0) {
+      c->idx[r][j] = we < E ? we : 0;
+      c->wt[r][j] = ws;   // the raw score until the sum is known
+    }
+    ssum += ws;   // selection order, fp32
+  }
+  __syncwarp();
+  if (lane < K) {
+    const float den = fmaxf(ssum, p.denom_clamp);
+    const float w = __fmul_rn(__fdiv_rn(c->wt[r][lane], den), p.route_scale);
+    c->wt[r][lane] = w;
+    if (blockIdx.x == 0) {
+      if (p.taps.idx) p.taps.idx[r * K + lane] = c->idx[r][lane];
+      if (p.taps.w) p.taps.w[r * K + lane] = w;
+    }
+  }
+  __syncwarp();
+}
+
+// ------------------------------------------------------------ work walkers --
+
+// The stage sequence of one CTA.  Producer and consumers run the same walker;
+// a stage is (phase, expert slot, first item, items, chunk index).
+enum Phase { PH_SGU = 0, PH_RGU = 1, PH_DN = 2 };
+
+struct Walk {
+  // shared expert gate/up: channels [c0, c1)
+  __device__ static void sgu_range(const Params& p, int& c0, int& c1) {
+    c0 = (int)((long long)blockIdx.x * p.I / p.G);
+    c1 = (int)((long long)(blockIdx.x + 1) * p.I / p.G);
+  }
+  // routed gate/up over the unique-expert list: global channels [g0, g1)
+  __device__ static void rgu_range(const Params& p, int nu, long long& g0, long long& g1) {
+    long long n = (long long)nu * p.I;
+    g0 = (long long)blockIdx.x * n / p.G;
+    g1 = (long long)(blockIdx.x + 1) * n / p.G;
+  }
+  // down: output channels [h0, h1) of every expert
+  __device__ static void dn_range(const Params& p, int& h0, int& h1) {
+    h0 = (int)((long long)blockIdx.x * p.H / p.G);
+    h1 = (int)((long long)(blockIdx.x + 1) * p.H / p.G);
+  }
+};
+
+// ============================================================== prologue ==
+// Thread numbering of the prologue group (compute warps 0-7 and control warps
+// 10-11): 0 .. kPreThreads-1.
+__device__ __forceinline__ int pre_tid() {
+  const int t = threadIdx.x;
+  return t < kCW * 32 ? t : t - (kCtlWarp0 - kCW) * 32;
+}
+
+// A2 (every CTA, on the h-range it also owns in the tail): materialise this
+// layer's residual streams from the previous layer's pending post/comb expand
+// (or read hc_in), then the partial mix products and square sums.  A3: wait
+// for every CTA's partials, reduce them in one fixed order in every CTA, and
+// derive rho, mix, pre and post.
+__device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep1) {
+  const int R = p.R, H = p.H, G = p.G;
+  const int ptid = pre_tid(), pwarp = ptid >> 5, lane = threadIdx.x & 31;
+  const int nout = R * kMixP;
+  {
+    int h0, h1;
+    Walk::dn_range(p, h0, h1);
+    const int nh = h1 - h0;
+    float* ws = reinterpret_cast<float*>(regA);          // [S][nh][24] slice of mix_w
+    float* xs = ws + (size_t)kS * nh * kMixC;            // [R][S][nh]
+    const int seg4 = nh * (kMixC / 4);
+    for (int i = ptid; i < kS * seg4; i += kPreThreads) {
+      const int sgm = i / seg4, j = i % seg4;
+      reinterpret_cast<float4*>(ws)[i] =
+          __ldg(reinterpret_cast<const float4*>(p.mix_w + ((size_t)sgm * H + h0) * kMixC) + j);
+    }
+    const float* ppost = p.pend_in;
+    const float* pcomb = p.pend_in + R * kS;
+    const float* py = p.pend_in + R * kS + R * kS * kS;
+    for (int i = ptid; i < R * kS * nh; i += kPreThreads) {
+      const int r = i / (kS * nh), sg = (i / nh) % kS, h = h0 + i % nh;
+      float v;
+      if (p.first) {
+        v = load_x(p.x_prev, ((size_t)r * kS + sg) * H + h, p.hc_bf16);
+      } else {
+        // the previous layer's deferred post: X_s = sum_j comb_sj Xprev_j + post_s y
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < kS; ++j)
+          acc = fmaf(pcomb[(r * kS + sg) * kS + j], load_x(p.x_prev, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
+        acc = fmaf(ppost[r * kS + sg], py[(size_t)r * H + h], acc);
+        v = p.hc_bf16 ? round_bf16(acc) : acc;
+        store_x(p.xbuf, ((size_t)r * kS + sg) * H + h, v, p.hc_bf16);
+      }
+      xs[i] = v;
+      if (p.taps.x) p.taps.x[((size_t)r * kS + sg) * H + h] = v;
+    }
+    bar_sync(kBarPre, kPreThreads);
+    // outputs o = r * 25 + col (col 24: the square sum), each split in P parts
+    const int P = max(1, kPreThreads / nout);
+    const int T = kS * nh;
+    for (int op = ptid; op < nout * P; op += kPreThreads) {
+      const int o = op / P, part = op % P, r = o / kMixP, col = o % kMixP;
+      float acc = 0.f;
+      for (int t = part; t < T; t += P) {
+        const float x = xs[r * T + t];
+        acc = col < kMixC ? fmaf(x, ws[t * kMixC + col], acc) : fmaf(x, x, acc);
+      }
+      c->red[op] = acc;
+    }
+    bar_sync(kBarPre, kPreThreads);
+    // partials stored output-major: mix_part[o][G]
+    for (int o = ptid; o < nout; o += kPreThreads) {
+      float acc = 0.f;
+      for (int part = 0; part < P; ++part) acc += c->red[o * P + part];
+      p.mix_part[(size_t)o * G + blockIdx.x] = acc;
+    }
+    bar_sync(kBarPre, kPreThreads);
+    if (ptid == 0) {
+      __threadfence();
+      red_release_add(&p.sync->cnt_mix, 1u);
+    }
+    trace(p, 1, ptid == 0);
+  }
+
+  if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix, ep1 * (uint32_t)G, 1u);
+  bar_sync(kBarPre, kPreThreads);
+  trace(p, 2, ptid == 0);
+  {
+    // lane-strided sums then a butterfly across the warp, the same order in
+    // every CTA
+    float* parts = reinterpret_cast<float*>(regA);
+    const int cap = p.regA_bytes / (int)sizeof(float) / G;   // outputs per pass
+    for (int o0 = 0; o0 < nout; o0 += cap) {
+      const int no = min(cap, nout - o0);
+      const int n4 = no * G / 4;   // G * 4 bytes is a multiple of 16 (the plan keeps G % 4 == 0)
+      const float4* src = reinterpret_cast<const float4*>(p.mix_part + (size_t)o0 * G);
+      for (int i = ptid; i < n4; i += kPreThreads)
+        reinterpret_cast<float4*>(parts)[i] = c->dead ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(src + i);
+      bar_sync(kBarPre, kPreThreads);
+      for (int o = pwarp; o < no; o += kPreThreads / 32) {
+        float acc = 0.f;
+        for (int m = lane; m < G; m += 32) acc += parts[o * G + m];
+        acc = warp_sum(acc);
+        if (lane == 0) c->smix[(o0 + o) / kMixP][(o0 + o) % kMixP] = acc;
+      }
+      bar_sync(kBarPre, kPreThreads);
+    }
+    if (ptid < R) {
+      const int r = ptid;
+      const float rho = 1.0f / sqrtf(c->smix[r][kMixC] / (float)(kS * H) + p.rms_eps);
+      for (int col = 0; col < kMixC; ++col) c->smix[r][col] *= rho;
+      for (int sg = 0; sg < kS; ++sg) {
+        c->pre[r][sg] = sigmoidf_(c->smix[r][sg]) + p.pre_eps;
+        c->post[r][sg] = p.post_mult * sigmoidf_(c->smix[r][kS + sg]);
+      }
+    }
+    bar_sync(kBarPre, kPreThreads);
+    if (blockIdx.x == 0) {
+      for (int i = ptid; i < R * kMixC; i += kPreThreads)
+        if (p.taps.mix) p.taps.mix[i] = c->smix[i / kMixC][i % kMixC];
+      for (int i = ptid; i < R * kS; i += kPreThreads) {
+        if (p.taps.pre) p.taps.pre[i] = c->pre[i / kS][i % kS];
+        if (p.taps.post) p.taps.post[i] = c->post[i / kS][i % kS];
+        if (!p.last) p.pend_out[i] = c->post[i / kS][i % kS];
+      }
+    }
+  }
+}
+
+// Control warps: Sinkhorn of the comb logits (16 threads per row), then, once
+// every CTA's router logits are out, the canonical top-k of each row and the
+// list of unique routed experts with their rows and act slots.
+__device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1) {
+  const int R = p.R, E = p.E, K = p.K, G = p.G;
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kCtlWarp0;
+  const int ct = threadIdx.x - kCtlWarp0 * 32;
+  for (int r0 = 0; r0 < kMaxR; r0 += kCtlWarps * 2) {
+    const int r = r0 + (ct >> 4), e = ct & 15;
+    const bool act = r < R;
+    float lg = act ? c->smix[r][2 * kS + e] : 0.f;
+    float mx = lg;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o, 16));
+    float v = expf(lg - mx);
+    for (int it = 0; it < p.sink_iters; ++it) {
+      float rs = v + __shfl_xor_sync(0xffffffffu, v, 1, 16);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 2, 16);
+      v = v / rs;
+      float cs = v + __shfl_xor_sync(0xffffffffu, v, 4, 16);
+      cs += __shfl_xor_sync(0xffffffffu, cs, 8, 16);
+      v = v / cs;
+    }
+    if (act) {
+      c->comb[r][e] = v;
+      if (blockIdx.x == 0) {
+        if (p.taps.comb) p.taps.comb[r * 16 + e] = v;
+        if (!p.last) p.pend_out[R * kS + r * 16 + e] = v;
+      }
+    }
+  }
+  if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
+  bar_sync(kBarCtl, kCtlWarps * 32);
+  for (int r = cw; r < R; r += kCtlWarps) {
+    if (E <= 32) topk_row<1>(p, c, r);
+    else if (E <= 64) topk_row<2>(p, c, r);
+    else if (E <= 128) topk_row<4>(p, c, r);
+    else if (E <= 256) topk_row<8>(p, c, r);
+    else if (E <= 512) topk_row<16>(p, c, r);
+    else topk_row<32>(p, c, r);
+  }
+  for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
+  bar_sync(kBarCtl, kCtlWarps * 32);
+  for (int i = ct; i < R * K; i += kCtlWarps * 32) {
+    const int e = c->idx[i / K][i % K];
+    if (e >= 0 && e < E) atomicOr(&c->bm[e >> 5], 1u << (e & 31));
+  }
+  bar_sync(kBarCtl, kCtlWarps * 32);
+  if (cw == 0) {
+    static_assert(kMaxE / 32 == 32, "one bitmap word per lane");
+    uint32_t word = c->dead ? 0u : c->bm[lane];
+    const int cnt = __popc(word);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int pos = incl - cnt;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      word &= word - 1u;
+      c->ulist[pos++] = lane * 32 + b;
+    }
+    if (lane == 31) c->nu_ctl = incl;
+  }
+  bar_sync(kBarCtl, kCtlWarps * 32);
+  const int nu = c->nu_ctl;
+  for (int u = ct; u < nu; u += kCtlWarps * 32) {
+    const int e = c->ulist[u];
+    uint32_t mask = 0u;
+    for (int r = 0; r < kMaxR; ++r) {
+      signed char sl = -1;
+      if (r < R)
+        for (int j = 0; j < K; ++j)
+          if (c->idx[r][j] == e) sl = (signed char)j;
+      c->uslot[u][r] = sl;
+      if (sl >= 0) mask |= 1u << r;
+    }
+    c->umask[u] = mask;
+  }
+  bar_sync(kBarCtl, kCtlWarps * 32);
+  if (ct == 0) {
+    c->nu = nu;
+    __threadfence_block();
+    *(volatile int*)&c->lists_ready = 1;
+    trace(p, 5);
+  }
+}
+
+// Where n (the normed rows) lives in shared memory: row-major [R][H] (bf16 if
+// rounded, else fp32) for the CUDA-core kernel, or the tensor-core B operand
+// layout [H/8][8 rows][8] bf16 with rows >= R zero.
+template <bool CANON>
+__device__ __forceinline__ size_t n_off(int r, int h, int H, bool bf) {
+  if (CANON) return ((size_t)(h >> 3) * 8 + r) * 16 + (size_t)(h & 7) * 2;
+  return ((size_t)r * H + h) * (bf ? 2 : 4);
+}
+
+// Collapse a = sum_s pre_s X_s (-> bf16), weighted RMSNorm n = a / sqrt(mean
+// a^2 + eps) * norm_w (-> bf16), into shared memory; compute warps only.
+template <bool CANON>
+__device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA) {
+  const int R = p.R, H = p.H, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
+  const bool nbf = CANON || p.round_bf16;
+  const void* X = p.first ? p.x_prev : (const void*)p.xbuf;
+  const int H8 = H / 8;
+  float sq[kMaxR];
+#pragma unroll
+  for (int r = 0; r < kMaxR; ++r) sq[r] = 0.f;
+#pragma unroll 2
+  for (int i = ctid; i < R * H8; i += kCW * 32) {
+    const int r = i / H8, h = (i % H8) * 8;
+    float xv[kS][8];
+#pragma unroll
+    for (int sg = 0; sg < kS; ++sg) load_hc8(X, ((size_t)r * kS + sg) * H + h, p.hc_bf16, xv[sg]);
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float acc = 0.f;
+#pragma unroll
+      for (int sg = 0; sg < kS; ++sg) acc = fmaf(c->pre[r][sg], xv[sg][k], acc);
+      a[k] = p.round_bf16 ? round_bf16(acc) : acc;
+    }
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) q = fmaf(a[k], a[k], q);
+#pragma unroll
+    for (int r2 = 0; r2 < kMaxR; ++r2)
+      if (r2 == r) sq[r2] += q;
+    if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
+    else store8(regA, (size_t)r * H + h, nbf, a);
+  }
+  if (CANON) {
+    // rows R..7 of the B operand are zero
+    for (int i = ctid; i < (8 - R) * H8; i += kCW * 32) {
+      const int r = R + i / H8, h = (i % H8) * 8;
+      *reinterpret_cast<uint4*>(regA + n_off<true>(r, h, H, true)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kMaxR; ++r) {
+    float v = warp_sum(sq[r]);
+    if (lane == 0) c->sq[warp][r] = v;
+  }
+  bar_sync(kBarCons, kCW * 32);
+  if (ctid < R) {
+    float t = 0.f;
+    for (int w = 0; w < kCW; ++w) t += c->sq[w][ctid];
+    c->inv[ctid] = 1.0f / sqrtf(t / (float)H + p.rms_eps);
+  }
+  bar_sync(kBarCons, kCW * 32);
+#pragma unroll 2
+  for (int i = ctid; i < R * H8; i += kCW * 32) {
+    const int r = i / H8, h = (i % H8) * 8;
+    float a[8], w[8];
+    if (CANON) load8(regA + n_off<true>(r, h, H, true), 0, true, a);
+    else load8(regA, (size_t)r * H + h, nbf, a);
+    load_hc8(p.norm_w, h, p.norm_bf16, w);
+    const float inv = c->inv[r];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float v = a[k] * inv * w[k];
+      a[k] = p.round_bf16 ? round_bf16(v) : v;
+    }
+    if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
+    else store8(regA, (size_t)r * H + h, nbf, a);
+    if (blockIdx.x == 0 && p.taps.n) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) p.taps.n[(size_t)r * H + h + k] = a[k];
+    }
+  }
+  bar_sync(kBarCons, kCW * 32);
+}
+
+// Router logits of this CTA's experts (two rows of router_t at a time), then
+// the CTA's arrival at the logits counter; compute warps only.
+template <bool CANON>
+__device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
+  const int R = p.R, H = p.H, E = p.E, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
+  const bool nbf = CANON || p.round_bf16;
+  const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
+  for (int e = e0; e < e1; e += 2) {
+    const bool two = e + 1 < e1;
+    const float* w0 = p.router_t + (size_t)e * H;
+    const float* w1 = two ? w0 + H : w0;
+    float a0[kMaxR], a1[kMaxR];
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r) { a0[r] = 0.f; a1[r] = 0.f; }
+#pragma unroll 4
+    for (int h = ctid * 4; h < H; h += kCW * 32 * 4) {
+      const float4 v0 = __ldg(reinterpret_cast<const float4*>(w0 + h));
+      const float4 v1 = __ldg(reinterpret_cast<const float4*>(w1 + h));
+#pragma unroll
+      for (int r = 0; r < kMaxR; ++r) {
+        if (r < R) {
+          float nv[4];
+          if (nbf) load_vec<4, true>(n_s + n_off<CANON>(r, h, H, true), 0, nv);
+          else load_vec<4, false>(n_s + n_off<CANON>(r, h, H, false), 0, nv);
+          a0[r] = fmaf(v0.x, nv[0], fmaf(v0.y, nv[1], fmaf(v0.z, nv[2], fmaf(v0.w, nv[3], a0[r]))));
+          a1[r] = fmaf(v1.x, nv[0], fmaf(v1.y, nv[1], fmaf(v1.z, nv[2], fmaf(v1.w, nv[3], a1[r]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r) {
+      const float v0 = warp_sum(a0[r]);
+      const float v1 = warp_sum(a1[r]);
+      if (lane == 0) {
+        c->sq[warp][r] = v0;
+        c->sq2[warp][r] = v1;
+      }
+    }
+    bar_sync(kBarCons, kCW * 32);
+    if (ctid < 2 * R) {
+      const int r = ctid % R, which = ctid / R;
+      if (which == 0 || two) {
+        float t = 0.f;
+        for (int w = 0; w < kCW; ++w) t += which ? c->sq2[w][r] : c->sq[w][r];
+        p.logits[(size_t)r * E + e + which] = t;
+      }
+    }
+    bar_sync(kBarCons, kCW * 32);
+  }
+  if (ctid == 0 && (int)blockIdx.x != p.fault_cta) {
+    __threadfence();
+    red_release_add(&p.sync->cnt_logit, 1u);
+  }
+  trace(p, 4, ctid == 0);
+}
+
+// Tail on the CTA's h-range: y = bf16(routed + shared) from yfun(r, h), then
+// out_i = sum_j comb_ij X_j + post_i y (last layer) or the pending state for
+// the next layer's opening expand; compute warps only.
+template <class YF>
+__device__ void tail(const Params& p, Ctl* c, YF yfun) {
+  const int R = p.R, H = p.H, ctid = threadIdx.x;
+  int h0, h1;
+  Walk::dn_range(p, h0, h1);
+  const int nh = h1 - h0;
+  const void* X = p.first ? p.x_prev : (const void*)p.xbuf;
+  float* pend_y = p.pend_out + R * kS + R * kS * kS;
+  for (int i = ctid; i < R * nh; i += kCW * 32) {
+    const int r = i / nh, h = h0 + i % nh;
+    float y = c->dead ? 0.f : yfun(r, h);
+    if (p.round_bf16) y = round_bf16(y);
+    if (p.taps.y) p.taps.y[(size_t)r * H + h] = y;
+    if (!p.last) {
+      pend_y[(size_t)r * H + h] = y;
+    } else {
+#pragma unroll
+      for (int si = 0; si < kS; ++si) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < kS; ++j)
+          acc = fmaf(c->comb[r][si * kS + j], load_x_cg(X, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
+        acc = fmaf(c->post[r][si], y, acc);
+        store_x(p.hc_out, ((size_t)r * kS + si) * H + h, acc, p.hc_bf16);
+      }
+    }
+  }
+}
+
+// The CTA's arrival at the end counter; the last CTA of the step advances the
+// layer's epoch.  Compute thread 0.
+__device__ __forceinline__ void finish_step(const Params& p, Ctl* c, uint32_t ep1) {
+  if (threadIdx.x == 0 && !c->dead) {
+    __threadfence();
+    const uint32_t old = atomicAdd(&p.sync->cnt_done, 1u);
+    if (old == ep1 * (uint32_t)p.G - 1u) {
+      __threadfence();
+      atomicAdd(&p.sync->epoch, 1u);
+    }
+  }
+}
+
+}  // namespace mono

@@ -10,7 +10,8 @@
 #include <vector>
 
 #include "mono_ffn.h"
-#include "mono_ffn_kernel.cuh"
+#include "cc_kernel.cuh"
+#include "tc_kernel.cuh"
 
 using namespace mono;
 
@@ -34,6 +35,7 @@ struct LayerSlot {
 struct mono_ffn_plan_s {
   mono_ffn_config cfg{};
   int wt = 0;
+  bool tc = false;   // bf16 experts run on the tensor-core kernel
   int G = 0, nst = 0, slot_bytes = 0, regA_bytes = 0, ymax = 0, mix_ctas = 0, smem = 0;
   int gu_kc = 0, gu_nk = 0, gu_rc = 0, dn_kc = 0, dn_nk = 0, dn_rc = 0;
   long long gu_estride = 0, dn_estride = 0;
@@ -41,6 +43,12 @@ struct mono_ffn_plan_s {
   float* mix_part = nullptr;
   float* logits = nullptr;
   float* act = nullptr;
+  float* yp = nullptr;
+  float* gpart = nullptr;
+  float* dpart = nullptr;
+  uint32_t* gcnt = nullptr;
+  uint32_t* dcnt = nullptr;
+  size_t gcnt_n = 0, dcnt_n = 0;
   std::vector<float*> pend;
   void* xbuf[2] = {nullptr, nullptr};
   SyncBlock* sync = nullptr;
@@ -87,15 +95,33 @@ int cuda_fail(mono_ffn_plan_t* p, cudaError_t e, const char* what) {
 
 template <int WT>
 void* kernel_ptr() {
-  return reinterpret_cast<void*>(&mono_ffn_layer_kernel<WT>);
+  return reinterpret_cast<void*>(&mono_ffn_cc_kernel<WT>);
 }
 
-void* kernel_for(int wt) {
+void* kernel_for(int wt, bool tc) {
+  if (tc) return reinterpret_cast<void*>(&mono_ffn_tc_kernel<W_BF16>);
   switch (wt) {
     case W_F32: return kernel_ptr<W_F32>();
     case W_BF16: return kernel_ptr<W_BF16>();
     case W_FP8: return kernel_ptr<W_FP8>();
     default: return kernel_ptr<W_FP4>();
+  }
+}
+
+// Tensor-core layout of one [E+1][rows][cols] bf16 matrix set: blocks of 128
+// rows; inside a block, per contraction group kg (8 elements), the 16
+// rowgroups of 8 rows as core matrices of 8 rows x 16 bytes, each rg taking
+// rgb bytes (gate and up share one: sub = 0 or 128).  The 16-byte chunk of
+// (e, row, kg) lands at
+//   dst[((e * rows/128 + row/128) * cols/8 + kg) * 16 * rgb + ((row % 128) / 8) * rgb + sub + (row % 8) * 16].
+__global__ void pack_tc_kernel(const uint16_t* src, uint8_t* dst, long long e1, int rows, int cols, int rgb, int sub) {
+  const long long KG = cols / 8, NB = rows / 128;
+  const long long n = e1 * rows * KG;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long kg = i % KG, row = (i / KG) % rows, e = i / (KG * rows);
+    const uint4 v = *reinterpret_cast<const uint4*>(src + ((e * rows + row) * cols + kg * 8));
+    const long long off = ((e * NB + row / 128) * KG + kg) * 16 * rgb + ((row % 128) / 8) * rgb + sub + (row % 8) * 16;
+    *reinterpret_cast<uint4*>(dst + off) = v;
   }
 }
 
@@ -195,6 +221,11 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
   cudaFree(p->mix_part);
   cudaFree(p->logits);
   cudaFree(p->act);
+  cudaFree(p->yp);
+  cudaFree(p->gpart);
+  cudaFree(p->dpart);
+  cudaFree(p->gcnt);
+  cudaFree(p->dcnt);
   cudaFree(p->xbuf[0]);
   cudaFree(p->xbuf[1]);
   cudaFree(p->sync);
@@ -254,6 +285,8 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   cudaSetDevice(cfg.device);
   const int H = cfg.hidden, I = cfg.inter, E = cfg.n_routed, K = cfg.top_k, RM = cfg.max_rows;
 
+  // bf16 experts run on the tensor cores when the shapes allow it
+  p->tc = dt == MONO_BF16 && H % 128 == 0 && I % 128 == 0;   // whole 128-row blocks and 128-wide K units
   // chunking of the packed rows
   const int gu_target = dt == MONO_F32 ? 256 : dt == MONO_BF16 ? 512 : 1024;
   const int dn_target = dt == MONO_F32 ? 512 : dt == MONO_BF16 ? 1024 : 2048;
@@ -266,6 +299,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->gu_estride = (long long)I * p->gu_nk * 2 * p->gu_rc;
   p->dn_estride = (long long)H * p->dn_nk * p->dn_rc;
   p->slot_bytes = (int)align_up((size_t)std::max(kCW * 2 * p->gu_rc, kCW * p->dn_rc), 128);
+  if (p->tc) {
+    p->gu_estride = (long long)(I / 128) * (H / 8) * 4096;
+    p->dn_estride = (long long)(H / 128) * (I / 8) * 2048;
+    p->slot_bytes = 16384;
+  }
 
   // grid and shared memory
   // grid: one CTA per SM, a multiple of 4 (the mix partials are read as float4 per output)
@@ -280,10 +318,14 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   regA = std::max<size_t>(regA, (size_t)2 * I * 4 + 256);
   regA = std::max<size_t>(regA, ((size_t)kS * p->ymax * kMixC + (size_t)RM * kS * p->ymax) * 4);
   regA = std::max<size_t>(regA, (size_t)p->G * kMixP * 4);
+  if (p->tc) {
+    regA = std::max<size_t>(regA, (size_t)H * 16);   // n: 8 rows of bf16
+    regA = std::max<size_t>(regA, (size_t)I * 32);   // down B: 16 rows (hi/lo of 8 token rows)
+  }
   p->regA_bytes = (int)align_up(regA, 128);
   const int smem_max = prop.sharedMemPerBlockOptin;
   SmemLayout L0(0, p->slot_bytes, p->regA_bytes, p->ymax);
-  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16;
+  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard;
   p->nst = (int)std::min<long long>(16, room / p->slot_bytes);
   if (p->nst < 2) {
     std::string m = "shared memory: " + std::to_string(smem_max) + " bytes leave room for " + std::to_string(p->nst) +
@@ -293,7 +335,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     return fail(nullptr, MONO_ERR_INVALID_ARG, m);
   }
   p->smem = (int)SmemLayout(p->nst, p->slot_bytes, p->regA_bytes, p->ymax).total;
-  void* kfn = kernel_for(dt);
+  void* kfn = kernel_for(dt, p->tc);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
   int occ = 0;
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kfn, kThreads, p->smem);
@@ -321,6 +363,13 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->act, (size_t)RM * (K + 1) * I * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->yp, (size_t)RM * (K + 1) * H * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->gpart, (size_t)p->G * 4 * 128 * 16 * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->dpart, (size_t)p->G * 2 * 128 * 16 * 4, &p->scratch_bytes);
+  p->gcnt_n = (size_t)(RM * K + 2) * (I / 128);
+  p->dcnt_n = (size_t)(RM * K + 2) * (H / 128);
+  if (!rc && p->tc) rc = dalloc(p, &p->gcnt, p->gcnt_n * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->dcnt, p->dcnt_n * 4, &p->scratch_bytes);
   p->pend.assign(cfg.n_layers, nullptr);
   for (int l = 0; l + 1 < cfg.n_layers && !rc; ++l)
     rc = dalloc(p, &p->pend[l], (size_t)RM * (kS + kS * kS + H) * 4, &p->scratch_bytes);
@@ -336,6 +385,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     cudaMemset(p->sync, 0, sizeof(SyncBlock) * cfg.n_layers);
     cudaMemset(p->err, 0, sizeof(ErrBlock));
     cudaMemset(p->act, 0, (size_t)RM * (K + 1) * I * 4);
+    if (p->tc) {
+      cudaMemset(p->yp, 0, (size_t)RM * (K + 1) * H * 4);
+      cudaMemset(p->gcnt, 0, p->gcnt_n * 4);
+      cudaMemset(p->dcnt, 0, p->dcnt_n * 4);
+    }
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) rc = cuda_fail(p, e, "plan setup");
   }
@@ -372,6 +426,21 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
   cudaMemcpyAsync(l.bias, w->router_bias, (size_t)E * 4, cudaMemcpyDeviceToDevice, st);
   transpose_f32_kernel<<<dim3((E + 31) / 32, (H + 31) / 32), dim3(32, 8), 0, st>>>(w->router_w, l.router_t, H, E);
   int rc = 0;
+  if (p->tc) {
+    // 128-row blocks of core matrices: gate and up of a rowgroup side by
+    // side, down in its own blocks
+    const int th = 256;
+    auto grid = [&](long long n) { return (unsigned)std::min<long long>((n + th - 1) / th, 148LL * 64); };
+    const long long n_gu = (long long)(E + 1) * I * (H / 8), n_dn = (long long)(E + 1) * H * (I / 8);
+    pack_tc_kernel<<<grid(n_gu), th, 0, st>>>((const uint16_t*)w->w_gate, l.gu, E + 1, I, H, 256, 0);
+    pack_tc_kernel<<<grid(n_gu), th, 0, st>>>((const uint16_t*)w->w_up, l.gu, E + 1, I, H, 256, 128);
+    pack_tc_kernel<<<grid(n_dn), th, 0, st>>>((const uint16_t*)w->w_down, l.dn, E + 1, H, I, 128, 0);
+    cudaError_t e2 = cudaGetLastError();
+    cudaSetDevice(prev);
+    if (e2 != cudaSuccess) return cuda_fail(p, e2, "pack");
+    l.packed = true;
+    return MONO_OK;
+  }
   // gate and up share an item: [gate chunk | up chunk]
   rc = pack_matrix(p, w->w_gate, w->s_gate, l.gu, (long long)(E + 1) * I, H, p->gu_kc, p->gu_nk, p->gu_rc,
                    2 * p->gu_rc, 0, st);
@@ -430,7 +499,7 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
   cudaGetDevice(&prev);
   if (prev != p->cfg.device) cudaSetDevice(p->cfg.device);
   const int L = p->cfg.n_layers;
-  void* kfn = kernel_for(p->wt);
+  void* kfn = kernel_for(p->wt, p->tc);
   cudaError_t e = cudaSuccess;
   for (int l = 0; l < L && e == cudaSuccess; ++l) {
     const LayerSlot& ls = p->layers[l];
@@ -476,6 +545,11 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.mix_part = p->mix_part;
     prm.logits = p->logits;
     prm.act = p->act;
+    prm.yp = p->yp;
+    prm.gpart = p->gpart;
+    prm.dpart = p->dpart;
+    prm.gcnt = p->gcnt;
+    prm.dcnt = p->dcnt;
     prm.sync = p->sync + l;
     prm.err = p->err;
     prm.taps = ls.taps;
@@ -545,6 +619,8 @@ extern "C" int mono_ffn_query_error(mono_ffn_plan_t* p, mono_ffn_status* st) {
     // reset the sync state so the next step starts clean
     cudaMemset(p->sync, 0, sizeof(SyncBlock) * p->cfg.n_layers);
     cudaMemset(p->err, 0, sizeof(ErrBlock));
+    if (p->gcnt) cudaMemset(p->gcnt, 0, p->gcnt_n * 4);
+    if (p->dcnt) cudaMemset(p->dcnt, 0, p->dcnt_n * 4);
     cudaDeviceSynchronize();
   }
   if (st) {
