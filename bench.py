@@ -46,6 +46,10 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+L2_MODE = ["flush"]
+TRACE_DUMP = [None]
+
+
 def workload(name):
     from synth import configs as C
     return C.BY_NAME[name]
@@ -55,7 +59,8 @@ def wl_config(wl, extra=None):
     cfg = {"workload": wl.name, "rows": wl.rows, "hidden": wl.hidden, "hc_streams": wl.hc,
            "routed_experts": wl.n_routed, "top_k": wl.top_k, "shared_experts": 1, "inter": wl.inter,
            "layers_per_step": wl.n_layers, "expert_format": wl.w_dtype, "hc_format": wl.hc_dtype,
-           "l2": "flushed before every timed step (512 MiB write)",
+           "l2": "flushed before every timed step (512 MiB write)" if L2_MODE[0] == "flush" else
+                 "not flushed: every step streams its weights (larger than the 126 MB L2) through it",
            "inputs": f"{N_INPUT_SETS} rotating seeded hc_in sets"}
     if extra:
         cfg.update(extra)
@@ -172,26 +177,34 @@ def run_reference(args):
 
 TRACE_NAMES = ["start", "mix published", "mix totals seen", "n ready", "logits published", "lists ready",
                "shared gate/up done", "routed gate/up done", "activations seen", "down done", "end",
-               "producer saw lists", "producer issued all"]
+               "producer saw lists", "producer issued all", "issuer: 1st routed stage", "issuer: routed issued",
+               "issuer: 1st down operand", "issuer: all issued", "(unused)", "producer: 1st routed",
+               "producer: 1st down", "epilogue: 1st shared", "ctl: logits complete", "ctl: top-k done",
+               "pre/post ready", "collapse done", "router: dots done", "top-k: loads done", "collapse: sums done",
+               "mix: inputs in smem"]
+TRACE_POINTS = 32
 
 
 def print_trace(plan, wl, sets, out, flush):
     """One extra traced step: stage timestamps relative to the earliest CTA
     start, min / median / max over CTAs (µs), to stderr."""
+    import numpy as np
     import torch
     info = plan.info()
     G = info["grid"]
-    buf = torch.zeros(wl.n_layers * G * 16, dtype=torch.int64, device="cuda")
+    buf = torch.zeros(wl.n_layers * G * TRACE_POINTS, dtype=torch.int64, device="cuda")
     plan.set_trace(buf)
     flush.zero_()
     plan.step(wl.rows, sets[0], out)
     torch.cuda.synchronize()
     plan.set_trace(None)
-    t = buf.view(wl.n_layers, G, 16).cpu().numpy().astype("float64")
+    t = buf.view(wl.n_layers, G, TRACE_POINTS).cpu().numpy().astype("float64")
+    if TRACE_DUMP[0]:
+        np.save(TRACE_DUMP[0], t)
     for l in range(wl.n_layers):
         t0 = t[l, :, 0].min()
         print(f"layer {l}: stage times in us from the first CTA start (min / median / max over CTAs)", file=sys.stderr)
-        for i, nm in enumerate(TRACE_NAMES):
+        for i, nm in enumerate(TRACE_NAMES[:31]):
             col = t[l, :, i]
             col = col[col > 0]
             if len(col) == 0:
@@ -225,6 +238,8 @@ def run_gpu(args):
     wl = workload(args.config)
     if args.routed:
         wl = wl.with_(name=f"{wl.name}-e{args.routed}", n_routed=args.routed)
+    if args.inter:
+        wl = wl.with_(name=f"{wl.name}-i{args.inter}", inter=args.inter)
     plan = Plan.for_workload(wl, device=local)
     info = plan.info()
     for l in range(wl.n_layers):
@@ -255,8 +270,12 @@ def run_gpu(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
+    def flush_l2():
+        if args.l2 == "flush":
+            flush.zero_()
+
     for k in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         plan.step(wl.rows, sets[k % N_INPUT_SETS], out)
     torch.cuda.synchronize()
 
@@ -267,7 +286,7 @@ def run_gpu(args):
     barrier()
     torch.cuda.synchronize()
     for k in range(K):
-        flush.zero_()
+        flush_l2()
         ev[k][0].record(stream)
         plan.step(wl.rows, sets[k % N_INPUT_SETS], out)
         ev[k][1].record(stream)
@@ -284,7 +303,7 @@ def run_gpu(args):
     barrier()
     torch.cuda.synchronize()
     for k in range(KE):
-        flush.zero_()
+        flush_l2()
         ev2[k][0].record(stream)
         plan.step_host(wl.rows, host_in[k % N_INPUT_SETS], host_out)
         ev2[k][1].record(stream)
@@ -351,10 +370,16 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--routed", type=int, default=0, help="override the routed-expert count (small profiling cases)")
+    ap.add_argument("--inter", type=int, default=0, help="override the expert width (small profiling cases)")
+    ap.add_argument("--trace-dump", default=None, help="with --trace: save the raw [layers][grid][32] stamps (.npy)")
     ap.add_argument("--trace", action="store_true", help="print per-stage device timestamps (stderr) after the run")
+    ap.add_argument("--l2", default="flush", choices=["flush", "none"],
+                    help="flush: write 512 MiB before every step; none: rely on the step's weights exceeding L2")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    L2_MODE[0] = args.l2
+    TRACE_DUMP[0] = args.trace_dump
     if args.impl == "reference":
         run_reference(args)
     else:

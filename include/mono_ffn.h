@@ -208,12 +208,21 @@ int mono_ffn_query_error(mono_ffn_plan_t* plan, mono_ffn_status* st);
 int mono_ffn_get_info(const mono_ffn_plan_t* plan, mono_ffn_info* info);
 
 /* Stage timestamps for profiling: with buf != NULL (device memory of
- * n_layers * grid * 16 uint64), every CTA of layer l writes %globaltimer (ns)
- * at its stage boundaries to buf[(l * grid + cta) * 16 + point]:
+ * n_layers * grid * 32 uint64), every CTA of layer l writes %globaltimer (ns)
+ * at its stage boundaries to buf[(l * grid + cta) * 32 + point]:
  * 0 start, 1 mix partials published, 2 mix totals seen, 3 n ready,
  * 4 router logits published, 5 top-k lists ready, 6 shared gate/up done,
  * 7 routed gate/up done, 8 all activations seen, 9 down projections done,
- * 10 end, 11 producer saw the lists, 12 producer issued every copy.
+ * 10 end, 11 producer saw the lists, 12 producer issued every copy;
+ * tensor-core kernel also: 13 first routed gate/up stage arrived, 14 routed
+ * gate/up MMAs issued, 15 first down operand ready, 16 every MMA issued,
+ * 17 (unused), 18 first routed copy issued, 19 first down
+ * copy issued, 20 first shared gate/up tile read; both: 21 logits counter
+ * complete, 22 top-k done, 23 pre/post ready, 24 collapse done, 25 router
+ * dot products done, 26 top-k inputs loaded, 27 collapse sums done, 28 mix
+ * inputs in shared memory.
+ * The tensor-core kernel stores its SM id (not a time) at point 31.
+ * Points a kernel does not reach stay as they were.
  * NULL turns it off (the default). */
 int mono_ffn_set_trace(mono_ffn_plan_t* plan, unsigned long long* buf);
 

@@ -38,8 +38,8 @@ constexpr int kCtlWarps = 2;
 constexpr int kThreads = 12 * 32;                      // 384: 12 warps leave 168 registers a thread
 constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // named barriers: prologue (compute + control), compute, control, epilogue
-// warps 0-3, builder warps 4-7, end (epilogue warps + the issuer warp)
-constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarBld = 5, kBarEnd = 6;
+// warps 0-3, end (epilogue warps + the issuer warp)
+constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarEnd = 6;
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
 
 enum WType { W_F32 = 0, W_BF16 = 1, W_FP8 = 2, W_FP4 = 3 };
@@ -90,6 +90,7 @@ struct Params {
   float* logits;     // [R][E]
   float* act;        // [R][K+1][I]
   float* yp;         // tensor-core kernel: [R][K+1][H] weighted expert outputs
+  uint8_t* actb;     // tensor-core kernel: [R*K+1][I/8][16][8] bf16 down-projection B operands
   float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks
   float* dpart;      // tensor-core kernel: [G][2][128][16] partial down tiles
   uint32_t* gcnt;    // tensor-core kernel: [R*K+2][I/128] arrivals per split gate/up block (0 between launches)
@@ -103,7 +104,7 @@ struct Params {
   unsigned long long* trace;   // optional [G][kTracePoints] globaltimer stamps
 };
 
-constexpr int kTracePoints = 16;
+constexpr int kTracePoints = 32;
 // stage timestamps (one writer per point and CTA)
 __device__ __forceinline__ void trace(const Params& p, int point, bool who = true) {
   if (p.trace && who) p.trace[blockIdx.x * kTracePoints + point] = globaltimer();
@@ -132,9 +133,8 @@ struct Ctl {
   // tensor-core kernel
   uint32_t tmem_base;
   volatile int n_ready;         // n is in shared memory (B operand of gate/up)
-  volatile int bld_seq;         // activation B operands built so far
-  volatile int mma_seq;         // activation B operands released by the issuer
   uint64_t accfull[2], accempty[2], drain;
+  uint64_t bfull;               // the down projection's B operand has landed
   volatile int bcast;           // epilogue: "this CTA completes the block"
 };
 
@@ -380,6 +380,7 @@ __device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
       key[q] = ord_key(score[q] + __ldg(p.bias + e));
     }
   }
+  trace(p, 26, r == 0 && lane == 0);
   uint32_t taken = 0u;
   float ssum = 0.f;
   for (int j = 0; j < K; ++j) {
@@ -494,6 +495,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       if (p.taps.x) p.taps.x[((size_t)r * kS + sg) * H + h] = v;
     }
     bar_sync(kBarPre, kPreThreads);
+    trace(p, 28, ptid == 0);
     // outputs o = r * 25 + col (col 24: the square sum), each split in P parts
     const int P = max(1, kPreThreads / nout);
     const int T = kS * nh;
@@ -554,6 +556,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       }
     }
     bar_sync(kBarPre, kPreThreads);
+    trace(p, 23, ptid == 0);
     if (blockIdx.x == 0) {
       for (int i = ptid; i < R * kMixC; i += kPreThreads)
         if (p.taps.mix) p.taps.mix[i] = c->smix[i / kMixC][i % kMixC];
@@ -598,6 +601,7 @@ __device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1) {
     }
   }
   if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
+  trace(p, 21, ct == 0);
   bar_sync(kBarCtl, kCtlWarps * 32);
   for (int r = cw; r < R; r += kCtlWarps) {
     if (E <= 32) topk_row<1>(p, c, r);
@@ -609,6 +613,7 @@ __device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1) {
   }
   for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
   bar_sync(kBarCtl, kCtlWarps * 32);
+  trace(p, 22, ct == 0);
   for (int i = ct; i < R * K; i += kCtlWarps * 32) {
     const int e = c->idx[i / K][i % K];
     if (e >= 0 && e < E) atomicOr(&c->bm[e >> 5], 1u << (e & 31));
@@ -699,6 +704,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA) {
     if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
     else store8(regA, (size_t)r * H + h, nbf, a);
   }
+  trace(p, 27, ctid == 0);
   if (CANON) {
     // rows R..7 of the B operand are zero
     for (int i = ctid; i < (8 - R) * H8; i += kCW * 32) {
@@ -712,6 +718,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA) {
     if (lane == 0) c->sq[warp][r] = v;
   }
   bar_sync(kBarCons, kCW * 32);
+  trace(p, 24, threadIdx.x == 0);
   if (ctid < R) {
     float t = 0.f;
     for (int w = 0; w < kCW; ++w) t += c->sq[w][ctid];
@@ -770,6 +777,7 @@ __device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
         }
       }
     }
+    trace(p, 25, ctid == 0 && e == e0);
 #pragma unroll
     for (int r = 0; r < kMaxR; ++r) {
       const float v0 = warp_sum(a0[r]);

@@ -44,6 +44,7 @@ struct mono_ffn_plan_s {
   float* logits = nullptr;
   float* act = nullptr;
   float* yp = nullptr;
+  uint8_t* actb = nullptr;
   float* gpart = nullptr;
   float* dpart = nullptr;
   uint32_t* gcnt = nullptr;
@@ -222,6 +223,7 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
   cudaFree(p->logits);
   cudaFree(p->act);
   cudaFree(p->yp);
+  cudaFree(p->actb);
   cudaFree(p->gpart);
   cudaFree(p->dpart);
   cudaFree(p->gcnt);
@@ -364,6 +366,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->act, (size_t)RM * (K + 1) * I * 4, &p->scratch_bytes);
   if (!rc && p->tc) rc = dalloc(p, &p->yp, (size_t)RM * (K + 1) * H * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->actb, (size_t)(RM * K + 1) * I * 32, &p->scratch_bytes);
   if (!rc && p->tc) rc = dalloc(p, &p->gpart, (size_t)p->G * 4 * 128 * 16 * 4, &p->scratch_bytes);
   if (!rc && p->tc) rc = dalloc(p, &p->dpart, (size_t)p->G * 2 * 128 * 16 * 4, &p->scratch_bytes);
   p->gcnt_n = (size_t)(RM * K + 2) * (I / 128);
@@ -546,6 +549,7 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.logits = p->logits;
     prm.act = p->act;
     prm.yp = p->yp;
+    prm.actb = p->actb;
     prm.gpart = p->gpart;
     prm.dpart = p->dpart;
     prm.gcnt = p->gcnt;

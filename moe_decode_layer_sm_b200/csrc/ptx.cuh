@@ -24,6 +24,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
@@ -55,6 +59,16 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const void* src, uint32_t
 
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// L2 prefetch of the 16-byte granules inside [src, src + bytes)
+__device__ __forceinline__ void prefetch_l2_span(const void* src, size_t bytes) {
+  const uintptr_t a = ((uintptr_t)src + 15) & ~(uintptr_t)15;
+  const uintptr_t e = ((uintptr_t)src + bytes) & ~(uintptr_t)15;
+  for (uintptr_t q = a; q < e; q += 65536) {
+    const uintptr_t n = e - q < 65536 ? e - q : 65536;
+    prefetch_l2(reinterpret_cast<const void*>(q), (uint32_t)n);
+  }
 }
 
 // 16-byte asynchronous copy global -> shared (L2 only), grouped by commit
@@ -138,6 +152,23 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
       "l"(da), "l"(db), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// The same from a converged warp: one elected lane issues (the same lane
+// every time, so its commits track all of its MMAs); the operands stay
+// warp-uniform, which keeps the descriptor arithmetic cheap.
+__device__ __forceinline__ void umma_bf16_warp(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
       : "memory");
 }
 

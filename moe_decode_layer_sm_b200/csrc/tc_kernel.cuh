@@ -12,14 +12,18 @@
 // CTA that completes a split block last (an atomic per block) adds the parts
 // in CTA order, so results do not depend on timing.
 //
-//   producer (warp 8)   TMA bulk copies into the ring, plus L2 prefetch ahead
+//   producer (warp 8)   TMA bulk copies into the ring (the ring's depth is
+//                       what keeps enough bytes in flight: an L2 prefetch
+//                       ahead of it only queues on the same copy engine)
 //   issuer (warp 9)     one thread: tcgen05.mma A from the ring, B from
-//                       shared memory (n for gate/up, activations for down),
-//                       D in tensor memory; tcgen05.commit releases slots
+//                       shared memory (n for gate/up, activations for down,
+//                       one bulk copy per down expert), D in tensor memory;
+//                       tcgen05.commit releases slots
 //   epilogue (0-3)      tcgen05.ld (warp w: TMEM lanes 32w..32w+31 = rows),
-//                       partial tiles, SwiGLU -> activations, down -> yp
-//   builders (4-7)      the down B operand: each token row's fp32 activation
-//                       as bf16 hi + lo rows (hi = bf16(a), lo = bf16(a - hi))
+//                       partial tiles, SwiGLU written straight in the down
+//                       B operand's layout: each token row's fp32 activation
+//                       as bf16 hi + lo rows (hi = bf16(a), lo = bf16(a - hi));
+//                       down -> yp
 //
 // B operands have N = 16 columns.  Gate/up uses the 8 rows of n twice (the
 // descriptor's row-group stride is 0: columns 8-15 repeat 0-7); down uses
@@ -33,7 +37,6 @@ constexpr int kTmemCols = 64;    // two accumulator buffers of 32 columns (gate 
 constexpr int kKS = 16;          // contraction groups (of 8) per work unit
 constexpr int kGuKgStage = 4;    // contraction groups per ring stage, gate/up (4 KB each)
 constexpr int kDnKgStage = 8;    // contraction groups per ring stage, down (2 KB each)
-constexpr int kPrefetch = 8;     // stages fetched into L2 ahead of the TMA copy
 enum TcList { L_SGU = 0, L_RGU = 1, L_DN = 2 };
 
 // One segment of a CTA's unit range: list, expert entry x (0 = shared),
@@ -126,8 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     c->lists_ready = 0;
     c->nu = 0;
     c->n_ready = 0;
-    c->bld_seq = 0;
-    c->mma_seq = 0;
     c->epoch = ld_relaxed(&p.sync->epoch);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       mbar_init(&c->accempty[b], 4);
     }
     mbar_init(&c->drain, 1);
+    mbar_init(&c->bfull, 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -150,11 +152,17 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   const uint32_t ep1 = c->epoch + 1u;
   const uint32_t tmem = c->tmem_base;
   trace(p, 0, tid == 0);
+  if (p.trace && tid == 0) {   // which SM this CTA runs on
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    p.trace[blockIdx.x * kTracePoints + 31] = sm;
+  }
 
   // ================================================================ producer
   if (warp == kProdWarp) {
     uint32_t s = 0, issued = 0;
     bool ok = true;
+    bool first_copy[2] = {false, false};
     auto seg = [&](const Seg& sg) {
       if (lane != 0) return;
       size_t kgb;
@@ -165,37 +173,34 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       for (int kg = kg0; kg < kg1; kg += kgs) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
         if (ok) {
-          const int pk = kg + kPrefetch * kgs;
-          if (pk < kg1) prefetch_l2(base + (size_t)pk * kgb, bytes);
           if (q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
           if (ok) {
             mbar_arrive_expect_tx(&full[slot], bytes);
             tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)kg * kgb, bytes, &full[slot]);
             issued = s + 1;
+            if (sg.list != L_SGU && !first_copy[sg.list - 1]) {
+              first_copy[sg.list - 1] = true;
+              trace(p, 17 + sg.list);
+            }
           }
         }
         ++s;
       }
     };
-    // the first stages of each segment go to L2 before its copies start
-    auto warm = [&](const Seg& sg) {
-      if (lane != 0 || !ok) return;
-      size_t kgb;
-      const uint8_t* base = seg_base(p, c, geo, sg, kgb);
-      const int kgs = sg.list != L_DN ? kGuKgStage : kDnKgStage;
-      const int kg0 = sg.k0 * kKS, kg1 = sg.k1 * kKS;
-      for (int j = 0; j < kPrefetch && kg0 + j * kgs < kg1; ++j)
-        prefetch_l2(base + (size_t)(kg0 + j * kgs) * kgb, (uint32_t)(kgs * kgb));
-    };
-    tc_segments(p, geo, L_SGU, 0, warm);
+    if (lane == 0) {
+      // the prologue's later inputs go to L2 ahead of the weight stream:
+      // this CTA's router rows, the norm weights and the router bias
+      const int e0 = (int)((long long)blockIdx.x * p.E / G), e1 = (int)((long long)(blockIdx.x + 1) * p.E / G);
+      prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
+      prefetch_l2_span(p.norm_w, (size_t)H * (p.norm_bf16 ? 2 : 4));
+      prefetch_l2_span(p.bias, (size_t)p.E * 4);
+    }
     tc_segments(p, geo, L_SGU, 0, seg);
     if (ok && lane == 0) ok = wait_flag(p, c, &c->lists_ready);
     ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
     const int nu = ok ? *(volatile int*)&c->nu : 0;
     trace(p, 11, lane == 0);
-    tc_segments(p, geo, L_RGU, nu, warm);
     tc_segments(p, geo, L_RGU, nu, seg);
-    tc_segments(p, geo, L_DN, nu, warm);
     tc_segments(p, geo, L_DN, nu, seg);
     trace(p, 12, lane == 0);
     if (lane == 0) {   // no bulk copy may still target this CTA's shared memory at exit
@@ -212,82 +217,115 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   }
 
   // =========================================================== MMA issuer
+  // The whole warp runs the loop (waits in lane 0, results broadcast), one
+  // elected lane issues the MMAs and commits.
   if (warp == kMmaWarp) {
-    int dgroup = -1;
-    if (lane == 0) {
-      uint32_t s = 0, t = 0;
-      int prev_x = -1;
-      bool ok = wait_flag(p, c, &c->n_ready);
-      const uint32_t b_addr = smem_u32(regA);
-      const uint32_t idesc = umma_idesc_bf16(128, 16);
-      auto seg = [&](const Seg& sg) {
-        const bool gu = sg.list != L_DN;
-        if (!gu && sg.x != prev_x) {
-          // a new down expert: hand the previous B operand back once its
-          // MMAs are done, then wait for this expert's operand
-          if (dgroup >= 0) {
-            umma_commit(&c->drain);
-            if (ok) ok = wait_bar(p, c, &c->drain, (uint32_t)dgroup & 1u);
-            tc_fence_after();
-            *(volatile int*)&c->mma_seq = dgroup + 1;
-          }
-          ++dgroup;
-          prev_x = sg.x;
-          volatile int* seq = &c->bld_seq;
-          const uint64_t t0 = globaltimer();
-          while (ok && *seq <= dgroup) {
-            if (c->dead) ok = false;
-            else if (globaltimer() - t0 > 2 * p.timeout_ns) {
-              record_error(p, c, 7u, 4u);
-              ok = false;
-            }
-            __nanosleep(32);
-          }
-          tc_fence_after();
+    uint32_t s = 0, t = 0, ndrain = 0, nb = 0;
+    int prev_x = -1;
+    bool first_rgu = true, b_pending = false;
+    auto warp_ok = [&](bool v) { return __shfl_sync(0xffffffffu, (int)v, 0) != 0; };
+    bool ok = true;
+    if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
+    ok = warp_ok(ok);
+    const uint32_t b_addr = smem_u32(regA);
+    const uint32_t idesc = umma_idesc_bf16(128, 16);
+    const uint32_t b_bytes = (uint32_t)I * 32u;
+    // descriptors: the start address sits in the low 14 bits (in 16-byte
+    // units), so moving an operand by d bytes adds d >> 4
+    const uint64_t bdesc_gu = umma_desc(b_addr, 128u, 0u), bdesc_dn = umma_desc(b_addr, 256u, 128u);
+    auto seg = [&](const Seg& sg) {
+      const bool gu = sg.list != L_DN;
+      if (!gu && sg.x != prev_x) {
+        // a new down expert: once every MMA reading the B region is done
+        // (and, the first time, every CTA's activations are out), one bulk
+        // copy brings this expert's operand in
+        if (prev_x < 0) {
+          if (lane == 0 && ok) ok = wait_count(p, c, &p.sync->cnt_act, ep1 * (uint32_t)G, 4u);
+          ok = warp_ok(ok);
+          fence_proxy_async_global();
+          trace(p, 8, lane == 0);
         }
-        const uint32_t buf = t & 1u;
-        if (t >= 2 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t >> 1) - 1) & 1u);
+        umma_commit_warp(&c->drain);
+        if (lane == 0 && ok) ok = wait_bar(p, c, &c->drain, ndrain & 1u);
+        ok = warp_ok(ok);
+        ++ndrain;
         tc_fence_after();
-        const uint32_t d0 = tmem + 32u * buf;
-        const int kgs = gu ? kGuKgStage : kDnKgStage;
-        const uint32_t kgb = gu ? 4096u : 2048u;
-        const int kg0 = sg.k0 * kKS, kg1 = sg.k1 * kKS;
-        for (int kg = kg0; kg < kg1; kg += kgs) {
-          const uint32_t slot = s % p.nst, q = s / p.nst;
-          if (ok) ok = wait_bar(p, c, &full[slot], q & 1);
-          tc_fence_after();
-          if (ok) {
-            const uint32_t a0 = smem_u32(ring + (size_t)slot * p.slot_bytes);
-            for (int ks = 0; ks < kgs / 2; ++ks) {
+        prev_x = sg.x;
+        if (ok) {   // (a copy whose wait failed is waited for again at exit)
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&c->bfull, b_bytes);
+            tma_load_1d(regA, p.actb + (size_t)sg.x * b_bytes, b_bytes, &c->bfull);
+            ok = wait_bar(p, c, &c->bfull, nb & 1u);
+          }
+          ok = warp_ok(ok);
+          b_pending = !ok;
+          ++nb;
+        }
+        tc_fence_after();
+        trace(p, 15, nb == 1 && lane == 0);
+      }
+      const uint32_t buf = t & 1u;
+      if (t >= 2) {
+        if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t >> 1) - 1) & 1u);
+        ok = warp_ok(ok);
+      }
+      tc_fence_after();
+      const uint32_t d0 = tmem + 32u * buf;
+      const int kgs = gu ? kGuKgStage : kDnKgStage;
+      const uint32_t kgb = gu ? 4096u : 2048u;
+      const int kg0 = sg.k0 * kKS, kg1 = sg.k1 * kKS;
+      for (int kg = kg0; kg < kg1; kg += kgs) {
+        const uint32_t slot = s % p.nst, q = s / p.nst;
+        if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
+        ok = warp_ok(ok);
+        tc_fence_after();
+        if (sg.list == L_RGU && first_rgu) {
+          first_rgu = false;
+          trace(p, 13, lane == 0);
+        }
+        if (ok) {
+          const uint64_t adesc = umma_desc(smem_u32(ring + (size_t)slot * p.slot_bytes), kgb, gu ? 256u : 128u);
+          if (gu) {
+            const uint64_t bd = bdesc_gu + (uint64_t)(kg * 8);   // kg * 128 bytes
+#pragma unroll
+            for (int ks = 0; ks < kGuKgStage / 2; ++ks) {
               const uint32_t acc = (kg > kg0 || ks > 0) ? 1u : 0u;
-              const uint32_t aa = a0 + (uint32_t)(2 * ks) * kgb;
-              const int kb = kg + 2 * ks;   // contraction group of the B operand
-              if (gu) {
-                const uint64_t db = umma_desc(b_addr + (uint32_t)kb * 128u, 128u, 0u);
-                umma_bf16(d0, umma_desc(aa, kgb, 256u), db, idesc, acc);
-                umma_bf16(d0 + 16u, umma_desc(aa + 128u, kgb, 256u), db, idesc, acc);
-              } else {
-                const uint64_t db = umma_desc(b_addr + (uint32_t)kb * 256u, 256u, 128u);
-                umma_bf16(d0, umma_desc(aa, kgb, 128u), db, idesc, acc);
-              }
+              const uint64_t da = adesc + (uint64_t)(ks * 512);   // 2 ks * 4096 bytes
+              const uint64_t db = bd + (uint64_t)(ks * 16);        // 2 ks * 128 bytes
+              umma_bf16_warp(d0, da, db, idesc, acc);
+              umma_bf16_warp(d0 + 16u, da + 8u, db, idesc, acc);   // up: 128 bytes on
+            }
+          } else {
+            const uint64_t bd = bdesc_dn + (uint64_t)(kg * 16);  // kg * 256 bytes
+#pragma unroll
+            for (int ks = 0; ks < kDnKgStage / 2; ++ks) {
+              const uint32_t acc = (kg > kg0 || ks > 0) ? 1u : 0u;
+              umma_bf16_warp(d0, adesc + (uint64_t)(ks * 256), bd + (uint64_t)(ks * 32), idesc, acc);
             }
           }
-          umma_commit(&empty[slot]);
-          ++s;
         }
-        umma_commit(&c->accfull[buf]);
-        ++t;
-      };
-      tc_segments(p, geo, L_SGU, 0, seg);
-      if (ok) ok = wait_flag(p, c, &c->lists_ready);
-      const int nu = ok ? *(volatile int*)&c->nu : 0;
-      tc_segments(p, geo, L_RGU, nu, seg);
-      tc_segments(p, geo, L_DN, nu, seg);
-      // every MMA of this CTA is complete before the tensor memory goes away
-      umma_commit(&c->drain);
+        umma_commit_warp(&empty[slot]);
+        ++s;
+      }
+      umma_commit_warp(&c->accfull[buf]);
+      ++t;
+    };
+    tc_segments(p, geo, L_SGU, 0, seg);
+    if (lane == 0 && ok) ok = wait_flag(p, c, &c->lists_ready);
+    ok = warp_ok(ok);
+    const int nu = ok ? *(volatile int*)&c->nu : 0;
+    tc_segments(p, geo, L_RGU, nu, seg);
+    trace(p, 14, lane == 0);
+    tc_segments(p, geo, L_DN, nu, seg);
+    trace(p, 16, lane == 0);
+    // every MMA of this CTA is complete before the tensor memory goes
+    // away, and no bulk copy still targets shared memory at exit
+    umma_commit_warp(&c->drain);
+    if (lane == 0) {
       const uint64_t t0 = globaltimer();
-      const uint32_t par = (uint32_t)(dgroup > 0 ? dgroup : 0) & 1u;   // one commit per handed-back operand
-      while (!mbar_test(&c->drain, par) && globaltimer() - t0 < p.timeout_ns) __nanosleep(64);
+      while (!mbar_test(&c->drain, ndrain & 1u) && globaltimer() - t0 < p.timeout_ns) __nanosleep(64);
+      while (b_pending && !mbar_test(&c->bfull, (nb - 1) & 1u) && globaltimer() - t0 < 2 * p.timeout_ns)
+        __nanosleep(64);
     }
     __syncwarp();
     bar_sync(kBarEnd, 5 * 32);
@@ -330,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       const uint32_t buf = t & 1u;
       if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t >> 1) & 1u);
       tc_fence_after();
+      trace(p, 20, t == 0 && tid == 0);
       uint32_t v[16], w2[16];
       tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf, v);
       tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf + 16u, w2);
@@ -352,22 +391,24 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
         }
       }
       // a block split across CTAs: publish this part; the CTA that arrives
-      // last adds every part in CTA order
+      // last adds every part in CTA order.  A part is [a0..a7 | b0..b7] of
+      // this row; only the quarters the rows and the list need move.
       const long long u0 = sg.gblk * upb, u1 = u0 + upb;
       const int c_lo = part_owner(sg.N, G, u0), c_hi = part_owner(sg.N, G, u1 - 1);
       bool complete = c_lo == c_hi;
       // part slots: a CTA's first and last segment of a list (0 / 1), the
       // routed gate/up list after the shared one (2 / 3)
       const int nsl = gu ? 4 : 2, sl0 = sg.list == L_RGU ? 2 : 0;
+      const bool q1 = R > 4;
       if (!complete) {
         const int slot = sl0 + (part_start(sg.N, G, blockIdx.x) >= u0 ? 0 : 1);
-        float* mine = (gu ? p.gpart : p.dpart) + (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16;
+        float4* mine = reinterpret_cast<float4*>((gu ? p.gpart : p.dpart) +
+                                                 (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16);
         if (live) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            mine[r] = a[r];
-            mine[8 + r] = b[r];
-          }
+          __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
+          if (q1) __stcg(mine + 1, make_float4(a[4], a[5], a[6], a[7]));
+          if (gu) __stcg(mine + 2, make_float4(b[0], b[1], b[2], b[3]));
+          if (gu && q1) __stcg(mine + 3, make_float4(b[4], b[5], b[6], b[7]));
         }
         __threadfence();
         bar_sync(kBarEpi, 4 * 32);
@@ -386,14 +427,31 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
         if (complete) {
 #pragma unroll
           for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
-          for (int cc = c_lo; cc <= c_hi; ++cc) {
-            if (part_start(sg.N, G, cc) == part_start(sg.N, G, cc + 1)) continue;   // empty range
-            const int sl = sl0 + (part_start(sg.N, G, cc) >= u0 ? 0 : 1);
-            const float* src = (gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + sl) * 128 + i) * 16;
+          // four parts in flight at a time, added in CTA order
+          for (int cb = c_lo; cb <= c_hi; cb += 4) {
+            float4 ld[4][4];
+            bool use[4];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-              a[r] += __ldcg(src + r);
-              b[r] += __ldcg(src + 8 + r);
+            for (int j = 0; j < 4; ++j) {
+              const int cc = cb + j;
+              const long long ps = part_start(sg.N, G, cc);
+              use[j] = cc <= c_hi && ps != part_start(sg.N, G, cc + 1);   // skip empty ranges
+              const int sl = sl0 + (ps >= u0 ? 0 : 1);
+              const float4* src =
+                  reinterpret_cast<const float4*>((gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + sl) * 128 + i) * 16);
+              const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+              ld[j][0] = use[j] ? __ldcg(src) : z;
+              ld[j][1] = use[j] && q1 ? __ldcg(src + 1) : z;
+              ld[j][2] = use[j] && gu ? __ldcg(src + 2) : z;
+              ld[j][3] = use[j] && gu && q1 ? __ldcg(src + 3) : z;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (!use[j]) continue;
+              a[0] += ld[j][0].x; a[1] += ld[j][0].y; a[2] += ld[j][0].z; a[3] += ld[j][0].w;
+              a[4] += ld[j][1].x; a[5] += ld[j][1].y; a[6] += ld[j][1].z; a[7] += ld[j][1].w;
+              b[0] += ld[j][2].x; b[1] += ld[j][2].y; b[2] += ld[j][2].z; b[3] += ld[j][2].w;
+              b[4] += ld[j][3].x; b[5] += ld[j][3].y; b[6] += ld[j][3].z; b[7] += ld[j][3].w;
             }
           }
         }
@@ -402,18 +460,28 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       if (!complete || !live) return;
       const int x = sg.x;
       if (gu) {
+        // SwiGLU, written as the down projection's B operand of expert entry
+        // x: [I/8][16 rows][8] bf16, row 2r = hi, 2r + 1 = lo of token row r,
+        // zero for rows that do not use the expert
         const int ch = sg.blk * 128 + i;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.actb + (size_t)x * I * 32 + (size_t)(ch >> 3) * 256) + (ch & 7);
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r) {
           const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
+          uint16_t hb = 0, lb = 0;
           if (r < R && sl >= 0) {
             float gg = a[r], uu = b[r];
             if (p.round_bf16) {
               gg = round_bf16(gg);
               uu = round_bf16(uu);
             }
-            p.act[((size_t)r * (K + 1) + sl) * I + ch] = gg / (1.0f + expf(-gg)) * uu;
+            const float act = gg / (1.0f + expf(-gg)) * uu;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(act);
+            hb = __bfloat16_as_ushort(hi);
+            lb = __bfloat16_as_ushort(__float2bfloat16_rn(act - __bfloat162float(hi)));
           }
+          dst[(2 * r) * 8] = hb;
+          dst[(2 * r + 1) * 8] = lb;
         }
       } else {
         const int h = sg.blk * 128 + i;
@@ -432,8 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     tc_segments(p, geo, L_RGU, nu, seg);
     trace(p, 7, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
-    if (tid == 0) {
+    if (tid == 0) {   // the activations are read by bulk copies (async proxy)
       __threadfence();
+      fence_proxy_async_global();
       red_release_add(&p.sync->cnt_act, 1u);
     }
     tc_segments(p, geo, L_DN, nu, seg);
@@ -445,60 +514,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     }
     tc_fence_before();
     bar_arrive(kBarEnd, 5 * 32);   // the issuer may free the tensor memory
-  } else {
-    // ======================================================= B builders
-    const int bt = tid - 4 * 32;   // 0..127
-    if (bt == 0) wait_count(p, c, &p.sync->cnt_act, ep1 * (uint32_t)G, 4u);
-    bar_sync(kBarBld, 4 * 32);
-    trace(p, 8, bt == 0);
-    int dgroup = -1, prev_x = -1;
-    auto seg = [&](const Seg& sg) {
-      if (sg.x == prev_x) return;
-      prev_x = sg.x;
-      ++dgroup;
-      if (dgroup > 0) {   // the previous operand must be released first
-        volatile int* seq = &c->mma_seq;
-        const uint64_t t0 = globaltimer();
-        while (*seq < dgroup && !c->dead) {
-          if (globaltimer() - t0 > 2 * p.timeout_ns) {
-            record_error(p, c, 7u, 4u);
-            break;
-          }
-          __nanosleep(32);
-        }
-      }
-      const int x = sg.x;
-      // layout [kg][2 row groups][8 rows][8]: row 2r = hi, 2r + 1 = lo of
-      // token row r; rows of tokens that do not use the expert are zero
-      for (int q = bt; q < geo.kgi * 8; q += 128) {
-        const int kg = q / 8, r = q % 8;
-        int sl = -1;
-        if (r < R) sl = x == 0 ? K : c->uslot[x - 1][r];
-        uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
-        if (sl >= 0 && !c->dead) {
-          const float4* src = reinterpret_cast<const float4*>(p.act + ((size_t)r * (K + 1) + sl) * I + kg * 8);
-          const float4 a = __ldcg(src), b = __ldcg(src + 1);
-          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float h0 = round_bf16(f[2 * k]), h1 = round_bf16(f[2 * k + 1]);
-            hw[k] = pack_bf16x2(h0, h1);
-            lw[k] = pack_bf16x2(f[2 * k] - h0, f[2 * k + 1] - h1);
-          }
-          hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-        uint8_t* blk = regA + (size_t)kg * 256;
-        *reinterpret_cast<uint4*>(blk + (size_t)(2 * r) * 16) = hi;
-        *reinterpret_cast<uint4*>(blk + (size_t)(2 * r + 1) * 16) = lo;
-      }
-      fence_proxy_async_smem();
-      bar_sync(kBarBld, 4 * 32);
-      if (bt == 0) *(volatile int*)&c->bld_seq = dgroup + 1;
-    };
-    tc_segments(p, geo, L_DN, nu, seg);
   }
+  // warps 4-7 have no part in the main phase
 
   // ==================================================================== tail
   bar_sync(kBarCons, kCW * 32);

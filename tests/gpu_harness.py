@@ -128,10 +128,12 @@ def compare_out(wl, got, want, what="hc_out", allow_rows_off=0, ulps=1):
     max-abs 5e-2, where an element may also differ by `ulps` bf16 spacings of
     the oracle's value: both sides round the same quantity to bf16 last, and
     at |x| >= 8 one spacing (0.0625) already exceeds 5e-2.  One layer against
-    the oracle on the same inputs: one spacing.  A chain compared end to end
-    rounds its residual streams to bf16 once per layer on both sides, and a
-    rounding that went the other way in an earlier layer moves the next
-    layer's input by a spacing: two spacings there.
+    the oracle on the same inputs: one spacing.  A chain of L layers compared
+    end to end: L spacings.  Each layer rounds the residual streams to bf16
+    once on both sides, so each may add one rounding that went the other way,
+    and the next expand carries an earlier difference on with gain at most
+    about one: its comb matrix is doubly stochastic (out_i = sum_j C_ij X_j,
+    sum_j C_ij = 1).
     allow_rows_off: for multi-layer chains compared end to end, up to this
     many rows may be excluded when they exceed the tolerance (a routing
     decision that met a near tie in an earlier layer changes that row)."""
