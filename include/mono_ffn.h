@@ -230,8 +230,45 @@ int mono_ffn_set_trace(mono_ffn_plan_t* plan, unsigned long long* buf);
  * the router-logits counter, so every CTA's bounded wait expires. */
 int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* plan, int cta);
 
+/* Router select without a plan and without allocating anything.
+ *
+ * No counterpart on the pages: their router stage lives inside the fused
+ * layer kernel.  This is a standalone variant of that stage (the router
+ * logits, sqrt(softplus) scores, selection bias, canonical top-k and the
+ * normalised, scaled weights; ds4 "v41: fuse the single-box decode glue",
+ * the router "Mega-Gate" commit), for callers that cannot allocate device
+ * memory when they need a routing decision: a serving engine that reserves
+ * all device memory up front, or code between captured graph segments that
+ * must not reach the allocator.  Its scratch is a fixed static device array,
+ * so no call allocates (no cudaMalloc, no library allocation).
+ *
+ *   n          [rows][hidden] device, bf16 (n_bf16 = 1) or fp32, the normed rows
+ *   router_w   [hidden][n_routed] fp32 device (logits = n @ router_w)
+ *   router_bias[n_routed] fp32 device, added for selection only
+ *   idx        [rows][top_k] int32 device, out: selected experts in order
+ *   w          [rows][top_k] fp32 device, out: score / max(sum, denom_clamp) * route_scale
+ *   stream     cudaStream_t (NULL = legacy default stream)
+ *
+ * Limits (the size of the static scratch): rows <= 8, n_routed <= 1024,
+ * top_k <= 16 (and <= n_routed).  Anything beyond is refused with
+ * MONO_ERR_INVALID_ARG and every reason in mono_ffn_last_error(NULL);
+ * rows == 0 is a no-op.  Asynchronous: errors of the running kernel show up
+ * on the stream.
+ *
+ * Scratch: 256 KB of partial logits, which need no initial value, and one
+ * arrival counter, which must be zero when a call starts.  It is zero from
+ * static initialisation and every call leaves it at zero.  Calls that overlap
+ * in time on one device (other streams, other threads) share the scratch and
+ * race: order them.  The first call on each device looks the scratch address
+ * up (cudaGetSymbolAddress, which may load the module); make that first call
+ * outside stream capture. */
+int mono_ffn_route_noalloc(int rows, int hidden, int n_routed, int top_k, const void* n, int n_bf16,
+                           const float* router_w, const float* router_bias, float route_scale, float denom_clamp,
+                           int* idx, float* w, void* stream);
+
 /* Every reason of the last failure on this plan (or, for plan == NULL, of
- * the last failed mono_ffn_plan call on this thread). */
+ * the last failed mono_ffn_plan or mono_ffn_route_noalloc call on this
+ * thread). */
 const char* mono_ffn_last_error(const mono_ffn_plan_t* plan);
 
 void mono_ffn_destroy(mono_ffn_plan_t* plan);

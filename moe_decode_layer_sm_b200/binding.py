@@ -20,7 +20,7 @@ ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED_ARCH", -3: "NOT_CORESIDEN
 
 SYMBOLS = ["mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
            "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_last_error",
-           "mono_ffn_destroy", "mono_ffn_abi_version", "mono_ffn_set_trace"]
+           "mono_ffn_destroy", "mono_ffn_abi_version", "mono_ffn_set_trace", "mono_ffn_route_noalloc"]
 
 
 class Config(ctypes.Structure):
@@ -78,9 +78,11 @@ def lib():
         L.mono_ffn_last_error.restype = ctypes.c_char_p
         L.mono_ffn_destroy.argtypes = [vp]
         L.mono_ffn_destroy.restype = None
+        f32 = ctypes.c_float
+        L.mono_ffn_route_noalloc.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, f32, f32, vp, vp, vp]
         for f in ("mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
                   "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_abi_version",
-                  "mono_ffn_set_trace"):
+                  "mono_ffn_set_trace", "mono_ffn_route_noalloc"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -176,3 +178,19 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def route_noalloc(n, router_w, router_bias, top_k, route_scale, denom_clamp, idx, w, stream=None):
+    """mono_ffn_route_noalloc: router select with no plan and no allocation.
+    n [rows][hidden] (bf16 or fp32), router_w [hidden][n_routed] fp32,
+    router_bias [n_routed] fp32, idx [rows][top_k] int32 and w [rows][top_k]
+    fp32 written in place; all CUDA tensors on the current device."""
+    import torch
+    rows, hidden = n.shape
+    n_routed = router_w.shape[1]
+    rc = lib().mono_ffn_route_noalloc(rows, hidden, n_routed, top_k, _ptr(n), 1 if n.dtype == torch.bfloat16 else 0,
+                                      _ptr(router_w), _ptr(router_bias), route_scale, denom_clamp, _ptr(idx), _ptr(w),
+                                      _stream(stream))
+    if rc != 0:
+        msg = lib().mono_ffn_last_error(None)
+        raise RuntimeError(f"mono_ffn_route_noalloc: {ERRORS.get(rc, rc)}: {msg.decode() if msg else ''}")

@@ -664,3 +664,5 @@ extern "C" int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* p, int cta) {
   p->fault_cta = cta;
   return MONO_OK;
 }
+
+#include "route_noalloc.cuh"

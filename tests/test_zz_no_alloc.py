@@ -1,0 +1,72 @@
+"""mono_ffn_route_noalloc (router select with no plan and no allocation)
+against the fused step's own routing: same normed rows n, same router
+weights and bias, two calls in a row.  The file name puts it last in
+collection, so it also runs after every other GPU test (the static scratch's
+arrival counter must still be zero then)."""
+
+import numpy as np
+import pytest
+
+from moe_decode_layer_sm_b200 import binding
+from synth import configs as C
+from synth import synth as S
+from tests.gpu_harness import FP32_MAX_ABS, GpuRun, routing_ok
+
+
+def _sel(wl, logits, bias):
+    lg = np.asarray(logits, np.float64)
+    sp = np.maximum(lg, 0.0) + np.log1p(np.exp(-np.abs(lg)))
+    return np.sqrt(sp) + np.asarray(bias, np.float64)[None, :]
+
+
+CASES = {
+    "tiny-fp32-r3": lambda: C.TINY_FP32.with_(rows=3),
+    "scaled-bf16-r8": lambda: C.scaled(C.FLASH_BF16_R8, seed=611),
+    "v41flash-bf16-r8": lambda: C.FLASH_BF16_R8,
+}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", list(CASES))
+def test_route_noalloc_matches_fused_step(case):
+    import torch
+    wl = CASES[case]()
+    run = GpuRun(wl)
+    run.step()
+    R, K = wl.rows, wl.top_k
+    d = S.gpu_dense(wl, 0)
+    n = run.taps[0]["n"]
+    if wl.round_bf16:
+        n = n.to(torch.bfloat16)   # the fused step's n is bf16-valued; exact
+    want_idx, want_w = run.tap(0, "idx"), run.tap(0, "w")
+    sel = _sel(wl, run.tap(0, "logits"), d["router_bias"].cpu().numpy())
+    got = []
+    for _ in range(2):   # two calls in a row on one stream
+        idx = torch.full((R, K), -1, dtype=torch.int32, device="cuda")
+        w = torch.full((R, K), -1.0, dtype=torch.float32, device="cuda")
+        binding.route_noalloc(n, d["router_w"], d["router_bias"], K, wl.route_scale, wl.denom_clamp, idx, w)
+        torch.cuda.synchronize()
+        got.append((idx.cpu().numpy(), w.cpu().numpy()))
+    for idx, w in got:
+        for r in range(R):
+            ok, exempt = routing_ok(idx[r], want_idx[r], sel[r], K)
+            assert ok, f"row {r}: noalloc {idx[r]} fused {want_idx[r]}"
+            if not exempt:
+                assert np.abs(w[r] - want_w[r]).max() <= FP32_MAX_ABS, f"row {r}: w {w[r]} vs {want_w[r]}"
+    # the same inputs give the same bytes on the second call
+    assert np.array_equal(got[0][0], got[1][0]) and np.array_equal(got[0][1], got[1][1])
+    run.close()
+
+
+def test_route_noalloc_refuses_sizes_beyond_its_scratch():
+    """Refusals happen on the host, before any CUDA call."""
+    import ctypes
+    L = binding.lib()
+    null = ctypes.c_void_p(0)
+    for rows, E, k, what in [(9, 256, 8, b"rows 9 above the scratch limit 8"),
+                             (1, 2048, 8, b"n_routed 2048 outside 1..1024"),
+                             (1, 256, 17, b"top_k 17 outside")]:
+        rc = L.mono_ffn_route_noalloc(rows, 5120, E, k, null, 1, null, null, 2.5, 1e-20, null, null, null)
+        assert rc == -1
+        assert what in L.mono_ffn_last_error(None)
+    assert L.mono_ffn_route_noalloc(0, 5120, 256, 8, null, 1, null, null, 2.5, 1e-20, null, null, null) == 0
