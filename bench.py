@@ -176,12 +176,12 @@ def run_reference(args):
 # --------------------------------------------------------------- GPU path --
 
 TRACE_NAMES = ["start", "mix published", "mix totals seen", "n ready", "logits published", "lists ready",
-               "shared gate/up done", "routed gate/up done", "activations seen", "down done", "end",
+               "shared gate/up done", "routed gate/up done", "1st down expert ready", "down done", "end",
                "producer saw lists", "producer issued all", "issuer: 1st routed stage", "issuer: routed issued",
                "issuer: 1st down operand", "issuer: all issued", "(unused)", "producer: 1st routed",
                "producer: 1st down", "epilogue: 1st shared", "ctl: logits complete", "ctl: top-k done",
-               "pre/post ready", "collapse done", "router: dots done", "top-k: loads done", "collapse: sums done",
-               "mix: inputs in smem"]
+               "pre/post ready", "collapse: all slices", "router: dots done", "top-k: loads done",
+               "collapse: slice out", "mix: inputs in smem"]
 TRACE_POINTS = 32
 
 

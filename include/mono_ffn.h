@@ -154,7 +154,9 @@ enum {
   MONO_STAGE_LOGITS = 2,  /* router logits of all CTAs */
   MONO_STAGE_LISTS = 3,   /* this CTA's top-k / work lists */
   MONO_STAGE_ACT = 4,     /* SwiGLU activations of all CTAs */
-  MONO_STAGE_RING = 5     /* a weight-ring stage (TMA completion or slot release) */
+  MONO_STAGE_RING = 5,    /* a weight-ring stage (TMA completion or slot release) */
+  MONO_STAGE_Y = 6,       /* expert outputs of all CTAs (tensor-core kernel) */
+  MONO_STAGE_COLLAPSE = 7 /* collapsed h-slices of all CTAs */
 };
 
 typedef struct {
@@ -212,15 +214,16 @@ int mono_ffn_get_info(const mono_ffn_plan_t* plan, mono_ffn_info* info);
  * at its stage boundaries to buf[(l * grid + cta) * 32 + point]:
  * 0 start, 1 mix partials published, 2 mix totals seen, 3 n ready,
  * 4 router logits published, 5 top-k lists ready, 6 shared gate/up done,
- * 7 routed gate/up done, 8 all activations seen, 9 down projections done,
+ * 7 routed gate/up done, 8 activations seen (tensor-core kernel: the first
+ * down expert's), 9 down projections done,
  * 10 end, 11 producer saw the lists, 12 producer issued every copy;
  * tensor-core kernel also: 13 first routed gate/up stage arrived, 14 routed
  * gate/up MMAs issued, 15 first down operand ready, 16 every MMA issued,
  * 17 (unused), 18 first routed copy issued, 19 first down
  * copy issued, 20 first shared gate/up tile read; both: 21 logits counter
- * complete, 22 top-k done, 23 pre/post ready, 24 collapse done, 25 router
- * dot products done, 26 top-k inputs loaded, 27 collapse sums done, 28 mix
- * inputs in shared memory.
+ * complete, 22 top-k done, 23 pre/post ready, 24 every CTA's collapsed
+ * slice seen, 25 router dot products done, 26 top-k inputs loaded, 27 this
+ * CTA's collapsed slice published, 28 mix inputs in shared memory.
  * The tensor-core kernel stores its SM id (not a time) at point 31.
  * Points a kernel does not reach stay as they were.
  * NULL turns it off (the default). */

@@ -321,13 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
 
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, ep1);
+    control_warps(p, c, ep1, true);
     return;
   }
 
   // ================================================ compute warps from here
   const int ctid = tid;   // 0..255
-  collapse_norm<false>(p, c, regA);
+  collapse_norm<false>(p, c, regA, ep1);
   const void* n_s = regA;
   trace(p, 3, ctid == 0);
   router_logits<false>(p, c, regA);

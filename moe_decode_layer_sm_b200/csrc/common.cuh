@@ -38,14 +38,15 @@ constexpr int kCtlWarps = 2;
 constexpr int kThreads = 12 * 32;                      // 384: 12 warps leave 168 registers a thread
 constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // named barriers: prologue (compute + control), compute, control, epilogue
-// warps 0-3, end (epilogue warps + the issuer warp)
-constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarEnd = 6;
+// warps 0-3, routing hand-over (compute + control), end (epilogue warps + the
+// issuer warp)
+constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6;
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
 
 enum WType { W_F32 = 0, W_BF16 = 1, W_FP8 = 2, W_FP4 = 3 };
 
 struct SyncBlock {   // one per layer slot, 64 bytes
-  uint32_t epoch, cnt_mix, cnt_logit, cnt_act, cnt_done, cnt_y, pad[10];
+  uint32_t epoch, cnt_mix, cnt_logit, cnt_act, cnt_done, cnt_y, cnt_a, pad[9];
 };
 struct ErrBlock {
   uint32_t abort, code, stage, cta, layer, pad[11];
@@ -89,7 +90,11 @@ struct Params {
   float* mix_part;   // [R*25][G] output-major partials of the mix
   float* logits;     // [R][E]
   float* act;        // [R][K+1][I]
+  void* abuf;        // [R][H] collapsed rows a (bf16 when rounded, else fp32), one h-slice per CTA
+  float* sq_part;    // [R][G] per-CTA partial sums of a^2
   float* yp;         // tensor-core kernel: [R][K+1][H] weighted expert outputs
+  uint32_t* xready;  // tensor-core kernel: [R*K+1] finished gate/up blocks per expert entry (0 between steps)
+  int n_xready;
   uint8_t* actb;     // tensor-core kernel: [R*K+1][I/8][16][8] bf16 down-projection B operands
   float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks
   float* dpart;      // tensor-core kernel: [G][2][128][16] partial down tiles
@@ -367,18 +372,29 @@ __device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
   const int E = p.E, K = p.K;
   float score[NQ];
   uint32_t key[NQ];
+  // every load first (a store in between would order them one by one)
+  float lg[NQ], bs[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = lane + 32 * q;
+    lg[q] = (e < E && !c->dead) ? __ldcg(p.logits + (size_t)r * E + e) : 0.f;
+    bs[q] = e < E ? __ldg(p.bias + e) : 0.f;
+  }
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
     const int e = lane + 32 * q;
     score[q] = 0.f;
     key[q] = 0u;
     if (e < E) {
-      const float lg = c->dead ? 0.f : __ldcg(p.logits + (size_t)r * E + e);
-      if (blockIdx.x == 0 && p.taps.logits) p.taps.logits[(size_t)r * E + e] = lg;
-      const float sp = fmaxf(lg, 0.f) + log1pf(expf(-fabsf(lg)));
+      const float sp = fmaxf(lg[q], 0.f) + log1pf(expf(-fabsf(lg[q])));
       score[q] = sqrtf(sp);
-      key[q] = ord_key(score[q] + __ldg(p.bias + e));
+      key[q] = ord_key(score[q] + bs[q]);
     }
+  }
+  if (blockIdx.x == 0 && p.taps.logits) {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      if (lane + 32 * q < E) p.taps.logits[(size_t)r * E + lane + 32 * q] = lg[q];
   }
   trace(p, 26, r == 0 && lane == 0);
   uint32_t taken = 0u;
@@ -452,48 +468,82 @@ __device__ __forceinline__ int pre_tid() {
   return t < kCW * 32 ? t : t - (kCtlWarp0 - kCW) * 32;
 }
 
+// Shared-memory offsets of the prologue's staging areas inside regA: the
+// CTA's slice of mix_w [S][nh][24], its slice of the residual streams
+// [R][S][nh] (kept until the collapse has used it), then room for the mix
+// partials of every CTA.
+struct PreLayout {
+  int h0, h1, nh;
+  size_t ws, xs, parts;
+  __device__ PreLayout(const Params& p) {
+    Walk::dn_range(p, h0, h1);
+    nh = h1 - h0;
+    ws = 0;
+    xs = ws + (size_t)kS * nh * kMixC * 4;
+    parts = align_up(xs + (size_t)p.R * kS * nh * 4, 16);
+  }
+};
+
 // A2 (every CTA, on the h-range it also owns in the tail): materialise this
 // layer's residual streams from the previous layer's pending post/comb expand
 // (or read hc_in), then the partial mix products and square sums.  A3: wait
 // for every CTA's partials, reduce them in one fixed order in every CTA, and
-// derive rho, mix, pre and post.
+// derive rho, mix, pre and post.  Loads are issued all at once (cp.async /
+// unrolled) so that each stage costs one memory round trip.
 __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep1) {
   const int R = p.R, H = p.H, G = p.G;
   const int ptid = pre_tid(), pwarp = ptid >> 5, lane = threadIdx.x & 31;
   const int nout = R * kMixP;
+  const PreLayout L(p);
+  const int h0 = L.h0, nh = L.nh;
+  float* ws = reinterpret_cast<float*>(regA + L.ws);   // [S][nh][24] slice of mix_w
+  float* xs = reinterpret_cast<float*>(regA + L.xs);   // [R][S][nh]
   {
-    int h0, h1;
-    Walk::dn_range(p, h0, h1);
-    const int nh = h1 - h0;
-    float* ws = reinterpret_cast<float*>(regA);          // [S][nh][24] slice of mix_w
-    float* xs = ws + (size_t)kS * nh * kMixC;            // [R][S][nh]
+    // mix_w rows s * H + h0 .. + nh are contiguous: 16-byte asynchronous copies
     const int seg4 = nh * (kMixC / 4);
     for (int i = ptid; i < kS * seg4; i += kPreThreads) {
       const int sgm = i / seg4, j = i % seg4;
-      reinterpret_cast<float4*>(ws)[i] =
-          __ldg(reinterpret_cast<const float4*>(p.mix_w + ((size_t)sgm * H + h0) * kMixC) + j);
+      cp_async16(reinterpret_cast<float4*>(ws) + i, reinterpret_cast<const float4*>(p.mix_w + ((size_t)sgm * H + h0) * kMixC) + j);
     }
+    cp_async_commit();
     const float* ppost = p.pend_in;
     const float* pcomb = p.pend_in + R * kS;
     const float* py = p.pend_in + R * kS + R * kS * kS;
-    for (int i = ptid; i < R * kS * nh; i += kPreThreads) {
-      const int r = i / (kS * nh), sg = (i / nh) % kS, h = h0 + i % nh;
-      float v;
-      if (p.first) {
-        v = load_x(p.x_prev, ((size_t)r * kS + sg) * H + h, p.hc_bf16);
-      } else {
-        // the previous layer's deferred post: X_s = sum_j comb_sj Xprev_j + post_s y
-        float acc = 0.f;
+    const int nx = R * kS * nh;
+    constexpr int kXU = 4;   // elements per thread in flight
+    for (int i0 = ptid; i0 < nx; i0 += kXU * kPreThreads) {
+      float v[kXU];
 #pragma unroll
-        for (int j = 0; j < kS; ++j)
-          acc = fmaf(pcomb[(r * kS + sg) * kS + j], load_x(p.x_prev, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
-        acc = fmaf(ppost[r * kS + sg], py[(size_t)r * H + h], acc);
-        v = p.hc_bf16 ? round_bf16(acc) : acc;
-        store_x(p.xbuf, ((size_t)r * kS + sg) * H + h, v, p.hc_bf16);
+      for (int u = 0; u < kXU; ++u) {
+        const int i = i0 + u * kPreThreads;
+        v[u] = 0.f;
+        if (i < nx) {
+          const int r = i / (kS * nh), sg = (i / nh) % kS, h = h0 + i % nh;
+          if (p.first) {
+            v[u] = load_x(p.x_prev, ((size_t)r * kS + sg) * H + h, p.hc_bf16);
+          } else {
+            // the previous layer's deferred post: X_s = sum_j comb_sj Xprev_j + post_s y
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < kS; ++j)
+              acc = fmaf(pcomb[(r * kS + sg) * kS + j], load_x(p.x_prev, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
+            acc = fmaf(ppost[r * kS + sg], py[(size_t)r * H + h], acc);
+            v[u] = p.hc_bf16 ? round_bf16(acc) : acc;
+          }
+        }
       }
-      xs[i] = v;
-      if (p.taps.x) p.taps.x[((size_t)r * kS + sg) * H + h] = v;
+#pragma unroll
+      for (int u = 0; u < kXU; ++u) {
+        const int i = i0 + u * kPreThreads;
+        if (i < nx) {
+          const int r = i / (kS * nh), sg = (i / nh) % kS, h = h0 + i % nh;
+          if (!p.first) store_x(p.xbuf, ((size_t)r * kS + sg) * H + h, v[u], p.hc_bf16);
+          xs[i] = v[u];
+          if (p.taps.x) p.taps.x[((size_t)r * kS + sg) * H + h] = v[u];
+        }
+      }
     }
+    cp_async_wait_all();
     bar_sync(kBarPre, kPreThreads);
     trace(p, 28, ptid == 0);
     // outputs o = r * 25 + col (col 24: the square sum), each split in P parts
@@ -527,16 +577,19 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
   bar_sync(kBarPre, kPreThreads);
   trace(p, 2, ptid == 0);
   {
-    // lane-strided sums then a butterfly across the warp, the same order in
-    // every CTA
-    float* parts = reinterpret_cast<float*>(regA);
-    const int cap = p.regA_bytes / (int)sizeof(float) / G;   // outputs per pass
+    // every CTA's partials into shared memory at once (behind the slices,
+    // which the collapse still needs), then lane-strided sums and a butterfly
+    // across the warp: the same order in every CTA
+    float* parts = reinterpret_cast<float*>(regA + L.parts);
+    const int cap = (int)(((size_t)p.regA_bytes - L.parts) / sizeof(float) / G);   // outputs per pass
     for (int o0 = 0; o0 < nout; o0 += cap) {
       const int no = min(cap, nout - o0);
       const int n4 = no * G / 4;   // G * 4 bytes is a multiple of 16 (the plan keeps G % 4 == 0)
       const float4* src = reinterpret_cast<const float4*>(p.mix_part + (size_t)o0 * G);
-      for (int i = ptid; i < n4; i += kPreThreads)
-        reinterpret_cast<float4*>(parts)[i] = c->dead ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(src + i);
+      if (!c->dead)
+        for (int i = ptid; i < n4; i += kPreThreads) cp_async16(reinterpret_cast<float4*>(parts) + i, src + i);
+      cp_async_commit();
+      cp_async_wait_all();
       bar_sync(kBarPre, kPreThreads);
       for (int o = pwarp; o < no; o += kPreThreads / 32) {
         float acc = 0.f;
@@ -569,10 +622,12 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
   }
 }
 
-// Control warps: Sinkhorn of the comb logits (16 threads per row), then, once
-// every CTA's router logits are out, the canonical top-k of each row and the
-// list of unique routed experts with their rows and act slots.
-__device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1) {
+// Control warps: Sinkhorn of the comb logits (16 threads per row), then the
+// canonical top-k of each row once every CTA's router logits are out (here
+// when ctl_topk; otherwise the compute warps do it in route_rows and hand
+// over at the routing barrier), then the list of unique routed experts with
+// their rows and act slots.
+__device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1, bool ctl_topk) {
   const int R = p.R, E = p.E, K = p.K, G = p.G;
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kCtlWarp0;
   const int ct = threadIdx.x - kCtlWarp0 * 32;
@@ -600,20 +655,27 @@ __device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1) {
       }
     }
   }
-  if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
-  trace(p, 21, ct == 0);
-  bar_sync(kBarCtl, kCtlWarps * 32);
-  for (int r = cw; r < R; r += kCtlWarps) {
-    if (E <= 32) topk_row<1>(p, c, r);
-    else if (E <= 64) topk_row<2>(p, c, r);
-    else if (E <= 128) topk_row<4>(p, c, r);
-    else if (E <= 256) topk_row<8>(p, c, r);
-    else if (E <= 512) topk_row<16>(p, c, r);
-    else topk_row<32>(p, c, r);
+  if (ctl_topk) {
+    // the top-k rows here, two warps over the rows
+    if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
+    trace(p, 21, ct == 0);
+    bar_sync(kBarCtl, kCtlWarps * 32);
+    for (int r = cw; r < R; r += kCtlWarps) {
+      if (E <= 32) topk_row<1>(p, c, r);
+      else if (E <= 64) topk_row<2>(p, c, r);
+      else if (E <= 128) topk_row<4>(p, c, r);
+      else if (E <= 256) topk_row<8>(p, c, r);
+      else if (E <= 512) topk_row<16>(p, c, r);
+      else topk_row<32>(p, c, r);
+    }
+    for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
+    bar_sync(kBarCtl, kCtlWarps * 32);
+    trace(p, 22, ct == 0);
+  } else {
+    for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
+    // the compute warps' top-k rows (route_rows) are in c->idx / c->wt after this
+    bar_sync(kBarRoute, kPreThreads);
   }
-  for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
-  bar_sync(kBarCtl, kCtlWarps * 32);
-  trace(p, 22, ct == 0);
   for (int i = ct; i < R * K; i += kCtlWarps * 32) {
     const int e = c->idx[i / K][i % K];
     if (e >= 0 && e < E) atomicOr(&c->bm[e >> 5], 1u << (e & 31));
@@ -672,121 +734,169 @@ __device__ __forceinline__ size_t n_off(int r, int h, int H, bool bf) {
 
 // Collapse a = sum_s pre_s X_s (-> bf16), weighted RMSNorm n = a / sqrt(mean
 // a^2 + eps) * norm_w (-> bf16), into shared memory; compute warps only.
+// Each CTA collapses its own h-slice from the residual streams it staged for
+// the mix, publishes it with its partial sum of a^2, and after a grid stage
+// copies every slice in (one round trip) and normalises in place.
 template <bool CANON>
-__device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA) {
-  const int R = p.R, H = p.H, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
+__device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep1) {
+  const int R = p.R, H = p.H, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
   const bool nbf = CANON || p.round_bf16;
-  const void* X = p.first ? p.x_prev : (const void*)p.xbuf;
-  const int H8 = H / 8;
-  float sq[kMaxR];
+  const bool abf = p.round_bf16 != 0;   // a is bf16-valued when rounded
+  const PreLayout L(p);
+  const int h0 = L.h0, nh = L.nh;
+  {
+    const float* xs = reinterpret_cast<const float*>(regA + L.xs);
+    float sq[kMaxR];
 #pragma unroll
-  for (int r = 0; r < kMaxR; ++r) sq[r] = 0.f;
-#pragma unroll 2
-  for (int i = ctid; i < R * H8; i += kCW * 32) {
-    const int r = i / H8, h = (i % H8) * 8;
-    float xv[kS][8];
-#pragma unroll
-    for (int sg = 0; sg < kS; ++sg) load_hc8(X, ((size_t)r * kS + sg) * H + h, p.hc_bf16, xv[sg]);
-    float a[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int r = 0; r < kMaxR; ++r) sq[r] = 0.f;
+    for (int i = ctid; i < R * nh; i += kCW * 32) {
+      const int r = i / nh, hh = i % nh;
       float acc = 0.f;
 #pragma unroll
-      for (int sg = 0; sg < kS; ++sg) acc = fmaf(c->pre[r][sg], xv[sg][k], acc);
-      a[k] = p.round_bf16 ? round_bf16(acc) : acc;
+      for (int sg = 0; sg < kS; ++sg) acc = fmaf(c->pre[r][sg], xs[(r * kS + sg) * nh + hh], acc);
+      const float a = abf ? round_bf16(acc) : acc;
+      store_x(p.abuf, (size_t)r * H + h0 + hh, a, abf);
+#pragma unroll
+      for (int r2 = 0; r2 < kMaxR; ++r2)
+        if (r2 == r) sq[r2] = fmaf(a, a, sq[r2]);
     }
-    float q = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) q = fmaf(a[k], a[k], q);
-#pragma unroll
-    for (int r2 = 0; r2 < kMaxR; ++r2)
-      if (r2 == r) sq[r2] += q;
-    if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
-    else store8(regA, (size_t)r * H + h, nbf, a);
+    for (int r = 0; r < kMaxR; ++r) {
+      const float v = warp_sum(sq[r]);
+      if (lane == 0) c->sq[warp][r] = v;
+    }
+    bar_sync(kBarCons, kCW * 32);
+    if (ctid < R) {
+      float t = 0.f;
+      for (int w = 0; w < kCW; ++w) t += c->sq[w][ctid];
+      p.sq_part[(size_t)ctid * G + blockIdx.x] = t;
+    }
+    bar_sync(kBarCons, kCW * 32);
+    if (ctid == 0) {
+      __threadfence();
+      red_release_add(&p.sync->cnt_a, 1u);
+    }
   }
   trace(p, 27, ctid == 0);
   if (CANON) {
-    // rows R..7 of the B operand are zero
+    // rows R..7 of the B operand are zero (the staging areas are dead now)
+    const int H8 = H / 8;
     for (int i = ctid; i < (8 - R) * H8; i += kCW * 32) {
       const int r = R + i / H8, h = (i % H8) * 8;
       *reinterpret_cast<uint4*>(regA + n_off<true>(r, h, H, true)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-#pragma unroll
-  for (int r = 0; r < kMaxR; ++r) {
-    float v = warp_sum(sq[r]);
-    if (lane == 0) c->sq[warp][r] = v;
-  }
+  if (ctid == 0) wait_count(p, c, &p.sync->cnt_a, ep1 * (uint32_t)G, 7u);
   bar_sync(kBarCons, kCW * 32);
-  trace(p, 24, threadIdx.x == 0);
-  if (ctid < R) {
-    float t = 0.f;
-    for (int w = 0; w < kCW; ++w) t += c->sq[w][ctid];
-    c->inv[ctid] = 1.0f / sqrtf(t / (float)H + p.rms_eps);
-  }
-  bar_sync(kBarCons, kCW * 32);
-#pragma unroll 2
-  for (int i = ctid; i < R * H8; i += kCW * 32) {
-    const int r = i / H8, h = (i % H8) * 8;
-    float a[8], w[8];
-    if (CANON) load8(regA + n_off<true>(r, h, H, true), 0, true, a);
-    else load8(regA, (size_t)r * H + h, nbf, a);
-    load_hc8(p.norm_w, h, p.norm_bf16, w);
-    const float inv = c->inv[r];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float v = a[k] * inv * w[k];
-      a[k] = p.round_bf16 ? round_bf16(v) : v;
+  trace(p, 24, ctid == 0);
+  // every slice of a into the n area, 16 bytes at a time
+  if (!c->dead) {
+    if (abf) {
+      const int H8 = H / 8;
+      for (int i = ctid; i < R * H8; i += kCW * 32) {
+        const int r = i / H8, h = (i % H8) * 8;
+        cp_async16(regA + n_off<CANON>(r, h, H, true), reinterpret_cast<const uint16_t*>(p.abuf) + (size_t)r * H + h);
+      }
+    } else {   // fp32 a, row-major fp32 n (CUDA-core kernel only)
+      const int H4 = H / 4;
+      for (int i = ctid; i < R * H4; i += kCW * 32)
+        cp_async16(regA + (size_t)i * 16, reinterpret_cast<const float*>(p.abuf) + (size_t)i * 4);
     }
-    if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
-    else store8(regA, (size_t)r * H + h, nbf, a);
-    if (blockIdx.x == 0 && p.taps.n) {
+  }
+  cp_async_commit();
+  // meanwhile: every CTA's a^2 partials, summed in the same order everywhere
+  if (warp < R) {
+    float t = 0.f;
+    for (int m = lane; m < G; m += 32) t += c->dead ? 0.f : __ldcg(p.sq_part + (size_t)warp * G + m);
+    t = warp_sum(t);
+    if (lane == 0) c->inv[warp] = 1.0f / sqrtf(t / (float)H + p.rms_eps);
+  }
+  cp_async_wait_all();
+  bar_sync(kBarCons, kCW * 32);
+  // n = a * inv * norm_w, in place: one norm_w load per 8 columns, all rows
+  {
+    const int H8 = H / 8;
+    constexpr int kNU = 4;
+    for (int i0 = ctid; i0 < H8; i0 += kNU * kCW * 32) {
+      float w[kNU][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) p.taps.n[(size_t)r * H + h + k] = a[k];
+      for (int u = 0; u < kNU; ++u) {
+        const int i = i0 + u * kCW * 32;
+        if (i < H8) load_hc8(p.norm_w, (size_t)i * 8, p.norm_bf16, w[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kNU; ++u) {
+        const int i = i0 + u * kCW * 32;
+        if (i >= H8) continue;
+        const int h = i * 8;
+        for (int r = 0; r < R; ++r) {
+          float a[8];
+          if (CANON) load8(regA + n_off<true>(r, h, H, true), 0, true, a);
+          else load8(regA, (size_t)r * H + h, nbf, a);
+          const float inv = c->inv[r];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float v = a[k] * inv * w[u][k];
+            a[k] = p.round_bf16 ? round_bf16(v) : v;
+          }
+          if (CANON) store8(regA + n_off<true>(r, h, H, true), 0, true, a);
+          else store8(regA, (size_t)r * H + h, nbf, a);
+          if (blockIdx.x == 0 && p.taps.n) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) p.taps.n[(size_t)r * H + h + k] = a[k];
+          }
+        }
+      }
     }
   }
   bar_sync(kBarCons, kCW * 32);
 }
 
-// Router logits of this CTA's experts (two rows of router_t at a time), then
-// the CTA's arrival at the logits counter; compute warps only.
+// Router logits of this CTA's experts (two rows of router_t at a time; each
+// thread's share of both rows is loaded at once), then the CTA's arrival at
+// the logits counter; compute warps only.
 template <bool CANON>
 __device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
   const int R = p.R, H = p.H, E = p.E, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
   const bool nbf = CANON || p.round_bf16;
   const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
+  constexpr int kRq = 5;                  // float4 per thread and row per pass
+  constexpr int kSpan = kRq * kCW * 32 * 4;   // columns per pass (5120)
   for (int e = e0; e < e1; e += 2) {
     const bool two = e + 1 < e1;
     const float* w0 = p.router_t + (size_t)e * H;
     const float* w1 = two ? w0 + H : w0;
-    float a0[kMaxR], a1[kMaxR];
+    for (int hb = 0; hb < H; hb += kSpan) {
+      float4 v0[kRq], v1[kRq];
 #pragma unroll
-    for (int r = 0; r < kMaxR; ++r) { a0[r] = 0.f; a1[r] = 0.f; }
-#pragma unroll 4
-    for (int h = ctid * 4; h < H; h += kCW * 32 * 4) {
-      const float4 v0 = __ldg(reinterpret_cast<const float4*>(w0 + h));
-      const float4 v1 = __ldg(reinterpret_cast<const float4*>(w1 + h));
+      for (int q = 0; q < kRq; ++q) {
+        const int h = hb + (ctid + q * kCW * 32) * 4;
+        v0[q] = h < H ? __ldg(reinterpret_cast<const float4*>(w0 + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v1[q] = h < H ? __ldg(reinterpret_cast<const float4*>(w1 + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      // one row at a time (a rolled loop keeps this code small)
+      for (int r = 0; r < R; ++r) {
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-      for (int r = 0; r < kMaxR; ++r) {
-        if (r < R) {
-          float nv[4];
-          if (nbf) load_vec<4, true>(n_s + n_off<CANON>(r, h, H, true), 0, nv);
-          else load_vec<4, false>(n_s + n_off<CANON>(r, h, H, false), 0, nv);
-          a0[r] = fmaf(v0.x, nv[0], fmaf(v0.y, nv[1], fmaf(v0.z, nv[2], fmaf(v0.w, nv[3], a0[r]))));
-          a1[r] = fmaf(v1.x, nv[0], fmaf(v1.y, nv[1], fmaf(v1.z, nv[2], fmaf(v1.w, nv[3], a1[r]))));
+        for (int q = 0; q < kRq; ++q) {
+          const int h = hb + (ctid + q * kCW * 32) * 4;
+          if (h < H) {
+            float nv[4];
+            if (nbf) load_vec<4, true>(n_s + n_off<CANON>(r, h, H, true), 0, nv);
+            else load_vec<4, false>(n_s + n_off<CANON>(r, h, H, false), 0, nv);
+            a0 = fmaf(v0[q].x, nv[0], fmaf(v0[q].y, nv[1], fmaf(v0[q].z, nv[2], fmaf(v0[q].w, nv[3], a0))));
+            a1 = fmaf(v1[q].x, nv[0], fmaf(v1[q].y, nv[1], fmaf(v1[q].z, nv[2], fmaf(v1[q].w, nv[3], a1))));
+          }
+        }
+        a0 = warp_sum(a0);
+        a1 = warp_sum(a1);
+        if (lane == 0) {
+          c->sq[warp][r] = (hb == 0 ? 0.f : c->sq[warp][r]) + a0;
+          c->sq2[warp][r] = (hb == 0 ? 0.f : c->sq2[warp][r]) + a1;
         }
       }
     }
     trace(p, 25, ctid == 0 && e == e0);
-#pragma unroll
-    for (int r = 0; r < kMaxR; ++r) {
-      const float v0 = warp_sum(a0[r]);
-      const float v1 = warp_sum(a1[r]);
-      if (lane == 0) {
-        c->sq[warp][r] = v0;
-        c->sq2[warp][r] = v1;
-      }
-    }
     bar_sync(kBarCons, kCW * 32);
     if (ctid < 2 * R) {
       const int r = ctid % R, which = ctid / R;
@@ -805,6 +915,26 @@ __device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
   trace(p, 4, ctid == 0);
 }
 
+// A6 on the compute warps, one row per warp: wait for every CTA's logits,
+// then the canonical top-k and weights of each row; the control warps take
+// over (expert lists) at the routing barrier.
+__device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1) {
+  const int R = p.R, E = p.E, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
+  bar_sync(kBarCons, kCW * 32);
+  trace(p, 21, threadIdx.x == 0);
+  for (int r = warp; r < R; r += kCW) {
+    if (E <= 32) topk_row<1>(p, c, r);
+    else if (E <= 64) topk_row<2>(p, c, r);
+    else if (E <= 128) topk_row<4>(p, c, r);
+    else if (E <= 256) topk_row<8>(p, c, r);
+    else if (E <= 512) topk_row<16>(p, c, r);
+    else topk_row<32>(p, c, r);
+  }
+  trace(p, 22, threadIdx.x == 0);
+  bar_sync(kBarRoute, kPreThreads);
+}
+
 // Tail on the CTA's h-range: y = bf16(routed + shared) from yfun(r, h), then
 // out_i = sum_j comb_ij X_j + post_i y (last layer) or the pending state for
 // the next layer's opening expand; compute warps only.
@@ -818,6 +948,10 @@ __device__ void tail(const Params& p, Ctl* c, YF yfun) {
   float* pend_y = p.pend_out + R * kS + R * kS * kS;
   for (int i = ctid; i < R * nh; i += kCW * 32) {
     const int r = i / nh, h = h0 + i % nh;
+    // all loads (the residual streams and the expert outputs) before any store
+    float xv[kS];
+#pragma unroll
+    for (int j = 0; j < kS; ++j) xv[j] = p.last ? load_x_cg(X, ((size_t)r * kS + j) * H + h, p.hc_bf16) : 0.f;
     float y = c->dead ? 0.f : yfun(r, h);
     if (p.round_bf16) y = round_bf16(y);
     if (p.taps.y) p.taps.y[(size_t)r * H + h] = y;
@@ -828,8 +962,7 @@ __device__ void tail(const Params& p, Ctl* c, YF yfun) {
       for (int si = 0; si < kS; ++si) {
         float acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < kS; ++j)
-          acc = fmaf(c->comb[r][si * kS + j], load_x_cg(X, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
+        for (int j = 0; j < kS; ++j) acc = fmaf(c->comb[r][si * kS + j], xv[j], acc);
         acc = fmaf(c->post[r][si], y, acc);
         store_x(p.hc_out, ((size_t)r * kS + si) * H + h, acc, p.hc_bf16);
       }
@@ -844,6 +977,8 @@ __device__ __forceinline__ void finish_step(const Params& p, Ctl* c, uint32_t ep
     __threadfence();
     const uint32_t old = atomicAdd(&p.sync->cnt_done, 1u);
     if (old == ep1 * (uint32_t)p.G - 1u) {
+      // every CTA is past its last read of the per-expert counters
+      for (int i = 0; i < p.n_xready; ++i) p.xready[i] = 0u;
       __threadfence();
       atomicAdd(&p.sync->epoch, 1u);
     }

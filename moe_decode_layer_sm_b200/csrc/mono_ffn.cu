@@ -41,6 +41,8 @@ struct mono_ffn_plan_s {
   long long gu_estride = 0, dn_estride = 0;
   std::vector<LayerSlot> layers;
   float* mix_part = nullptr;
+  void* abuf = nullptr;
+  float* sq_part = nullptr;
   float* logits = nullptr;
   float* act = nullptr;
   float* yp = nullptr;
@@ -48,6 +50,7 @@ struct mono_ffn_plan_s {
   float* gpart = nullptr;
   float* dpart = nullptr;
   uint32_t* gcnt = nullptr;
+  uint32_t* xready = nullptr;
   uint32_t* dcnt = nullptr;
   size_t gcnt_n = 0, dcnt_n = 0;
   std::vector<float*> pend;
@@ -220,6 +223,8 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
   }
   for (float* q : p->pend) cudaFree(q);
   cudaFree(p->mix_part);
+  cudaFree(p->abuf);
+  cudaFree(p->sq_part);
   cudaFree(p->logits);
   cudaFree(p->act);
   cudaFree(p->yp);
@@ -227,6 +232,7 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
   cudaFree(p->gpart);
   cudaFree(p->dpart);
   cudaFree(p->gcnt);
+  cudaFree(p->xready);
   cudaFree(p->dcnt);
   cudaFree(p->xbuf[0]);
   cudaFree(p->xbuf[1]);
@@ -288,7 +294,8 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   const int H = cfg.hidden, I = cfg.inter, E = cfg.n_routed, K = cfg.top_k, RM = cfg.max_rows;
 
   // bf16 experts run on the tensor cores when the shapes allow it
-  p->tc = dt == MONO_BF16 && H % 128 == 0 && I % 128 == 0;   // whole 128-row blocks and 128-wide K units
+  // whole 128-row blocks and 128-wide K units; n is the bf16 B operand
+  p->tc = dt == MONO_BF16 && cfg.round_bf16 && H % 128 == 0 && I % 128 == 0;
   // chunking of the packed rows
   const int gu_target = dt == MONO_F32 ? 256 : dt == MONO_BF16 ? 512 : 1024;
   const int dn_target = dt == MONO_F32 ? 512 : dt == MONO_BF16 ? 1024 : 2048;
@@ -318,8 +325,10 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   // of at least one row each, for the prefetch of the next expert)
   size_t regA = std::max<size_t>((size_t)RM * H * (cfg.round_bf16 ? 2 : 4), (size_t)RM * I * 4);
   regA = std::max<size_t>(regA, (size_t)2 * I * 4 + 256);
-  regA = std::max<size_t>(regA, ((size_t)kS * p->ymax * kMixC + (size_t)RM * kS * p->ymax) * 4);
-  regA = std::max<size_t>(regA, (size_t)p->G * kMixP * 4);
+  // prologue staging: the mix_w and residual-stream slices, then at least
+  // one row's mix partials of every CTA
+  regA = std::max<size_t>(regA, align_up(((size_t)kS * p->ymax * kMixC + (size_t)RM * kS * p->ymax) * 4, 16) +
+                                    (size_t)p->G * kMixP * 4);
   if (p->tc) {
     regA = std::max<size_t>(regA, (size_t)H * 16);   // n: 8 rows of bf16
     regA = std::max<size_t>(regA, (size_t)I * 32);   // down B: 16 rows (hi/lo of 8 token rows)
@@ -363,6 +372,8 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     if (!rc) rc = dalloc(p, &l.dn, (size_t)(E + 1) * p->dn_estride, &p->packed_bytes);
   }
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->abuf, (size_t)RM * H * 4, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->sq_part, (size_t)RM * p->G * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->act, (size_t)RM * (K + 1) * I * 4, &p->scratch_bytes);
   if (!rc && p->tc) rc = dalloc(p, &p->yp, (size_t)RM * (K + 1) * H * 4, &p->scratch_bytes);
@@ -372,6 +383,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->gcnt_n = (size_t)(RM * K + 2) * (I / 128);
   p->dcnt_n = (size_t)(RM * K + 2) * (H / 128);
   if (!rc && p->tc) rc = dalloc(p, &p->gcnt, p->gcnt_n * 4, &p->scratch_bytes);
+  if (!rc && p->tc) rc = dalloc(p, &p->xready, (size_t)(RM * K + 1) * 4, &p->scratch_bytes);
   if (!rc && p->tc) rc = dalloc(p, &p->dcnt, p->dcnt_n * 4, &p->scratch_bytes);
   p->pend.assign(cfg.n_layers, nullptr);
   for (int l = 0; l + 1 < cfg.n_layers && !rc; ++l)
@@ -392,6 +404,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
       cudaMemset(p->yp, 0, (size_t)RM * (K + 1) * H * 4);
       cudaMemset(p->gcnt, 0, p->gcnt_n * 4);
       cudaMemset(p->dcnt, 0, p->dcnt_n * 4);
+      cudaMemset(p->xready, 0, (size_t)(RM * K + 1) * 4);
     }
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) rc = cuda_fail(p, e, "plan setup");
@@ -546,6 +559,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.gu_estride = p->gu_estride;
     prm.dn_estride = p->dn_estride;
     prm.mix_part = p->mix_part;
+    prm.abuf = p->abuf;
+    prm.sq_part = p->sq_part;
     prm.logits = p->logits;
     prm.act = p->act;
     prm.yp = p->yp;
@@ -554,6 +569,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.dpart = p->dpart;
     prm.gcnt = p->gcnt;
     prm.dcnt = p->dcnt;
+    prm.xready = p->xready;
+    prm.n_xready = p->xready ? rows * p->cfg.top_k + 1 : 0;
     prm.sync = p->sync + l;
     prm.err = p->err;
     prm.taps = ls.taps;
@@ -625,6 +642,7 @@ extern "C" int mono_ffn_query_error(mono_ffn_plan_t* p, mono_ffn_status* st) {
     cudaMemset(p->err, 0, sizeof(ErrBlock));
     if (p->gcnt) cudaMemset(p->gcnt, 0, p->gcnt_n * 4);
     if (p->dcnt) cudaMemset(p->dcnt, 0, p->dcnt_n * 4);
+    if (p->xready) cudaMemset(p->xready, 0, (size_t)(p->cfg.max_rows * p->cfg.top_k + 1) * 4);
     cudaDeviceSynchronize();
   }
   if (st) {

@@ -239,12 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
         // a new down expert: once every MMA reading the B region is done
         // (and, the first time, every CTA's activations are out), one bulk
         // copy brings this expert's operand in
-        if (prev_x < 0) {
-          if (lane == 0 && ok) ok = wait_count(p, c, &p.sync->cnt_act, ep1 * (uint32_t)G, 4u);
-          ok = warp_ok(ok);
-          fence_proxy_async_global();
-          trace(p, 8, lane == 0);
-        }
+        // this expert's activations are complete once every one of its
+        // gate/up blocks has been finished (by whichever CTA)
+        if (lane == 0 && ok) ok = wait_count(p, c, &p.xready[sg.x], (uint32_t)geo.nbi, 4u);
+        ok = warp_ok(ok);
+        fence_proxy_async_global();
+        trace(p, 8, prev_x < 0 && lane == 0);
         umma_commit_warp(&c->drain);
         if (lane == 0 && ok) ok = wait_bar(p, c, &c->drain, ndrain & 1u);
         ok = warp_ok(ok);
@@ -337,15 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   // ================================================================ prologue
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, ep1);
+    control_warps(p, c, ep1, false);
     return;
   }
-  collapse_norm<true>(p, c, regA);
+  collapse_norm<true>(p, c, regA, ep1);
   fence_proxy_async_smem();   // n is read by the tensor cores (async proxy)
   bar_sync(kBarCons, kCW * 32);
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
   trace(p, 3, tid == 0);
   router_logits<true>(p, c, regA);
+  route_rows(p, c, ep1);
 
   // the compute warps agree on the expert list once
   if (tid == 0) {
@@ -457,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
         }
         bar_sync(kBarEpi, 4 * 32);   // bcast is reused by the next segment
       }
-      if (!complete || !live) return;
+      if (!complete) return;   // the same for every epilogue thread
       const int x = sg.x;
       if (gu) {
         // SwiGLU, written as the down projection's B operand of expert entry
@@ -467,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
         uint16_t* dst = reinterpret_cast<uint16_t*>(p.actb + (size_t)x * I * 32 + (size_t)(ch >> 3) * 256) + (ch & 7);
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r) {
+          if (!live) break;
           const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
           uint16_t hb = 0, lb = 0;
           if (r < R && sl >= 0) {
@@ -483,7 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
           dst[(2 * r) * 8] = hb;
           dst[(2 * r + 1) * 8] = lb;
         }
-      } else {
+        // the block's activations are out: count it for its expert (they are
+        // read by bulk copies, the async proxy)
+        __threadfence();
+        bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
+        if (tid == 0 && live) {
+          fence_proxy_async_global();
+          red_release_add(&p.xready[x], 1u);
+        }
+      } else if (live) {
         const int h = sg.blk * 128 + i;
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r) {
@@ -499,12 +509,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     trace(p, 6, tid == 0);
     tc_segments(p, geo, L_RGU, nu, seg);
     trace(p, 7, tid == 0);
-    bar_sync(kBarEpi, 4 * 32);
-    if (tid == 0) {   // the activations are read by bulk copies (async proxy)
-      __threadfence();
-      fence_proxy_async_global();
-      red_release_add(&p.sync->cnt_act, 1u);
-    }
     tc_segments(p, geo, L_DN, nu, seg);
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
@@ -522,9 +526,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   if (tid == 0) wait_count(p, c, &p.sync->cnt_y, ep1 * (uint32_t)G, 6u);
   bar_sync(kBarCons, kCW * 32);
   tail(p, c, [&](int r, int h) {
-    float y = 0.f;
     const float* src = p.yp + (size_t)r * (K + 1) * H + h;
-    for (int j = 0; j <= K; ++j) y += __ldcg(src + (size_t)j * H);
+    float v[kMaxK + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) v[j] = j <= K ? __ldcg(src + (size_t)j * H) : 0.f;
+    float y = 0.f;
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) y += v[j];   // slot order; the zero padding adds exactly
     return y;
   });
   bar_sync(kBarCons, kCW * 32);

@@ -90,7 +90,7 @@ def test_full_size_mxfp4_chain_row_sample():
     for l in range(wl.n_layers):
         out, t, keep = _check_rows(wl, run, r, layer=l, hc_rows=x)
         x = out
-    compare_out(wl, got[r], O.decode_hc(wl, x), "chain hc_out", ulps=wl.n_layers)
+    compare_out(wl, got[r], O.decode_hc(wl, x), "chain hc_out", layers=wl.n_layers)
     del w1
     run.close()
     del run

@@ -166,7 +166,7 @@ def test_scaled_chain_four_layers(wdt):
     # the whole chain against the oracle's chain: rows whose routing never
     # met a near tie along the way
     want = O.decode_hc(wl, O.chain(wl, lws, S.cpu_hc_in(wl), deferred=True))
-    compare_out(wl, got, want, "chain hc_out", allow_rows_off=2, ulps=wl.n_layers)
+    compare_out(wl, got, want, "chain hc_out", allow_rows_off=2, layers=wl.n_layers)
     run.close()
 
 
