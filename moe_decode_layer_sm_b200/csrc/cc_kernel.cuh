@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
 
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, ep1, true);
+    control_warps(p, c, regA, ep1, true);
     return;
   }
 
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
   collapse_norm<false>(p, c, regA, ep1);
   const void* n_s = regA;
   trace(p, 3, ctid == 0);
-  router_logits<false>(p, c, regA);
+  router_logits<false>(p, c, regA, false);
 
   // ---------------- expert matvecs from the weight ring
   uint32_t s = 0;   // stage counter (mirrors the producer)

@@ -366,8 +366,11 @@ __device__ __forceinline__ void load8(const uint8_t* base, size_t i, bool bf, fl
 // fp32, sel = score + bias, canonical top-k by (sel desc, index asc) through
 // warp max / min reductions, then weight = score / max(sum, clamp) * scale
 // with each op rounded to fp32.  Lane l holds experts l + 32 q, q < NQ.
+// dry: run the same code without storing anything (it is then warm in the
+// SM's instruction cache when the real call comes); not inlined, so that the
+// dry and the real call share one copy of the code.
 template <int NQ>
-__device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
+__device__ __noinline__ void topk_row(const Params& p, Ctl* c, int r, bool dry) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, K = p.K;
   float score[NQ];
@@ -391,14 +394,14 @@ __device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
       key[q] = ord_key(score[q] + bs[q]);
     }
   }
-  if (blockIdx.x == 0 && p.taps.logits) {
+  if (blockIdx.x == 0 && p.taps.logits && !dry) {
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       if (lane + 32 * q < E) p.taps.logits[(size_t)r * E + lane + 32 * q] = lg[q];
   }
-  trace(p, 26, r == 0 && lane == 0);
+  trace(p, 26, r == 0 && lane == 0 && !dry);
   uint32_t taken = 0u;
-  float ssum = 0.f;
+  float ssum = 0.f, wsel = 0.f;
   for (int j = 0; j < K; ++j) {
     uint32_t bk = 0u;
     int be = 0x7FFFFFFF;
@@ -416,16 +419,14 @@ __device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
     const int wl = we & 31;
     if (we < E && wl == lane) taken |= 1u << (we >> 5);
     const float ws = __shfl_sync(0xffffffffu, bs, wl);
-    if (lane == 0) {
-      c->idx[r][j] = we < E ? we : 0;
-      c->wt[r][j] = ws;   // the raw score until the sum is known
-    }
+    if (lane == j) wsel = ws;   // lane j keeps the j-th raw score
+    if (lane == 0 && !dry) c->idx[r][j] = we < E ? we : 0;
     ssum += ws;   // selection order, fp32
   }
   __syncwarp();
-  if (lane < K) {
+  if (lane < K && !dry) {
     const float den = fmaxf(ssum, p.denom_clamp);
-    const float w = __fmul_rn(__fdiv_rn(c->wt[r][lane], den), p.route_scale);
+    const float w = __fmul_rn(__fdiv_rn(wsel, den), p.route_scale);
     c->wt[r][lane] = w;
     if (blockIdx.x == 0) {
       if (p.taps.idx) p.taps.idx[r * K + lane] = c->idx[r][lane];
@@ -433,6 +434,17 @@ __device__ __forceinline__ void topk_row(const Params& p, Ctl* c, int r) {
     }
   }
   __syncwarp();
+}
+
+// the top-k of row r with the lane layout that fits E
+__device__ __forceinline__ void topk_dispatch(const Params& p, Ctl* c, int r, bool dry) {
+  const int E = p.E;
+  if (E <= 32) topk_row<1>(p, c, r, dry);
+  else if (E <= 64) topk_row<2>(p, c, r, dry);
+  else if (E <= 128) topk_row<4>(p, c, r, dry);
+  else if (E <= 256) topk_row<8>(p, c, r, dry);
+  else if (E <= 512) topk_row<16>(p, c, r, dry);
+  else topk_row<32>(p, c, r, dry);
 }
 
 // ------------------------------------------------------------ work walkers --
@@ -622,12 +634,15 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
   }
 }
 
+template <bool CANON>
+__device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s, bool dry);
+
 // Control warps: Sinkhorn of the comb logits (16 threads per row), then the
 // canonical top-k of each row once every CTA's router logits are out (here
 // when ctl_topk; otherwise the compute warps do it in route_rows and hand
 // over at the routing barrier), then the list of unique routed experts with
 // their rows and act slots.
-__device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1, bool ctl_topk) {
+__device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint32_t ep1, bool ctl_topk) {
   const int R = p.R, E = p.E, K = p.K, G = p.G;
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kCtlWarp0;
   const int ct = threadIdx.x - kCtlWarp0 * 32;
@@ -660,19 +675,18 @@ __device__ void control_warps(const Params& p, Ctl* c, uint32_t ep1, bool ctl_to
     if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
     trace(p, 21, ct == 0);
     bar_sync(kBarCtl, kCtlWarps * 32);
-    for (int r = cw; r < R; r += kCtlWarps) {
-      if (E <= 32) topk_row<1>(p, c, r);
-      else if (E <= 64) topk_row<2>(p, c, r);
-      else if (E <= 128) topk_row<4>(p, c, r);
-      else if (E <= 256) topk_row<8>(p, c, r);
-      else if (E <= 512) topk_row<16>(p, c, r);
-      else topk_row<32>(p, c, r);
-    }
+    for (int r = cw; r < R; r += kCtlWarps) topk_dispatch(p, c, r, false);
     for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
     bar_sync(kBarCtl, kCtlWarps * 32);
     trace(p, 22, ct == 0);
   } else {
     for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
+    // idle until the compute warps have the top-k rows: run the router and
+    // top-k code once without storing anything, so that it is warm in this
+    // SM's instruction cache when the compute warps get there (the tensor-
+    // core kernel is the only caller of this branch)
+    router_logits<true>(p, c, regA, true);
+    if (cw == 0) topk_dispatch(p, c, 0, true);
     // the compute warps' top-k rows (route_rows) are in c->idx / c->wt after this
     bar_sync(kBarRoute, kPreThreads);
   }
@@ -854,9 +868,11 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
 
 // Router logits of this CTA's experts (two rows of router_t at a time; each
 // thread's share of both rows is loaded at once), then the CTA's arrival at
-// the logits counter; compute warps only.
+// the logits counter; compute warps only.  dry: the same code without
+// barriers or stores, to warm the instruction cache (not inlined, so that
+// both calls share the code).
 template <bool CANON>
-__device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
+__device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s, bool dry) {
   const int R = p.R, H = p.H, E = p.E, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
   const bool nbf = CANON || p.round_bf16;
   const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
@@ -890,12 +906,13 @@ __device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
         }
         a0 = warp_sum(a0);
         a1 = warp_sum(a1);
-        if (lane == 0) {
+        if (lane == 0 && !dry) {
           c->sq[warp][r] = (hb == 0 ? 0.f : c->sq[warp][r]) + a0;
           c->sq2[warp][r] = (hb == 0 ? 0.f : c->sq2[warp][r]) + a1;
         }
       }
     }
+    if (dry) continue;
     trace(p, 25, ctid == 0 && e == e0);
     bar_sync(kBarCons, kCW * 32);
     if (ctid < 2 * R) {
@@ -908,6 +925,7 @@ __device__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s) {
     }
     bar_sync(kBarCons, kCW * 32);
   }
+  if (dry) return;
   if (ctid == 0 && (int)blockIdx.x != p.fault_cta) {
     __threadfence();
     red_release_add(&p.sync->cnt_logit, 1u);
@@ -923,14 +941,7 @@ __device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1) {
   if (threadIdx.x == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
   bar_sync(kBarCons, kCW * 32);
   trace(p, 21, threadIdx.x == 0);
-  for (int r = warp; r < R; r += kCW) {
-    if (E <= 32) topk_row<1>(p, c, r);
-    else if (E <= 64) topk_row<2>(p, c, r);
-    else if (E <= 128) topk_row<4>(p, c, r);
-    else if (E <= 256) topk_row<8>(p, c, r);
-    else if (E <= 512) topk_row<16>(p, c, r);
-    else topk_row<32>(p, c, r);
-  }
+  for (int r = warp; r < R; r += kCW) topk_dispatch(p, c, r, false);
   trace(p, 22, threadIdx.x == 0);
   bar_sync(kBarRoute, kPreThreads);
 }

@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   if (warp == kProdWarp) {
     uint32_t s = 0, issued = 0;
     bool ok = true;
-    bool first_copy[2] = {false, false};
+    uint32_t first_copy = 0u;
     auto seg = [&](const Seg& sg) {
       if (lane != 0) return;
       size_t kgb;
@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
             mbar_arrive_expect_tx(&full[slot], bytes);
             tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)kg * kgb, bytes, &full[slot]);
             issued = s + 1;
-            if (sg.list != L_SGU && !first_copy[sg.list - 1]) {
-              first_copy[sg.list - 1] = true;
+            if (sg.list != L_SGU && !(first_copy & (1u << sg.list))) {
+              first_copy |= 1u << sg.list;
               trace(p, 17 + sg.list);
             }
           }
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   // ================================================================ prologue
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, ep1, false);
+    control_warps(p, c, regA, ep1, false);
     return;
   }
   collapse_norm<true>(p, c, regA, ep1);
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   bar_sync(kBarCons, kCW * 32);
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
   trace(p, 3, tid == 0);
-  router_logits<true>(p, c, regA);
+  router_logits<true>(p, c, regA, false);
   route_rows(p, c, ep1);
 
   // the compute warps agree on the expert list once
