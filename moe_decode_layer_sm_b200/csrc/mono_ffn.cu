@@ -12,6 +12,7 @@
 #include "mono_ffn.h"
 #include "cc_kernel.cuh"
 #include "tc_kernel.cuh"
+#include "tq_kernel.cuh"
 
 using namespace mono;
 
@@ -26,6 +27,8 @@ struct LayerSlot {
   float* bias = nullptr;
   uint8_t* gu = nullptr;
   uint8_t* dn = nullptr;
+  float* gsc = nullptr;   // quantised tensor-core path, FP8: packed block scales
+  float* dsc = nullptr;
   bool packed = false;
   Taps taps{};
 };
@@ -36,6 +39,7 @@ struct mono_ffn_plan_s {
   mono_ffn_config cfg{};
   int wt = 0;
   bool tc = false;   // bf16 experts run on the tensor-core kernel
+  bool tq = false;   // FP8 / MXFP4 experts run on the quantised tensor-core kernel
   int G = 0, nst = 0, slot_bytes = 0, regA_bytes = 0, ymax = 0, mix_ctas = 0, smem = 0;
   int gu_kc = 0, gu_nk = 0, gu_rc = 0, dn_kc = 0, dn_nk = 0, dn_rc = 0;
   long long gu_estride = 0, dn_estride = 0;
@@ -102,8 +106,10 @@ void* kernel_ptr() {
   return reinterpret_cast<void*>(&mono_ffn_cc_kernel<WT>);
 }
 
-void* kernel_for(int wt, bool tc) {
+void* kernel_for(int wt, bool tc, bool tq) {
   if (tc) return reinterpret_cast<void*>(&mono_ffn_tc_kernel<W_BF16>);
+  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP8>)
+                             : reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP4>);
   switch (wt) {
     case W_F32: return kernel_ptr<W_F32>();
     case W_BF16: return kernel_ptr<W_BF16>();
@@ -127,6 +133,63 @@ __global__ void pack_tc_kernel(const uint16_t* src, uint8_t* dst, long long e1, 
     const long long off = ((e * NB + row / 128) * KG + kg) * 16 * rgb + ((row % 128) / 8) * rgb + sub + (row % 8) * 16;
     *reinterpret_cast<uint4*>(dst + off) = v;
   }
+}
+
+// Quantised tensor-core layout of one [E+1][rows][row_bytes] code matrix set:
+// units of 128 rows x ub bytes (128 contraction elements), the 16-byte chunk
+// j of unit-row i at j * 2048 + i * 16 inside the unit's matrix slot msub:
+//   dst[((e * rows/128 + row/128) * nu + u) * ustride + msub + j * 2048 + (row % 128) * 16]
+__global__ void pack_tq_codes_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int row_bytes, int ub,
+                                     long long ustride, int msub) {
+  const int nch = row_bytes / 16, nu = row_bytes / ub, cpu = ub / 16, NB = rows / 128;
+  const long long n = e1 * rows * nch;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int ch = (int)(i % nch);
+    const long long row = (i / nch) % rows, e = i / ((long long)nch * rows);
+    const int u = ch / cpu, j = ch % cpu;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)ch * 16);
+    const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + (long long)j * 2048 + (row % 128) * 16;
+    *reinterpret_cast<uint4*>(dst + off) = v;
+  }
+}
+
+// MXFP4 e8m0 scales [E+1][rows][cols/32] -> the 4 scales of each unit-row
+// after the unit's codes: dst[unit * ustride + msub + code_bytes + (row % 128) * 4 + jj]
+__global__ void pack_tq_e8m0_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int ns, long long ustride,
+                                    int msub, int code_bytes) {
+  const int nu = ns / 4, NB = rows / 128;
+  const long long n = e1 * rows * nu;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(i % nu);
+    const long long row = (i / nu) % rows, e = i / ((long long)nu * rows);
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(src + (e * rows + row) * ns + (long long)u * 4);
+    const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + code_bytes + (row % 128) * 4;
+    *reinterpret_cast<uint32_t*>(dst + off) = v;
+  }
+}
+
+// FP8 fp32 block scales [E+1][rows][cols/128] -> [E+1][rows/128][cols/128][nm * 128]
+// (slot m = gate 0 / up 1 of a gate/up pair, or the single down matrix)
+__global__ void pack_tq_scales_kernel(const float* src, float* dst, long long e1, int rows, int nu, int nm, int m) {
+  const int NB = rows / 128;
+  const long long n = e1 * rows * nu;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int u = (int)(i % nu);
+    const long long row = (i / nu) % rows, e = i / ((long long)nu * rows);
+    dst[((e * NB + row / 128) * nu + u) * (nm * 128) + m * 128 + row % 128] = src[(e * rows + row) * nu + u];
+  }
+}
+
+// smallest and largest byte of n (for the MXFP4 scale range check)
+__global__ void byte_range_kernel(const uint8_t* src, long long n, unsigned int* mm) {
+  unsigned int lo = 255, hi = 0;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const unsigned int v = src[i];
+    lo = min(lo, v);
+    hi = max(hi, v);
+  }
+  atomicMin(&mm[0], lo);
+  atomicMax(&mm[1], hi);
 }
 
 // ------------------------------------------------------------ pack kernels --
@@ -220,6 +283,8 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
     cudaFree(l.bias);
     cudaFree(l.gu);
     cudaFree(l.dn);
+    cudaFree(l.gsc);
+    cudaFree(l.dsc);
   }
   for (float* q : p->pend) cudaFree(q);
   cudaFree(p->mix_part);
@@ -296,6 +361,9 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   // bf16 experts run on the tensor cores when the shapes allow it
   // whole 128-row blocks and 128-wide K units; n is the bf16 B operand
   p->tc = dt == MONO_BF16 && cfg.round_bf16 && H % 128 == 0 && I % 128 == 0;
+  // FP8 / MXFP4 experts: converted to fp16 on the way into the tensor cores
+  p->tq = (dt == MONO_FP8E4M3_B128 || dt == MONO_MXFP4) && cfg.round_bf16 && H % 128 == 0 && I % 128 == 0;
+  const long long tq_mat = dt == MONO_FP8E4M3_B128 ? 16384 : 8192 + 512;   // one 128 x 128 unit of one matrix
   // chunking of the packed rows
   const int gu_target = dt == MONO_F32 ? 256 : dt == MONO_BF16 ? 512 : 1024;
   const int dn_target = dt == MONO_F32 ? 512 : dt == MONO_BF16 ? 1024 : 2048;
@@ -313,6 +381,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     p->dn_estride = (long long)(H / 128) * (I / 8) * 2048;
     p->slot_bytes = 16384;
   }
+  if (p->tq) {
+    p->gu_estride = (long long)(I / 128) * (H / 128) * 2 * tq_mat;
+    p->dn_estride = (long long)(H / 128) * (I / 128) * tq_mat;
+    p->slot_bytes = (int)(2 * tq_mat);
+  }
 
   // grid and shared memory
   // grid: one CTA per SM, a multiple of 4 (the mix partials are read as float4 per output)
@@ -329,8 +402,8 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   // one row's mix partials of every CTA
   regA = std::max<size_t>(regA, align_up(((size_t)kS * p->ymax * kMixC + (size_t)RM * kS * p->ymax) * 4, 16) +
                                     (size_t)p->G * kMixP * 4);
-  if (p->tc) {
-    regA = std::max<size_t>(regA, (size_t)H * 16);   // n: 8 rows of bf16
+  if (p->tc || p->tq) {
+    regA = std::max<size_t>(regA, (size_t)H * 16);   // n: 8 rows of 16-bit values
     regA = std::max<size_t>(regA, (size_t)I * 32);   // down B: 16 rows (hi/lo of 8 token rows)
   }
   p->regA_bytes = (int)align_up(regA, 128);
@@ -346,7 +419,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     return fail(nullptr, MONO_ERR_INVALID_ARG, m);
   }
   p->smem = (int)SmemLayout(p->nst, p->slot_bytes, p->regA_bytes, p->ymax).total;
-  void* kfn = kernel_for(dt, p->tc);
+  void* kfn = kernel_for(dt, p->tc, p->tq);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
   int occ = 0;
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kfn, kThreads, p->smem);
@@ -370,21 +443,25 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     if (!rc) rc = dalloc(p, &l.bias, (size_t)E * 4, &p->packed_bytes);
     if (!rc) rc = dalloc(p, &l.gu, (size_t)(E + 1) * p->gu_estride, &p->packed_bytes);
     if (!rc) rc = dalloc(p, &l.dn, (size_t)(E + 1) * p->dn_estride, &p->packed_bytes);
+    if (!rc && p->tq && dt == MONO_FP8E4M3_B128) {
+      rc = dalloc(p, &l.gsc, (size_t)(E + 1) * (I / 128) * (H / 128) * 256 * 4, &p->packed_bytes);
+      if (!rc) rc = dalloc(p, &l.dsc, (size_t)(E + 1) * (H / 128) * (I / 128) * 128 * 4, &p->packed_bytes);
+    }
   }
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->abuf, (size_t)RM * H * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->sq_part, (size_t)RM * p->G * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->act, (size_t)RM * (K + 1) * I * 4, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->yp, (size_t)RM * (K + 1) * H * 4, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->actb, (size_t)(RM * K + 1) * I * 32, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->gpart, (size_t)p->G * 4 * 128 * 16 * 4, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->dpart, (size_t)p->G * 2 * 128 * 16 * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->yp, (size_t)RM * (K + 1) * H * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->actb, (size_t)(RM * K + 1) * I * 32, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->gpart, (size_t)p->G * 4 * 128 * 16 * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->dpart, (size_t)p->G * 2 * 128 * 16 * 4, &p->scratch_bytes);
   p->gcnt_n = (size_t)(RM * K + 2) * (I / 128);
   p->dcnt_n = (size_t)(RM * K + 2) * (H / 128);
-  if (!rc && p->tc) rc = dalloc(p, &p->gcnt, p->gcnt_n * 4, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->xready, (size_t)(RM * K + 1) * 4, &p->scratch_bytes);
-  if (!rc && p->tc) rc = dalloc(p, &p->dcnt, p->dcnt_n * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->gcnt, p->gcnt_n * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->xready, (size_t)(RM * K + 1) * 4, &p->scratch_bytes);
+  if (!rc && (p->tc || p->tq)) rc = dalloc(p, &p->dcnt, p->dcnt_n * 4, &p->scratch_bytes);
   p->pend.assign(cfg.n_layers, nullptr);
   for (int l = 0; l + 1 < cfg.n_layers && !rc; ++l)
     rc = dalloc(p, &p->pend[l], (size_t)RM * (kS + kS * kS + H) * 4, &p->scratch_bytes);
@@ -400,7 +477,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     cudaMemset(p->sync, 0, sizeof(SyncBlock) * cfg.n_layers);
     cudaMemset(p->err, 0, sizeof(ErrBlock));
     cudaMemset(p->act, 0, (size_t)RM * (K + 1) * I * 4);
-    if (p->tc) {
+    if (p->tc || p->tq) {
       cudaMemset(p->yp, 0, (size_t)RM * (K + 1) * H * 4);
       cudaMemset(p->gcnt, 0, p->gcnt_n * 4);
       cudaMemset(p->dcnt, 0, p->dcnt_n * 4);
@@ -451,6 +528,68 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
     pack_tc_kernel<<<grid(n_gu), th, 0, st>>>((const uint16_t*)w->w_gate, l.gu, E + 1, I, H, 256, 0);
     pack_tc_kernel<<<grid(n_gu), th, 0, st>>>((const uint16_t*)w->w_up, l.gu, E + 1, I, H, 256, 128);
     pack_tc_kernel<<<grid(n_dn), th, 0, st>>>((const uint16_t*)w->w_down, l.dn, E + 1, H, I, 128, 0);
+    cudaError_t e2 = cudaGetLastError();
+    cudaSetDevice(prev);
+    if (e2 != cudaSuccess) return cuda_fail(p, e2, "pack");
+    l.packed = true;
+    return MONO_OK;
+  }
+  if (p->tq) {
+    const bool fp8 = p->wt == W_FP8;
+    const int th = 256;
+    auto grid = [&](long long n) { return (unsigned)std::min<long long>((n + th - 1) / th, 148LL * 64); };
+    const long long mat = fp8 ? 16384 : 8192 + 512;
+    const int code_b = fp8 ? 16384 : 8192, ub = fp8 ? 128 : 64;   // unit-row bytes of codes
+    const int gu_rb = fp8 ? H : H / 2, dn_rb = fp8 ? I : I / 2;    // code bytes per weight row
+    if (!fp8) {
+      // every e8m0 scale must keep e2m1 * scale exact in fp16: 2^-22 .. 2^12
+      unsigned int* mm = nullptr;
+      cudaError_t ea = cudaMalloc(&mm, 8);
+      if (ea != cudaSuccess) {
+        cudaSetDevice(prev);
+        return cuda_fail(p, ea, "pack: scale range scratch");
+      }
+      const unsigned int init[2] = {255u, 0u};
+      cudaMemcpyAsync(mm, init, 8, cudaMemcpyHostToDevice, st);
+      byte_range_kernel<<<148, 256, 0, st>>>((const uint8_t*)w->s_gate, (long long)(E + 1) * I * (H / 32), mm);
+      byte_range_kernel<<<148, 256, 0, st>>>((const uint8_t*)w->s_up, (long long)(E + 1) * I * (H / 32), mm);
+      byte_range_kernel<<<148, 256, 0, st>>>((const uint8_t*)w->s_down, (long long)(E + 1) * H * (I / 32), mm);
+      unsigned int got[2] = {0u, 0u};
+      cudaMemcpyAsync(got, mm, 8, cudaMemcpyDeviceToHost, st);
+      ea = cudaStreamSynchronize(st);
+      cudaFree(mm);
+      if (ea != cudaSuccess) {
+        cudaSetDevice(prev);
+        return cuda_fail(p, ea, "pack: scale range");
+      }
+      if (got[0] < 127u - 22u || got[1] > 127u + 12u) {
+        cudaSetDevice(prev);
+        return fail(p, MONO_ERR_INVALID_ARG,
+                    "pack: MXFP4 scales 2^" + std::to_string((int)got[0] - 127) + " .. 2^" + std::to_string((int)got[1] - 127) +
+                        " leave the range 2^-22 .. 2^12 in which the tensor-core path converts them exactly to fp16");
+      }
+    }
+    pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
+        (const uint8_t*)w->w_gate, l.gu, E + 1, I, gu_rb, ub, 2 * mat, 0);
+    pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
+        (const uint8_t*)w->w_up, l.gu, E + 1, I, gu_rb, ub, 2 * mat, (int)mat);
+    pack_tq_codes_kernel<<<grid((long long)(E + 1) * H * (dn_rb / 16)), th, 0, st>>>(
+        (const uint8_t*)w->w_down, l.dn, E + 1, H, dn_rb, ub, mat, 0);
+    if (fp8) {
+      pack_tq_scales_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
+          (const float*)w->s_gate, l.gsc, E + 1, I, H / 128, 2, 0);
+      pack_tq_scales_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
+          (const float*)w->s_up, l.gsc, E + 1, I, H / 128, 2, 1);
+      pack_tq_scales_kernel<<<grid((long long)(E + 1) * H * (I / 128)), th, 0, st>>>(
+          (const float*)w->s_down, l.dsc, E + 1, H, I / 128, 1, 0);
+    } else {
+      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
+          (const uint8_t*)w->s_gate, l.gu, E + 1, I, H / 32, 2 * mat, 0, code_b);
+      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
+          (const uint8_t*)w->s_up, l.gu, E + 1, I, H / 32, 2 * mat, (int)mat, code_b);
+      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * H * (I / 128)), th, 0, st>>>(
+          (const uint8_t*)w->s_down, l.dn, E + 1, H, I / 32, mat, 0, code_b);
+    }
     cudaError_t e2 = cudaGetLastError();
     cudaSetDevice(prev);
     if (e2 != cudaSuccess) return cuda_fail(p, e2, "pack");
@@ -515,7 +654,7 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
   cudaGetDevice(&prev);
   if (prev != p->cfg.device) cudaSetDevice(p->cfg.device);
   const int L = p->cfg.n_layers;
-  void* kfn = kernel_for(p->wt, p->tc);
+  void* kfn = kernel_for(p->wt, p->tc, p->tq);
   cudaError_t e = cudaSuccess;
   for (int l = 0; l < L && e == cudaSuccess; ++l) {
     const LayerSlot& ls = p->layers[l];
@@ -570,6 +709,9 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.gcnt = p->gcnt;
     prm.dcnt = p->dcnt;
     prm.xready = p->xready;
+    prm.gsc = ls.gsc;
+    prm.dsc = ls.dsc;
+    prm.q_f16 = p->tq;
     prm.n_xready = p->xready ? rows * p->cfg.top_k + 1 : 0;
     prm.sync = p->sync + l;
     prm.err = p->err;

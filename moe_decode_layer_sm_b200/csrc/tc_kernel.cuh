@@ -109,6 +109,139 @@ __device__ __forceinline__ const uint8_t* seg_base(const Params& p, const Ctl* c
   return p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * g.kgi * kgb;
 }
 
+// Epilogue, thread i (= row i of the 128-row tile) of warps 0-3, with this
+// CTA's part of a block in a[8] (gate, or the down output) and b[8] (up):
+// for a block split across CTAs, publish the part; the CTA that arrives last
+// adds every part in CTA order.  A part is [a0..a7 | b0..b7] of this row;
+// only the quarters the rows and the list need move.  Returns true in the
+// CTA that holds the complete block (then a and b hold its sums); the same
+// answer in every epilogue thread.
+__device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo& geo, const Seg& sg, int upb, bool gu,
+                                            bool live, int i, float (&a)[8], float (&b)[8]) {
+  const int G = p.G, R = p.R, tid = threadIdx.x;
+  volatile int* bcast = &c->bcast;
+  const long long u0 = sg.gblk * upb, u1 = u0 + upb;
+  const int c_lo = part_owner(sg.N, G, u0), c_hi = part_owner(sg.N, G, u1 - 1);
+  if (c_lo == c_hi) return true;
+  // part slots: a CTA's first and last segment of a list (0 / 1), the
+  // routed gate/up list after the shared one (2 / 3)
+  const int nsl = gu ? 4 : 2, sl0 = sg.list == L_RGU ? 2 : 0;
+  const bool q1 = R > 4;
+  const int slot = sl0 + (part_start(sg.N, G, blockIdx.x) >= u0 ? 0 : 1);
+  float4* mine = reinterpret_cast<float4*>((gu ? p.gpart : p.dpart) + (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16);
+  if (live) {
+    __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
+    if (q1) __stcg(mine + 1, make_float4(a[4], a[5], a[6], a[7]));
+    if (gu) __stcg(mine + 2, make_float4(b[0], b[1], b[2], b[3]));
+    if (gu && q1) __stcg(mine + 3, make_float4(b[4], b[5], b[6], b[7]));
+  }
+  __threadfence();
+  bar_sync(kBarEpi, 4 * 32);
+  if (tid == 0) {
+    uint32_t* cnt = (gu ? p.gcnt : p.dcnt) + (size_t)sg.x * (gu ? geo.nbi : geo.nbh) + sg.blk;
+    int parts = 0;
+    for (int cc = c_lo; cc <= c_hi; ++cc) parts += part_start(sg.N, G, cc) != part_start(sg.N, G, cc + 1);
+    const uint32_t old = live ? atomicAdd(cnt, 1u) : 0u;
+    const bool last = live && old == (uint32_t)(parts - 1);
+    if (last) atomicExch(cnt, 0u);   // ready for the next step
+    __threadfence();
+    *bcast = last ? 1 : 0;
+  }
+  bar_sync(kBarEpi, 4 * 32);
+  const bool complete = *bcast != 0;
+  if (complete) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
+    // four parts in flight at a time, added in CTA order
+    for (int cb = c_lo; cb <= c_hi; cb += 4) {
+      float4 ld[4][4];
+      bool use[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int cc = cb + j;
+        const long long ps = part_start(sg.N, G, cc);
+        use[j] = cc <= c_hi && ps != part_start(sg.N, G, cc + 1);   // skip empty ranges
+        const int sl = sl0 + (ps >= u0 ? 0 : 1);
+        const float4* src =
+            reinterpret_cast<const float4*>((gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + sl) * 128 + i) * 16);
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        ld[j][0] = use[j] ? __ldcg(src) : z;
+        ld[j][1] = use[j] && q1 ? __ldcg(src + 1) : z;
+        ld[j][2] = use[j] && gu ? __ldcg(src + 2) : z;
+        ld[j][3] = use[j] && gu && q1 ? __ldcg(src + 3) : z;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!use[j]) continue;
+        a[0] += ld[j][0].x; a[1] += ld[j][0].y; a[2] += ld[j][0].z; a[3] += ld[j][0].w;
+        a[4] += ld[j][1].x; a[5] += ld[j][1].y; a[6] += ld[j][1].z; a[7] += ld[j][1].w;
+        b[0] += ld[j][2].x; b[1] += ld[j][2].y; b[2] += ld[j][2].z; b[3] += ld[j][2].w;
+        b[4] += ld[j][3].x; b[5] += ld[j][3].y; b[6] += ld[j][3].z; b[7] += ld[j][3].w;
+      }
+    }
+  }
+  bar_sync(kBarEpi, 4 * 32);   // bcast is reused by the next segment
+  return complete;
+}
+
+// A complete block.  Gate/up: SwiGLU, written as the down projection's B
+// operand of expert entry x, [I/8][16 rows][8] 16-bit, row 2r = hi, 2r + 1 =
+// lo of token row r (bf16, or fp16 when p.q_f16), zero for rows that do not
+// use the expert; then the block counts for its expert.  Down: the weighted
+// output of every row that uses the expert into yp.
+__device__ __forceinline__ void epi_store(const Params& p, Ctl* c, const TcGeo& geo, const Seg& sg, bool gu, bool live,
+                                          int i, const float (&a)[8], const float (&b)[8]) {
+  const int R = p.R, K = p.K, H = p.H, I = p.I, tid = threadIdx.x;
+  const int x = sg.x;
+  if (gu) {
+    const int ch = sg.blk * 128 + i;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(p.actb + (size_t)x * I * 32 + (size_t)(ch >> 3) * 256) + (ch & 7);
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r) {
+      if (!live) break;
+      const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
+      uint16_t hb = 0, lb = 0;
+      if (r < R && sl >= 0) {
+        float gg = a[r], uu = b[r];
+        if (p.round_bf16) {
+          gg = round_bf16(gg);
+          uu = round_bf16(uu);
+        }
+        const float act = gg / (1.0f + expf(-gg)) * uu;
+        if (p.q_f16) {
+          const __half hi = __float2half_rn(act);
+          hb = __half_as_ushort(hi);
+          lb = __half_as_ushort(__float2half_rn(act - __half2float(hi)));
+        } else {
+          const __nv_bfloat16 hi = __float2bfloat16_rn(act);
+          hb = __bfloat16_as_ushort(hi);
+          lb = __bfloat16_as_ushort(__float2bfloat16_rn(act - __bfloat162float(hi)));
+        }
+      }
+      dst[(2 * r) * 8] = hb;
+      dst[(2 * r + 1) * 8] = lb;
+    }
+    // the block's activations are out: count it for its expert (they are
+    // read by bulk copies, the async proxy)
+    __threadfence();
+    bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
+    if (tid == 0 && live) {
+      fence_proxy_async_global();
+      red_release_add(&p.xready[x], 1u);
+    }
+  } else if (live) {
+    const int h = sg.blk * 128 + i;
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r) {
+      const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
+      if (r < R && sl >= 0) {
+        const float wgt = x == 0 ? 1.0f : c->wt[r][sl];
+        p.yp[((size_t)r * (K + 1) + sl) * H + h] = wgt * a[r];
+      }
+    }
+  }
+}
+
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -362,7 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     const int i = tid;
     uint32_t t = 0;
     bool ok = true;
-    volatile int* bcast = &c->bcast;
     auto seg = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
       const int upb = gu ? geo.upb_gu : geo.upb_dn;
@@ -391,119 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
           b[r] = 0.f;
         }
       }
-      // a block split across CTAs: publish this part; the CTA that arrives
-      // last adds every part in CTA order.  A part is [a0..a7 | b0..b7] of
-      // this row; only the quarters the rows and the list need move.
-      const long long u0 = sg.gblk * upb, u1 = u0 + upb;
-      const int c_lo = part_owner(sg.N, G, u0), c_hi = part_owner(sg.N, G, u1 - 1);
-      bool complete = c_lo == c_hi;
-      // part slots: a CTA's first and last segment of a list (0 / 1), the
-      // routed gate/up list after the shared one (2 / 3)
-      const int nsl = gu ? 4 : 2, sl0 = sg.list == L_RGU ? 2 : 0;
-      const bool q1 = R > 4;
-      if (!complete) {
-        const int slot = sl0 + (part_start(sg.N, G, blockIdx.x) >= u0 ? 0 : 1);
-        float4* mine = reinterpret_cast<float4*>((gu ? p.gpart : p.dpart) +
-                                                 (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16);
-        if (live) {
-          __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
-          if (q1) __stcg(mine + 1, make_float4(a[4], a[5], a[6], a[7]));
-          if (gu) __stcg(mine + 2, make_float4(b[0], b[1], b[2], b[3]));
-          if (gu && q1) __stcg(mine + 3, make_float4(b[4], b[5], b[6], b[7]));
-        }
-        __threadfence();
-        bar_sync(kBarEpi, 4 * 32);
-        if (tid == 0) {
-          uint32_t* cnt = (gu ? p.gcnt : p.dcnt) + (size_t)sg.x * (gu ? geo.nbi : geo.nbh) + sg.blk;
-          int parts = 0;
-          for (int cc = c_lo; cc <= c_hi; ++cc) parts += part_start(sg.N, G, cc) != part_start(sg.N, G, cc + 1);
-          const uint32_t old = live ? atomicAdd(cnt, 1u) : 0u;
-          const bool last = live && old == (uint32_t)(parts - 1);
-          if (last) atomicExch(cnt, 0u);   // ready for the next step
-          __threadfence();
-          *bcast = last ? 1 : 0;
-        }
-        bar_sync(kBarEpi, 4 * 32);
-        complete = *bcast != 0;
-        if (complete) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
-          // four parts in flight at a time, added in CTA order
-          for (int cb = c_lo; cb <= c_hi; cb += 4) {
-            float4 ld[4][4];
-            bool use[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int cc = cb + j;
-              const long long ps = part_start(sg.N, G, cc);
-              use[j] = cc <= c_hi && ps != part_start(sg.N, G, cc + 1);   // skip empty ranges
-              const int sl = sl0 + (ps >= u0 ? 0 : 1);
-              const float4* src =
-                  reinterpret_cast<const float4*>((gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + sl) * 128 + i) * 16);
-              const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-              ld[j][0] = use[j] ? __ldcg(src) : z;
-              ld[j][1] = use[j] && q1 ? __ldcg(src + 1) : z;
-              ld[j][2] = use[j] && gu ? __ldcg(src + 2) : z;
-              ld[j][3] = use[j] && gu && q1 ? __ldcg(src + 3) : z;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (!use[j]) continue;
-              a[0] += ld[j][0].x; a[1] += ld[j][0].y; a[2] += ld[j][0].z; a[3] += ld[j][0].w;
-              a[4] += ld[j][1].x; a[5] += ld[j][1].y; a[6] += ld[j][1].z; a[7] += ld[j][1].w;
-              b[0] += ld[j][2].x; b[1] += ld[j][2].y; b[2] += ld[j][2].z; b[3] += ld[j][2].w;
-              b[4] += ld[j][3].x; b[5] += ld[j][3].y; b[6] += ld[j][3].z; b[7] += ld[j][3].w;
-            }
-          }
-        }
-        bar_sync(kBarEpi, 4 * 32);   // bcast is reused by the next segment
-      }
-      if (!complete) return;   // the same for every epilogue thread
-      const int x = sg.x;
-      if (gu) {
-        // SwiGLU, written as the down projection's B operand of expert entry
-        // x: [I/8][16 rows][8] bf16, row 2r = hi, 2r + 1 = lo of token row r,
-        // zero for rows that do not use the expert
-        const int ch = sg.blk * 128 + i;
-        uint16_t* dst = reinterpret_cast<uint16_t*>(p.actb + (size_t)x * I * 32 + (size_t)(ch >> 3) * 256) + (ch & 7);
-#pragma unroll
-        for (int r = 0; r < kMaxR; ++r) {
-          if (!live) break;
-          const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
-          uint16_t hb = 0, lb = 0;
-          if (r < R && sl >= 0) {
-            float gg = a[r], uu = b[r];
-            if (p.round_bf16) {
-              gg = round_bf16(gg);
-              uu = round_bf16(uu);
-            }
-            const float act = gg / (1.0f + expf(-gg)) * uu;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(act);
-            hb = __bfloat16_as_ushort(hi);
-            lb = __bfloat16_as_ushort(__float2bfloat16_rn(act - __bfloat162float(hi)));
-          }
-          dst[(2 * r) * 8] = hb;
-          dst[(2 * r + 1) * 8] = lb;
-        }
-        // the block's activations are out: count it for its expert (they are
-        // read by bulk copies, the async proxy)
-        __threadfence();
-        bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
-        if (tid == 0 && live) {
-          fence_proxy_async_global();
-          red_release_add(&p.xready[x], 1u);
-        }
-      } else if (live) {
-        const int h = sg.blk * 128 + i;
-#pragma unroll
-        for (int r = 0; r < kMaxR; ++r) {
-          const int sl = x == 0 ? K : c->uslot[x == 0 ? 0 : x - 1][r];
-          if (r < R && sl >= 0) {
-            const float wgt = x == 0 ? 1.0f : c->wt[r][sl];
-            p.yp[((size_t)r * (K + 1) + sl) * H + h] = wgt * a[r];
-          }
-        }
-      }
+      if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
+      epi_store(p, c, geo, sg, gu, live, i, a, b);
     };
     tc_segments(p, geo, L_SGU, 0, seg);
     trace(p, 6, tid == 0);
