@@ -42,6 +42,7 @@ constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // issuer warp)
 constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6;
 constexpr int kMaxAb = 3;          // A-tile buffers of the quantised tensor-core kernel
+constexpr int kMaxAcc = 4;         // accumulator buffers in tensor memory
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
 
 enum WType { W_F32 = 0, W_BF16 = 1, W_FP8 = 2, W_FP4 = 3 };
@@ -142,7 +143,7 @@ struct Ctl {
   // tensor-core kernel
   uint32_t tmem_base;
   volatile int n_ready;         // n is in shared memory (B operand of gate/up)
-  uint64_t accfull[2], accempty[2], drain;
+  uint64_t accfull[kMaxAcc], accempty[kMaxAcc], drain;
   uint64_t bfull;               // the down projection's B operand has landed
   uint64_t abfull[kMaxAb], abempty[kMaxAb];   // quantised tensor-core kernel: converted A tiles in tensor memory
   volatile int bcast;           // epilogue: "this CTA completes the block"

@@ -187,6 +187,68 @@ __device__ __forceinline__ void umma_f16_tmem_a_warp(uint32_t tmem_d, uint32_t t
       : "memory");
 }
 
+// One 128 x 128 unit of the quantised kernels, issued by one elected lane
+// of a converged warp: 8 K-steps of 16, A from tensor memory (columns a, a +
+// 8, ..; pairs: up at a + 64 into d + 16), B from the descriptor db advanced
+// by db_step (16-byte units) per K-step.  acc0: accumulate from the first
+// K-step on (else the first one overwrites D).
+__device__ __forceinline__ void umma_unit_f16(uint32_t d, uint32_t a, uint64_t db, uint32_t db_step, uint32_t idesc,
+                                              uint32_t acc0, bool pair) {
+  if (pair) {
+    asm volatile(
+        "{\n .reg .pred e, p, t;\n .reg .b32 rx, a0, a1, d1;\n .reg .b64 b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %5, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " mov.b32 a0, %1;\n add.u32 a1, %1, 64;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, p;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
+        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(acc0)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred e, p, t;\n .reg .b32 rx, a0;\n .reg .b64 b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %5, 0;\n setp.eq.b32 t, 0, 0;\n"
+        " mov.b32 a0, %1;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, p;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
+        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(acc0)
+        : "memory");
+  }
+}
+
 // 32 lanes x 16 consecutive 32-bit columns from registers (thread l of the
 // warp writes its quadrant's lane l)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {

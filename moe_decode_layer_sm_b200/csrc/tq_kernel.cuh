@@ -29,6 +29,8 @@ namespace mono {
 constexpr int kTqTmemCols = 512;   // 2 accumulators of 32 columns, then 3 A buffers of 128
 constexpr uint32_t kAbCol = 64;    // first A buffer; buffer b at kAbCol + 128 b (gate 64 | up 64)
 constexpr int kAb = kMaxAb;        // A buffers: the converters run up to 3 units ahead of the MMAs
+// accumulator buffer b: columns 32 b for b < 2, behind the A buffers for b >= 2
+__device__ __forceinline__ uint32_t acc_col(uint32_t b) { return b < 2 ? 32u * b : 448u + 32u * (b - 2); }
 static_assert(kTqTmemCols >= (int)kAbCol + 128 * kAb, "A buffers fit in the tensor memory");
 
 template <int WT> struct TqFmt;
@@ -94,6 +96,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   // throughput of all eight compute warps; its epilogue runs once a segment
   // on warps 0-3 between their conversions.  FP8 converts on warps 4-7.
   constexpr int NCV = WT == W_FP4 ? 8 : 4;
+  // FP8 hands every unit to the epilogue: four accumulators keep the MMAs
+  // three units ahead of it; MXFP4 hands over once per segment
+  constexpr uint32_t NACC = PER_UNIT ? 4 : 2;
+  static_assert(NACC <= kMaxAcc && 448 + 32 * 2 <= kTqTmemCols, "accumulators fit");
   extern __shared__ __align__(1024) uint8_t smem[];
   const SmemLayout L(p.nst, p.slot_bytes, p.regA_bytes, p.ymax);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NCV);   // the converter warps
     }
-    for (int b = 0; b < 2; ++b) {
+    for (uint32_t b = 0; b < NACC; ++b) {
       mbar_init(&c->accfull[b], 1);
       mbar_init(&c->accempty[b], 4);
     }
@@ -216,13 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     const uint32_t b_bytes = (uint32_t)I * 32u;
     const uint64_t bdesc_gu = umma_desc(b_addr, 128u, 0u), bdesc_dn = umma_desc(b_addr, 256u, 128u);
     auto acc_claim = [&]() {   // the accumulator buffer for the next tile
-      const uint32_t buf = t & 1u;
-      if (t >= 2) {
-        if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t >> 1) - 1) & 1u);
+      const uint32_t buf = t % NACC;
+      if (t >= NACC) {
+        if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / NACC) - 1) & 1u);
         ok = warp_ok(ok);
       }
       tc_fence_after();
-      return tmem + 32u * buf;
+      return tmem + acc_col(buf);
     };
     auto seg = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
@@ -260,30 +266,23 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         ok = warp_ok(ok);
         tc_fence_after();
         if (ok) {
+          // the unit's 8 K-steps (gate and up as a pair) from one elected lane
           const uint32_t a0 = tmem + kAbCol + 128u * ab;
-          const int kg0 = u * kKS;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t acc = (PER_UNIT ? ks > 0 : (u > sg.k0 || ks > 0)) ? 1u : 0u;
-            const int kb = kg0 + 2 * ks;   // contraction group of the B operand
-            if (gu) {
-              const uint64_t db = bdesc_gu + (uint64_t)(kb * 8);   // kb * 128 bytes
-              umma_f16_tmem_a_warp(d0, a0 + 8u * ks, db, idesc, acc);
-              umma_f16_tmem_a_warp(d0 + 16u, a0 + 64u + 8u * ks, db, idesc, acc);
-            } else {
-              umma_f16_tmem_a_warp(d0, a0 + 8u * ks, bdesc_dn + (uint64_t)(kb * 16), idesc, acc);   // kb * 256 bytes
-            }
-          }
+          const int kg0 = u * kKS;   // contraction group of the B operand
+          // a fresh accumulator per FP8 unit; MXFP4 adds the segment's units up
+          const uint32_t acc0 = (!PER_UNIT && u > sg.k0) ? 1u : 0u;
+          if (gu) umma_unit_f16(d0, a0, bdesc_gu + (uint64_t)(kg0 * 8), 16u, idesc, acc0, true);   // 2 groups of 128 B a step
+          else umma_unit_f16(d0, a0, bdesc_dn + (uint64_t)(kg0 * 16), 32u, idesc, acc0, false);   // 2 groups of 256 B
         }
         umma_commit_warp(&c->abempty[ab]);
         ++ua;
         if (PER_UNIT) {
-          umma_commit_warp(&c->accfull[t & 1u]);
+          umma_commit_warp(&c->accfull[t % NACC]);
           ++t;
         }
       }
       if (!PER_UNIT) {
-        umma_commit_warp(&c->accfull[t & 1u]);
+        umma_commit_warp(&c->accfull[t % NACC]);
         ++t;
       }
     };
@@ -399,11 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     uint32_t t = 0;
     bool ok = true;
     auto take = [&](uint32_t* v, uint32_t* w2) {   // the next accumulator tile
-      const uint32_t buf = t & 1u;
-      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t >> 1) & 1u);
+      const uint32_t buf = t % NACC;
+      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / NACC) & 1u);
       tc_fence_after();
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf, v);
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf + 16u, w2);
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + acc_col(buf), v);
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + acc_col(buf) + 16u, w2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c->accempty[buf]);
