@@ -146,8 +146,11 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   const uint32_t tmem = c->tmem_base;
   trace(p, 0, tid == 0);
 
-  // unit bytes in the ring and the first byte of a segment's block
+  // unit bytes in the ring and the first byte of a segment's block; a ring
+  // stage holds one gate/up unit or two down units (one copy of 2 MAT bytes:
+  // a single down unit of MXFP4 would be a copy too small to stream well)
   auto unit_bytes = [&](const Seg& sg) { return sg.list != L_DN ? 2u * MAT : MAT; };
+  auto stage_units = [&](const Seg& sg) { return sg.list != L_DN ? 1 : 2; };
   auto block_base = [&](const Seg& sg) -> const uint8_t* {
     const int e = seg_expert(p, c, sg.x);
     if (sg.list != L_DN) return p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT;
@@ -169,14 +172,16 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         sc_base = sg.list != L_DN ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * geo.upb_gu) * 256
                                   : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * geo.upb_dn) * 128;
       }
-      for (int u = sg.k0; u < sg.k1; ++u) {
+      const int per = stage_units(sg);
+      for (int u = sg.k0; u < sg.k1; u += per) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
+        const uint32_t n = (uint32_t)min(per, sg.k1 - u), bytes = n * ub;
         if (ok && q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
         if (ok) {
-          mbar_arrive_expect_tx(&full[slot], ub);
-          tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, ub, &full[slot]);
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
           issued = s + 1;
-          if (PER_UNIT) prefetch_l2(sc_base + (size_t)u * sc_unit, sc_unit * 4);   // read by the epilogue
+          if (PER_UNIT) prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
         }
         ++s;
       }
@@ -358,36 +363,40 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   bool cok = true;
   auto convert_units = [&](const Seg& sg) {
     const bool gu = sg.list != L_DN;
-    for (int u = sg.k0; u < sg.k1; ++u) {
-      const uint32_t slot = s % p.nst, q = s / p.nst, ab = ua % kAb;
+    const int per = stage_units(sg);
+    for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+      const uint32_t slot = s % p.nst, q = s / p.nst;
+      const int n = min(per, sg.k1 - u0);
       // lane 0 waits; the warp follows its answer (tcgen05.st is warp-wide)
       if (lane == 0 && cok) cok = wait_bar(p, c, &full[slot], q & 1);
-      if (lane == 0 && ua >= kAb && cok) cok = wait_bar(p, c, &c->abempty[ab], ((ua / kAb) - 1) & 1u);
-      cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
-      tc_fence_after();
-      const uint8_t* st = ring + (size_t)slot * p.slot_bytes;
-      const uint32_t col = lane_base + kAbCol + 128u * ab;
-      if (cok) {
-        if (NCV == 4) {
-          tq_convert<WT>(st, row, col, 0, F::CHUNKS);
-          if (gu) tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
-        } else if (gu) {
-          if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS);
-          else tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
-        } else {
-          if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS / 2);
-          else tq_convert<WT>(st, row, col, F::CHUNKS / 2, F::CHUNKS);
+      cok = __shfl_sync(0xffffffffu, (int)cok, 0) != 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t ab = ua % kAb;
+        if (lane == 0 && ua >= kAb && cok) cok = wait_bar(p, c, &c->abempty[ab], ((ua / kAb) - 1) & 1u);
+        cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
+        tc_fence_after();
+        const uint8_t* st = ring + (size_t)slot * p.slot_bytes + (size_t)j * MAT;
+        const uint32_t col = lane_base + kAbCol + 128u * ab;
+        if (cok) {
+          if (NCV == 4) {
+            tq_convert<WT>(st, row, col, 0, F::CHUNKS);
+            if (gu) tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
+          } else if (gu) {
+            if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS);
+            else tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
+          } else {
+            if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS / 2);
+            else tq_convert<WT>(st, row, col, F::CHUNKS / 2, F::CHUNKS);
+          }
         }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c->abfull[ab]);
+        ++ua;
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&c->abfull[ab]);
-        mbar_arrive(&empty[slot]);
-      }
+      if (lane == 0) mbar_arrive(&empty[slot]);   // every unit of the stage is read
       ++s;
-      ++ua;
     }
   };
 

@@ -132,6 +132,29 @@ def test_scaled_fp8_rows4():
     run.close()
 
 
+def test_cuda_core_fp8_fp32_streams():
+    """FP8 experts with fp32 residual streams and no bf16 rounding: the
+    CUDA-core kernel (the tensor-core kernels take only the rounded layer);
+    compared at the fp32 tolerance."""
+    wl = C.scaled(C.FLASH_FP8_R4, seed=311, hc_dtype="f32", norm_dtype="f32", round_bf16=False)
+    run = GpuRun(wl)
+    assert run.plan.info()["ring_slot_bytes"] != 2 * 16384   # not the tensor-core layout
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
+def test_cuda_core_mxfp4_hidden_not_multiple_of_128():
+    """MXFP4 with hidden 1056 and inter 544 (multiples of 32, not of 128): the
+    CUDA-core kernel."""
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=411, hidden=1056, inter=544, rows=3)
+    run = GpuRun(wl)
+    assert run.plan.info()["ring_slot_bytes"] != 2 * (8192 + 512)
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
 def test_scaled_mxfp4_single_layer():
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=401)
     run = GpuRun(wl)
