@@ -200,16 +200,15 @@ __device__ bool wait_count(const Params& p, Ctl* c, const uint32_t* cnt, uint32_
 
 __device__ bool wait_bar(const Params& p, Ctl* c, uint64_t* bar, uint32_t parity) {
   volatile int* dead = &c->dead;
-  if (mbar_test(bar, parity)) return true;
+  if (mbar_try(bar, parity)) return true;   // waits in hardware, wakes on the phase
   uint64_t t0 = globaltimer();
   while (true) {
     if (*dead) return false;
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
     if (globaltimer() - t0 > 2 * p.timeout_ns) {   // downstream of the grid-wide waits
       record_error(p, c, 7u, 5u);
       return false;
     }
-    __nanosleep(20);
   }
 }
 

@@ -806,6 +806,8 @@ extern "C" int mono_ffn_get_info(const mono_ffn_plan_t* p, mono_ffn_info* info) 
   info->ring_stages = p->nst;
   info->ring_slot_bytes = p->slot_bytes;
   info->expert_bytes = p->gu_estride + p->dn_estride;
+  if (p->tq && p->wt == W_FP8)   // the FP8 block scales travel in their own arrays
+    info->expert_bytes += (int64_t)(p->cfg.inter / 128) * (H / 128) * 256 * 4 + (int64_t)(H / 128) * (p->cfg.inter / 128) * 128 * 4;
   info->dense_bytes = (int64_t)kS * H * kMixC * 4 + (int64_t)E * H * 4 + (int64_t)E * 4 +
                       (int64_t)H * (p->cfg.norm_dtype == MONO_BF16 ? 2 : 4);
   info->packed_bytes = p->packed_bytes;

@@ -417,10 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       if (lane == 0) mbar_arrive(&c->accempty[buf]);
       ++t;
     };
-    auto seg = [&](const Seg& sg) {
+    // the accumulator work of a segment (its conversion is done)
+    auto finish = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
       const int upb = gu ? geo.upb_gu : geo.upb_dn;
-      if (converts) convert_units(sg);
       float a[8], b[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
@@ -469,11 +469,35 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
       epi_store(p, c, geo, sg, gu, live, i, a, b);
     };
+    // When these warps also convert (MXFP4), a segment's accumulator work
+    // waits until the next segment of the list is converted: the MMAs of
+    // that segment run meanwhile (the accumulators alternate).  The last
+    // segment of a list is finished before the next list starts converting
+    // (a down expert may wait for this CTA's own gate/up block).
+    Seg pend;
+    bool has_pend = false;
+    auto seg = [&](const Seg& sg) {
+      if (!converts) {
+        finish(sg);
+        return;
+      }
+      convert_units(sg);
+      if (has_pend) finish(pend);
+      pend = sg;
+      has_pend = true;
+    };
+    auto flush = [&]() {
+      if (has_pend) finish(pend);
+      has_pend = false;
+    };
     tc_segments(p, geo, L_SGU, 0, seg);
+    flush();
     trace(p, 6, tid == 0);
     tc_segments(p, geo, L_RGU, nu, seg);
+    flush();
     trace(p, 7, tid == 0);
     tc_segments(p, geo, L_DN, nu, seg);
+    flush();
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
     if (tid == 0) {
