@@ -132,6 +132,17 @@ def test_scaled_fp8_rows4():
     run.close()
 
 
+def test_cuda_core_bf16_hidden_not_multiple_of_128():
+    """bf16 experts with hidden 1056 and inter 544: not whole 128-row blocks,
+    so the CUDA-core kernel."""
+    wl = C.scaled(C.FLASH_BF16_R8, seed=221, hidden=1056, inter=544, rows=5)
+    run = GpuRun(wl)
+    assert run.plan.info()["ring_slot_bytes"] != 16384   # not the tensor-core layout
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
 def test_cuda_core_fp8_fp32_streams():
     """FP8 experts with fp32 residual streams and no bf16 rounding: the
     CUDA-core kernel (the tensor-core kernels take only the rounded layer);
