@@ -147,6 +147,10 @@ struct Ctl {
   uint64_t bfull;               // the down projection's B operand has landed
   uint64_t abfull[kMaxAb], abempty[kMaxAb];   // quantised tensor-core kernel: converted A tiles in tensor memory
   volatile int bcast;           // epilogue: "this CTA completes the block"
+  // FP8 tensor-core kernel: inverse power-of-two scale of each row of n, and
+  // the epilogue warps' per-row maxima of a block's activations
+  float nsc[kMaxR];
+  float amax[4][kMaxR];
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

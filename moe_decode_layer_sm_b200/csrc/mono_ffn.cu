@@ -13,6 +13,7 @@
 #include "cc_kernel.cuh"
 #include "tc_kernel.cuh"
 #include "tq_kernel.cuh"
+#include "tf8_kernel.cuh"
 
 using namespace mono;
 
@@ -108,7 +109,7 @@ void* kernel_ptr() {
 
 void* kernel_for(int wt, bool tc, bool tq) {
   if (tc) return reinterpret_cast<void*>(&mono_ffn_tc_kernel<W_BF16>);
-  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP8>)
+  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tf8_kernel)
                              : reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP4>);
   switch (wt) {
     case W_F32: return kernel_ptr<W_F32>();

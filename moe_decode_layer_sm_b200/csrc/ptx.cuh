@@ -261,6 +261,53 @@ __device__ __forceinline__ void umma_unit_f16(uint32_t d, uint32_t a, uint64_t d
   }
 }
 
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0 in both
+// fields), fp32 accumulator, both K-major, M = m, N = n.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int m, int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// One 128 x 128 e4m3 unit from shared memory, issued by one elected lane of
+// a converged warp: 4 K-steps of 32 (kind::f8f6f4), the first overwriting D.
+// A advances 4096 bytes a K-step (256 descriptor units), B db_step units.
+// pair: a second A matrix (up) 16384 bytes on, into d + 16.
+__device__ __forceinline__ void umma_unit_e4m3(uint32_t d, uint64_t da, uint64_t db, uint32_t db_step, uint32_t idesc,
+                                               bool pair) {
+  if (pair) {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, d1;\n .reg .b64 a0, a1, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " mov.b64 a0, %1;\n add.u64 a1, %1, 1024;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, f;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], a1, b, %4, f;\n"
+        " add.u64 a0, a0, 256;\n add.u64 a1, a1, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], a1, b, %4, t;\n"
+        " add.u64 a0, a0, 256;\n add.u64 a1, a1, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], a1, b, %4, t;\n"
+        " add.u64 a0, a0, 256;\n add.u64 a1, a1, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], a1, b, %4, t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx;\n .reg .b64 a0, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " mov.b64 a0, %1;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, f;\n"
+        " add.u64 a0, a0, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        " add.u64 a0, a0, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        " add.u64 a0, a0, 256;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a0, b, %4, t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
+        : "memory");
+  }
+}
+
 // 32 lanes x 16 consecutive 32-bit columns from registers (thread l of the
 // warp writes its quadrant's lane l)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {

@@ -1,0 +1,518 @@
+// FP8 experts on the tensor cores with no conversion pass: tcgen05.mma of
+// kind::f8f6f4 reads the e4m3 weight codes straight from the ring (A, in
+// shared memory), and the activations as e4m3 as well (B).
+//
+// An activation vector y goes into B as two e4m3 terms after a power-of-two
+// scale 2^e that puts its largest magnitude in [128, 256): hi = e4m3(y 2^e)
+// and lo = e4m3(y 2^e - hi).  B rows 0-7 carry hi of the 8 token rows, rows
+// 8-15 lo; the epilogue adds the two halves of the accumulator and multiplies
+// by 2^-e (exact).  A bf16 value has 8 significant bits and hi and lo hold 4
+// each, so n (bf16) is represented exactly down to 2^-9 of its row's largest
+// magnitude; smaller values, and the SwiGLU activations (fp32), keep an
+// absolute error below 2^-10 of the scaled unit, about 2^-17 of the block's
+// largest magnitude.
+//   gate/up B: n, one scale per token row
+//   down B:    the activations, one scale per (token row, 128-block of I),
+//              chosen by the epilogue that completes the gate/up block and
+//              stored behind the expert's codes
+// The FP8 block scales (fp32, one per 1 x 128 block of a weight row) scale
+// each unit's fp32 tile in the epilogue, so every unit gets its own
+// accumulator (four in flight).
+//
+// Packed units as in the converting kernel: [8 chunks][128 rows][16] e4m3,
+// chunk j of row i at [j][i]: K-major core matrices of 8 rows x 16 bytes,
+// 2048 bytes between K-neighbours and 128 between row groups.  A ring stage
+// is one gate/up unit (gate, then up) or two down units, 32 KB.
+#pragma once
+#include <cuda_fp8.h>
+
+#include "tq_kernel.cuh"
+
+namespace mono {
+
+constexpr int kF8TmemCols = 128;   // four accumulators of 32 columns (gate 16 | up 16)
+constexpr uint32_t kF8Acc = 4;
+static_assert(kF8Acc <= (uint32_t)kMaxAcc, "accumulator barriers");
+
+// bytes of one expert entry's down B operand: [I/16][16 rows][16] e4m3 codes,
+// then [I/128][8] fp32 inverse scales
+__host__ __device__ inline size_t f8_act_stride(int I) { return (size_t)I * 16 + (size_t)(I / 128) * 32; }
+
+// e with m 2^e in [128, 256) for m > 0 (0 for m = 0), within [-126, 126] so
+// that 2^e and 2^-e are normal floats
+__device__ __forceinline__ int f8_exp(float m) {
+  if (!(m > 0.f)) return 0;
+  const int ex = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;   // floor(log2 m) for normal m
+  return max(-126, min(126, 7 - ex));
+}
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// two scaled values -> e4m3 hi and lo code pairs (the first value in the low byte)
+__device__ __forceinline__ void f8_split2(float y0, float y1, uint32_t& hi, uint32_t& lo) {
+  const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+  const float2 hf = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3)));
+  const __nv_fp8x2_storage_t l =
+      __nv_cvt_float2_to_fp8x2(make_float2(y0 - hf.x, y1 - hf.y), __NV_SATFINITE, __NV_E4M3);
+  hi = h;
+  lo = l;
+}
+
+// n, bf16 in the layout [H/8][8 rows][8], becomes the e4m3 B operand
+// [H/16][16 rows][16] (rows 0-7 hi, 8-15 lo) in place, one 128-column block
+// per warp at a time (the two layouts put a block in the same 2 KB); c->nsc
+// gets each row's inverse scale.  Compute warps.
+__device__ void f8_convert_n(const Params& p, Ctl* c, uint8_t* regA) {
+  const int H = p.H, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // row maxima: 16-byte item q of the bf16 layout holds row q & 7, and this
+  // thread's items all have row tid & 7
+  float m = 0.f;
+  for (int q = tid; q < H; q += kCW * 32) {
+    const uint4 v = *reinterpret_cast<const uint4*>(regA + (size_t)q * 16);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x))), fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y)))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))), fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w)))));
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+  if (lane < 8) c->sq[warp][lane] = m;
+  bar_sync(kBarCons, kCW * 32);
+  const int r = lane & 7, q = lane >> 3;
+  float mr = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCW; ++w) mr = fmaxf(mr, c->sq[w][r]);
+  const int e = f8_exp(mr);
+  if (tid < 8) c->nsc[tid] = pow2i(-e);
+  const float sc = pow2i(e);
+  // lane (r, q): columns 32 q .. 32 q + 31 of row r of the block, i.e. bf16
+  // chunks 4q .. 4q + 3 in, e4m3 chunks 2q and 2q + 1 out
+  for (int kb = warp; kb < H / 128; kb += kCW) {
+    uint8_t* blk = regA + (size_t)kb * 2048;
+    uint4 v[4];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) v[cc] = *reinterpret_cast<const uint4*>(blk + (4 * q + cc) * 128 + r * 16);
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int m2 = 0; m2 < 4; ++m2) {
+        const uint4 s = v[2 * h + (m2 >> 1)];
+        const uint32_t w0 = (m2 & 1) ? s.z : s.x, w1 = (m2 & 1) ? s.w : s.y;
+        uint32_t h01, l01, h23, l23;
+        f8_split2(bf16lo(w0) * sc, bf16hi(w0) * sc, h01, l01);
+        f8_split2(bf16lo(w1) * sc, bf16hi(w1) * sc, h23, l23);
+        hi[m2] = h01 | (h23 << 16);
+        lo[m2] = l01 | (l23 << 16);
+      }
+      *reinterpret_cast<uint4*>(blk + (2 * q + h) * 256 + r * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(blk + (2 * q + h) * 256 + (8 + r) * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+}
+
+// A complete gate/up block: SwiGLU, then each token row's 128 activations of
+// the block as e4m3 hi/lo under the block's power-of-two scale, into the
+// down B operand of expert entry x, with the inverse scale behind the codes;
+// zero for rows that do not use the expert.  Then the block counts for its
+// expert.  Every epilogue thread, live or not.
+__device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg& sg, bool live, int i,
+                                             const float (&a)[8], const float (&b)[8]) {
+  const int R = p.R, K = p.K, I = p.I, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int x = sg.x;
+  float act[8];
+#pragma unroll
+  for (int r = 0; r < kMaxR; ++r) {
+    const int sl = x == 0 ? K : c->uslot[x - 1][r];
+    act[r] = 0.f;
+    if (live && r < R && sl >= 0) {
+      float gg = a[r], uu = b[r];
+      if (p.round_bf16) {
+        gg = round_bf16(gg);
+        uu = round_bf16(uu);
+      }
+      act[r] = gg / (1.0f + expf(-gg)) * uu;
+    }
+    const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(act[r])));
+    if (lane == 0) c->amax[warp][r] = __uint_as_float(mb);
+  }
+  bar_sync(kBarEpi, 4 * 32);
+  uint8_t* base = p.actb + (size_t)x * f8_act_stride(I);
+  const int ch = sg.blk * 128 + i;
+  uint8_t* dst = base + (size_t)(ch >> 4) * 256 + (ch & 15);
+#pragma unroll
+  for (int r = 0; r < kMaxR; r += 2) {
+    int e[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int rr = r + k;
+      e[k] = f8_exp(fmaxf(fmaxf(c->amax[0][rr], c->amax[1][rr]), fmaxf(c->amax[2][rr], c->amax[3][rr])));
+    }
+    uint32_t hb, lb;
+    f8_split2(act[r] * pow2i(e[0]), act[r + 1] * pow2i(e[1]), hb, lb);
+    if (live) {
+      dst[r * 16] = (uint8_t)(hb & 0xFFu);
+      dst[(r + 1) * 16] = (uint8_t)(hb >> 8);
+      dst[(8 + r) * 16] = (uint8_t)(lb & 0xFFu);
+      dst[(9 + r) * 16] = (uint8_t)(lb >> 8);
+      float* inv = reinterpret_cast<float*>(base + (size_t)I * 16) + sg.blk * 8;
+      if (i == r) inv[r] = pow2i(-e[0]);
+      if (i == r + 1) inv[r + 1] = pow2i(-e[1]);
+    }
+  }
+  // the block's activations are out: count it for its expert (the codes are
+  // read by a bulk copy, the async proxy; the scales by the epilogues)
+  __threadfence();
+  bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
+  if (tid == 0 && live) {
+    fence_proxy_async_global();
+    red_release_add(&p.xready[x], 1u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_constant__ Params p) {
+  constexpr uint32_t MAT = TqFmt<W_FP8>::MAT_BYTES;   // one unit of one matrix
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const SmemLayout L(p.nst, p.slot_bytes, p.regA_bytes, p.ymax);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + p.nst;
+  Ctl* c = reinterpret_cast<Ctl*>(smem + L.ctl);
+  uint8_t* regA = smem + L.regA;   // n (gate/up B operand), then the down B operand
+  uint8_t* ring = smem + L.ring;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int H = p.H, I = p.I, K = p.K, G = p.G;
+  const TcGeo geo(p);
+
+  if (tid == 0) {
+    c->dead = 0;
+    c->lists_ready = 0;
+    c->nu = 0;
+    c->n_ready = 0;
+    c->epoch = ld_relaxed(&p.sync->epoch);
+    if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
+    for (int s = 0; s < p.nst; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);   // the MMAs' commit
+    }
+    for (uint32_t b = 0; b < kF8Acc; ++b) {
+      mbar_init(&c->accfull[b], 1);
+      mbar_init(&c->accempty[b], 4);
+    }
+    mbar_init(&c->drain, 1);
+    mbar_init(&c->bfull, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (c->dead) return;
+  if (warp == kMmaWarp) tmem_alloc(&c->tmem_base, kF8TmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t ep1 = c->epoch + 1u;
+  const uint32_t tmem = c->tmem_base;
+  trace(p, 0, tid == 0);
+
+  // a ring stage: one gate/up unit (gate, up) or two down units
+  auto stage_units = [&](const Seg& sg) { return sg.list != L_DN ? 1 : 2; };
+
+  // ================================================================ producer
+  if (warp == kProdWarp) {
+    uint32_t s = 0, issued = 0;
+    bool ok = true;
+    auto seg = [&](const Seg& sg) {
+      if (lane != 0) return;
+      const int e = seg_expert(p, c, sg.x);
+      const bool gu = sg.list != L_DN;
+      const uint8_t* base = gu ? p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT
+                               : p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * geo.upb_dn * MAT;
+      const uint32_t ub = gu ? 2u * MAT : MAT;
+      const uint32_t sc_unit = gu ? 256u : 128u;   // block scales of one unit
+      const float* sc_base = gu ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * geo.upb_gu) * 256
+                                : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * geo.upb_dn) * 128;
+      const int per = stage_units(sg);
+      for (int u = sg.k0; u < sg.k1; u += per) {
+        const uint32_t slot = s % p.nst, q = s / p.nst;
+        const uint32_t n = (uint32_t)min(per, sg.k1 - u), bytes = n * ub;
+        if (ok && q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
+        if (ok) {
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
+          issued = s + 1;
+          prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
+        }
+        ++s;
+      }
+    };
+    if (lane == 0) {
+      const int e0 = (int)((long long)blockIdx.x * p.E / G), e1 = (int)((long long)(blockIdx.x + 1) * p.E / G);
+      prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
+      prefetch_l2_span(p.norm_w, (size_t)H * (p.norm_bf16 ? 2 : 4));
+      prefetch_l2_span(p.bias, (size_t)p.E * 4);
+    }
+    tc_segments(p, geo, L_SGU, 0, seg);
+    if (ok && lane == 0) ok = wait_flag(p, c, &c->lists_ready);
+    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    const int nu = ok ? *(volatile int*)&c->nu : 0;
+    trace(p, 11, lane == 0);
+    tc_segments(p, geo, L_RGU, nu, seg);
+    tc_segments(p, geo, L_DN, nu, seg);
+    trace(p, 12, lane == 0);
+    if (lane == 0) {   // no bulk copy may still target this CTA's shared memory at exit
+      const uint32_t first = issued > (uint32_t)p.nst ? issued - p.nst : 0;
+      for (uint32_t t = first; t < issued; ++t) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_test(&full[t % p.nst], (t / p.nst) & 1)) {
+          if (globaltimer() - t0 > p.timeout_ns) break;
+          __nanosleep(64);
+        }
+      }
+    }
+    return;
+  }
+
+  // =========================================================== MMA issuer
+  if (warp == kMmaWarp) {
+    uint32_t s = 0, t = 0, ndrain = 0, nb = 0;
+    int prev_x = -1;
+    bool first_rgu = true, b_pending = false;
+    auto warp_ok = [&](bool v) { return __shfl_sync(0xffffffffu, (int)v, 0) != 0; };
+    bool ok = true;
+    if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
+    ok = warp_ok(ok);
+    const uint32_t idesc = umma_idesc_e4m3(128, 16);
+    const uint32_t b_bytes = (uint32_t)I * 16u;
+    // B (n, or a down expert's activations): [K/16][16 rows][16], 256 bytes
+    // between K-neighbours, rows 8-15 128 bytes on; a unit is 2048 bytes
+    const uint64_t bdesc = umma_desc(smem_u32(regA), 256u, 128u);
+    auto seg = [&](const Seg& sg) {
+      const bool gu = sg.list != L_DN;
+      if (!gu && sg.x != prev_x) {
+        // a new down expert: its activations complete, every MMA on the B
+        // region done, then one bulk copy of this expert's operand
+        if (lane == 0 && ok) ok = wait_count(p, c, &p.xready[sg.x], (uint32_t)geo.nbi, 4u);
+        ok = warp_ok(ok);
+        fence_proxy_async_global();
+        trace(p, 8, prev_x < 0 && lane == 0);
+        umma_commit_warp(&c->drain);
+        if (lane == 0 && ok) ok = wait_bar(p, c, &c->drain, ndrain & 1u);
+        ok = warp_ok(ok);
+        ++ndrain;
+        tc_fence_after();
+        prev_x = sg.x;
+        if (ok) {   // (a copy whose wait failed is waited for again at exit)
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&c->bfull, b_bytes);
+            tma_load_1d(regA, p.actb + (size_t)sg.x * f8_act_stride(I), b_bytes, &c->bfull);
+            ok = wait_bar(p, c, &c->bfull, nb & 1u);
+          }
+          ok = warp_ok(ok);
+          b_pending = !ok;
+          ++nb;
+        }
+        tc_fence_after();
+        trace(p, 15, nb == 1 && lane == 0);
+      }
+      const int per = stage_units(sg);
+      for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+        const uint32_t slot = s % p.nst, q = s / p.nst;
+        const int n = min(per, sg.k1 - u0);
+        if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
+        ok = warp_ok(ok);
+        tc_fence_after();
+        if (sg.list == L_RGU && first_rgu) {
+          first_rgu = false;
+          trace(p, 13, lane == 0);
+        }
+        for (int j = 0; j < n; ++j) {
+          const int u = u0 + j;
+          const uint32_t buf = t % kF8Acc;
+          if (t >= kF8Acc) {
+            if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / kF8Acc) - 1) & 1u);
+            ok = warp_ok(ok);
+          }
+          tc_fence_after();
+          if (ok) {
+            const uint64_t da = umma_desc(smem_u32(ring + (size_t)slot * p.slot_bytes + (size_t)j * MAT), 2048u, 128u);
+            umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
+          }
+          umma_commit_warp(&c->accfull[buf]);
+          ++t;
+        }
+        umma_commit_warp(&empty[slot]);
+        ++s;
+      }
+    };
+    tc_segments(p, geo, L_SGU, 0, seg);
+    if (lane == 0 && ok) ok = wait_flag(p, c, &c->lists_ready);
+    ok = warp_ok(ok);
+    const int nu = ok ? *(volatile int*)&c->nu : 0;
+    tc_segments(p, geo, L_RGU, nu, seg);
+    trace(p, 14, lane == 0);
+    tc_segments(p, geo, L_DN, nu, seg);
+    trace(p, 16, lane == 0);
+    // every MMA of this CTA is complete before the tensor memory goes away,
+    // and no bulk copy still targets shared memory at exit
+    umma_commit_warp(&c->drain);
+    if (lane == 0) {
+      const uint64_t t0 = globaltimer();
+      while (!mbar_test(&c->drain, ndrain & 1u) && globaltimer() - t0 < p.timeout_ns) __nanosleep(64);
+      while (b_pending && !mbar_test(&c->bfull, (nb - 1) & 1u) && globaltimer() - t0 < 2 * p.timeout_ns)
+        __nanosleep(64);
+    }
+    __syncwarp();
+    bar_sync(kBarEnd, 5 * 32);
+    tc_fence_after();
+    tmem_dealloc(tmem, kF8TmemCols);
+    return;
+  }
+
+  // ================================================================ prologue
+  prologue_mix(p, c, regA, ep1);
+  if (warp >= kCtlWarp0) {
+    control_warps(p, c, regA, ep1, false);
+    return;
+  }
+  collapse_norm<true>(p, c, regA, ep1);
+  // the router reads n as bf16 (the layer's values); the MMAs then take it
+  // as e4m3 hi/lo
+  router_logits<true>(p, c, regA, false);
+  f8_convert_n(p, c, regA);
+  fence_proxy_async_smem();   // n is read by the tensor cores (async proxy)
+  bar_sync(kBarCons, kCW * 32);
+  if (tid == 0) *(volatile int*)&c->n_ready = 1;
+  trace(p, 3, tid == 0);
+  route_rows(p, c, ep1);
+
+  // the compute warps agree on the expert list once
+  if (tid == 0) {
+    const bool ok = wait_flag(p, c, &c->lists_ready);
+    c->nu_comp = (ok && !c->dead) ? c->nu : 0;
+  }
+  bar_sync(kBarCons, kCW * 32);
+  const int nu = c->nu_comp;
+
+  if (warp < 4) {
+    // ============================================================ epilogue
+    // thread <-> row i = 32 w + l of the 128-row tile (its TMEM lane)
+    const int i = tid;
+    uint32_t t = 0;
+    bool ok = true;
+    auto take = [&](uint32_t* v, uint32_t* w2, bool gu) {   // the next unit's tile
+      const uint32_t buf = t % kF8Acc;
+      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / kF8Acc) & 1u);
+      tc_fence_after();
+      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf;
+      tmem_ld16(ta, v);
+      if (gu) tmem_ld16(ta + 16u, w2);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c->accempty[buf]);
+      ++t;
+    };
+    auto seg = [&](const Seg& sg) {
+      const bool gu = sg.list != L_DN;
+      const int upb = gu ? geo.upb_gu : geo.upb_dn;
+      const int e = seg_expert(p, c, sg.x);
+      float a[8], b[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
+      uint32_t v[16], w2[16];
+      // the units' block scales (brought to L2 by the producer), two units ahead
+      const float* sc = gu ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * upb) * 256
+                           : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * upb) * 128;
+      const int us = gu ? 256 : 128;
+      auto ld_g = [&](int u) { return u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
+      auto ld_u = [&](int u) { return gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
+      float sg0 = ld_g(sg.k0), su0 = ld_u(sg.k0), sg1 = ld_g(sg.k0 + 1), su1 = ld_u(sg.k0 + 1);
+      if (gu) {
+        for (int u = sg.k0; u < sg.k1; ++u) {
+          const float sg2 = ld_g(u + 2), su2 = ld_u(u + 2);
+          take(v, w2, true);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            a[r] = fmaf(sg0, __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
+            b[r] = fmaf(su0, __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]), b[r]);
+          }
+          sg0 = sg1;
+          su0 = su1;
+          sg1 = sg2;
+          su1 = su2;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {   // n's row scale, a power of two
+          a[r] *= c->nsc[r];
+          b[r] *= c->nsc[r];
+        }
+      } else {
+        // this expert's activation scales were published with its block
+        // counts: acquire them once (the issuer has seen them complete)
+        if (tid == 0 && ok) ok = wait_count(p, c, &p.xready[sg.x], (uint32_t)geo.nbi, 4u);
+        bar_sync(kBarEpi, 4 * 32);
+        const float4* asc =
+            reinterpret_cast<const float4*>(p.actb + (size_t)sg.x * f8_act_stride(I) + (size_t)I * 16);
+        auto ld_a = [&](int u, float4& lo4, float4& hi4) {
+          const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+          lo4 = u < sg.k1 ? __ldcg(asc + 2 * u) : z;
+          hi4 = u < sg.k1 ? __ldcg(asc + 2 * u + 1) : z;
+        };
+        float4 a0l, a0h, a1l, a1h;
+        ld_a(sg.k0, a0l, a0h);
+        ld_a(sg.k0 + 1, a1l, a1h);
+        for (int u = sg.k0; u < sg.k1; ++u) {
+          const float sg2 = ld_g(u + 2);
+          float4 a2l, a2h;
+          ld_a(u + 2, a2l, a2h);
+          take(v, w2, false);
+          const float k8[8] = {a0l.x, a0l.y, a0l.z, a0l.w, a0h.x, a0h.y, a0h.z, a0h.w};
+#pragma unroll
+          for (int r = 0; r < 8; ++r) a[r] = fmaf(sg0 * k8[r], __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
+          sg0 = sg1;
+          sg1 = sg2;
+          a0l = a1l;
+          a0h = a1h;
+          a1l = a2l;
+          a1h = a2h;
+        }
+      }
+      trace(p, 20, t == 1 && tid == 0);
+      const bool live = ok && !c->dead;
+      if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
+      if (gu) f8_store_act(p, c, sg, live, i, a, b);
+      else epi_store(p, c, geo, sg, false, live, i, a, b);
+    };
+    tc_segments(p, geo, L_SGU, 0, seg);
+    trace(p, 6, tid == 0);
+    tc_segments(p, geo, L_RGU, nu, seg);
+    trace(p, 7, tid == 0);
+    tc_segments(p, geo, L_DN, nu, seg);
+    trace(p, 9, tid == 0);
+    bar_sync(kBarEpi, 4 * 32);
+    if (tid == 0) {
+      __threadfence();
+      red_release_add(&p.sync->cnt_y, 1u);
+    }
+    tc_fence_before();
+    bar_arrive(kBarEnd, 5 * 32);   // the issuer may free the tensor memory
+  }
+  // warps 4-7 have no part in the main phase
+
+  // ==================================================================== tail
+  bar_sync(kBarCons, kCW * 32);
+  if (tid == 0) wait_count(p, c, &p.sync->cnt_y, ep1 * (uint32_t)G, 6u);
+  bar_sync(kBarCons, kCW * 32);
+  tail(p, c, [&](int r, int h) {
+    const float* src = p.yp + (size_t)r * (K + 1) * H + h;
+    float v[kMaxK + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) v[j] = j <= K ? __ldcg(src + (size_t)j * H) : 0.f;
+    float y = 0.f;
+#pragma unroll
+    for (int j = 0; j <= kMaxK; ++j) y += v[j];   // slot order; the zero padding adds exactly
+    return y;
+  });
+  bar_sync(kBarCons, kCW * 32);
+  trace(p, 10, tid == 0);
+  finish_step(p, c, ep1);
+}
+
+}  // namespace mono
