@@ -109,8 +109,8 @@ void* kernel_ptr() {
 
 void* kernel_for(int wt, bool tc, bool tq) {
   if (tc) return reinterpret_cast<void*>(&mono_ffn_tc_kernel<W_BF16>);
-  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tf8_kernel)
-                             : reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP4>);
+  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tf8_kernel<W_FP8>)
+                             : reinterpret_cast<void*>(&mono_ffn_tf8_kernel<W_FP4>);
   switch (wt) {
     case W_F32: return kernel_ptr<W_F32>();
     case W_BF16: return kernel_ptr<W_BF16>();
@@ -141,31 +141,45 @@ __global__ void pack_tc_kernel(const uint16_t* src, uint8_t* dst, long long e1, 
 // j of unit-row i at j * 2048 + i * 16 inside the unit's matrix slot msub:
 //   dst[((e * rows/128 + row/128) * nu + u) * ustride + msub + j * 2048 + (row % 128) * 16]
 __global__ void pack_tq_codes_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int row_bytes, int ub,
-                                     long long ustride, int msub) {
+                                     long long ustride, int msub, int f4) {
   const int nch = row_bytes / 16, nu = row_bytes / ub, cpu = ub / 16, NB = rows / 128;
   const long long n = e1 * rows * nch;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int ch = (int)(i % nch);
     const long long row = (i / nch) % rows, e = i / ((long long)nch * rows);
     const int u = ch / cpu, j = ch % cpu;
-    const uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)ch * 16);
+    uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)ch * 16);
+    if (f4) v = make_uint4(f4_pack_word(v.x), f4_pack_word(v.y), f4_pack_word(v.z), f4_pack_word(v.w));
     const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + (long long)j * 2048 + (row % 128) * 16;
     *reinterpret_cast<uint4*>(dst + off) = v;
   }
 }
 
-// MXFP4 e8m0 scales [E+1][rows][cols/32] -> the 4 scales of each unit-row
-// after the unit's codes: dst[unit * ustride + msub + code_bytes + (row % 128) * 4 + jj]
-__global__ void pack_tq_e8m0_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int ns, long long ustride,
-                                    int msub, int code_bytes) {
+// MXFP4 e8m0 scales [E+1][rows][ns] -> per weight row the reference
+// exponent s_ref = (largest scale exponent) - 6, stored as 2^s_ref in
+// ref[E+1][rows/128][nm * 128] (slot m as below), and per block d = s - s_ref
+// as int8 (at least -127) after each unit's codes, 4 per unit-row:
+// dst[unit * ustride + msub + code_bytes + (row % 128) * 4 + jj]
+__global__ void pack_tq_rel_kernel(const uint8_t* src, uint8_t* dst, float* ref, long long e1, int rows, int ns,
+                                   long long ustride, int msub, int code_bytes, int nm, int m) {
   const int nu = ns / 4, NB = rows / 128;
-  const long long n = e1 * rows * nu;
+  const long long n = e1 * rows;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const int u = (int)(i % nu);
-    const long long row = (i / nu) % rows, e = i / ((long long)nu * rows);
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(src + (e * rows + row) * ns + (long long)u * 4);
-    const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + code_bytes + (row % 128) * 4;
-    *reinterpret_cast<uint32_t*>(dst + off) = v;
+    const long long row = i % rows, e = i / rows;
+    const uint8_t* sc = src + (e * rows + row) * ns;
+    int mx = 0;
+    for (int k = 0; k < ns; ++k) mx = max(mx, (int)sc[k]);
+    const int sref = mx - 127 - 6;
+    ref[(e * NB + row / 128) * (nm * 128) + m * 128 + row % 128] = ldexpf(1.0f, sref);
+    for (int u = 0; u < nu; ++u) {
+      uint32_t v = 0;
+      for (int jj = 0; jj < 4; ++jj) {
+        const int d = max(-127, (int)sc[u * 4 + jj] - 127 - sref);
+        v |= (uint32_t)(uint8_t)(int8_t)d << (8 * jj);
+      }
+      const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + code_bytes + (row % 128) * 4;
+      *reinterpret_cast<uint32_t*>(dst + off) = v;
+    }
   }
 }
 
@@ -410,7 +424,9 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->regA_bytes = (int)align_up(regA, 128);
   const int smem_max = prop.sharedMemPerBlockOptin;
   SmemLayout L0(0, p->slot_bytes, p->regA_bytes, p->ymax);
-  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard;
+  // MXFP4 on the tensor cores: two A buffers behind the ring
+  const long long abuf_room = p->tq && dt == MONO_MXFP4 ? (long long)kF4Ab * kF4AbBytes + 1024 : 0;
+  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard - abuf_room;
   p->nst = (int)std::min<long long>(16, room / p->slot_bytes);
   if (p->nst < 2) {
     std::string m = "shared memory: " + std::to_string(smem_max) + " bytes leave room for " + std::to_string(p->nst) +
@@ -419,7 +435,10 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     cudaSetDevice(prev);
     return fail(nullptr, MONO_ERR_INVALID_ARG, m);
   }
-  p->smem = (int)SmemLayout(p->nst, p->slot_bytes, p->regA_bytes, p->ymax).total;
+  {
+    const SmemLayout L1(p->nst, p->slot_bytes, p->regA_bytes, p->ymax);
+    p->smem = (int)(abuf_room ? f4_abuf_off(L1) + (size_t)kF4Ab * kF4AbBytes : L1.total);
+  }
   void* kfn = kernel_for(dt, p->tc, p->tq);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
   int occ = 0;
@@ -444,9 +463,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     if (!rc) rc = dalloc(p, &l.bias, (size_t)E * 4, &p->packed_bytes);
     if (!rc) rc = dalloc(p, &l.gu, (size_t)(E + 1) * p->gu_estride, &p->packed_bytes);
     if (!rc) rc = dalloc(p, &l.dn, (size_t)(E + 1) * p->dn_estride, &p->packed_bytes);
-    if (!rc && p->tq && dt == MONO_FP8E4M3_B128) {
-      rc = dalloc(p, &l.gsc, (size_t)(E + 1) * (I / 128) * (H / 128) * 256 * 4, &p->packed_bytes);
-      if (!rc) rc = dalloc(p, &l.dsc, (size_t)(E + 1) * (H / 128) * (I / 128) * 128 * 4, &p->packed_bytes);
+    if (!rc && p->tq) {
+      // FP8: one block scale per (row, unit); MXFP4: one reference per row
+      const size_t nu_g = dt == MONO_FP8E4M3_B128 ? H / 128 : 1, nu_d = dt == MONO_FP8E4M3_B128 ? I / 128 : 1;
+      rc = dalloc(p, &l.gsc, (size_t)(E + 1) * (I / 128) * nu_g * 256 * 4, &p->packed_bytes);
+      if (!rc) rc = dalloc(p, &l.dsc, (size_t)(E + 1) * (H / 128) * nu_d * 128 * 4, &p->packed_bytes);
     }
   }
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
@@ -543,7 +564,7 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
     const int code_b = fp8 ? 16384 : 8192, ub = fp8 ? 128 : 64;   // unit-row bytes of codes
     const int gu_rb = fp8 ? H : H / 2, dn_rb = fp8 ? I : I / 2;    // code bytes per weight row
     if (!fp8) {
-      // every e8m0 scale must keep e2m1 * scale exact in fp16: 2^-22 .. 2^12
+      // e8m0 code 255 is NaN: not a scale the tensor-core path can expand
       unsigned int* mm = nullptr;
       cudaError_t ea = cudaMalloc(&mm, 8);
       if (ea != cudaSuccess) {
@@ -563,19 +584,17 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
         cudaSetDevice(prev);
         return cuda_fail(p, ea, "pack: scale range");
       }
-      if (got[0] < 127u - 22u || got[1] > 127u + 12u) {
+      if (got[1] > 254u) {
         cudaSetDevice(prev);
-        return fail(p, MONO_ERR_INVALID_ARG,
-                    "pack: MXFP4 scales 2^" + std::to_string((int)got[0] - 127) + " .. 2^" + std::to_string((int)got[1] - 127) +
-                        " leave the range 2^-22 .. 2^12 in which the tensor-core path converts them exactly to fp16");
+        return fail(p, MONO_ERR_INVALID_ARG, "pack: MXFP4 scale code 255 (NaN)");
       }
     }
     pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_gate, l.gu, E + 1, I, gu_rb, ub, 2 * mat, 0);
+        (const uint8_t*)w->w_gate, l.gu, E + 1, I, gu_rb, ub, 2 * mat, 0, !fp8);
     pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_up, l.gu, E + 1, I, gu_rb, ub, 2 * mat, (int)mat);
+        (const uint8_t*)w->w_up, l.gu, E + 1, I, gu_rb, ub, 2 * mat, (int)mat, !fp8);
     pack_tq_codes_kernel<<<grid((long long)(E + 1) * H * (dn_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_down, l.dn, E + 1, H, dn_rb, ub, mat, 0);
+        (const uint8_t*)w->w_down, l.dn, E + 1, H, dn_rb, ub, mat, 0, !fp8);
     if (fp8) {
       pack_tq_scales_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
           (const float*)w->s_gate, l.gsc, E + 1, I, H / 128, 2, 0);
@@ -584,12 +603,12 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
       pack_tq_scales_kernel<<<grid((long long)(E + 1) * H * (I / 128)), th, 0, st>>>(
           (const float*)w->s_down, l.dsc, E + 1, H, I / 128, 1, 0);
     } else {
-      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
-          (const uint8_t*)w->s_gate, l.gu, E + 1, I, H / 32, 2 * mat, 0, code_b);
-      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
-          (const uint8_t*)w->s_up, l.gu, E + 1, I, H / 32, 2 * mat, (int)mat, code_b);
-      pack_tq_e8m0_kernel<<<grid((long long)(E + 1) * H * (I / 128)), th, 0, st>>>(
-          (const uint8_t*)w->s_down, l.dn, E + 1, H, I / 32, mat, 0, code_b);
+      pack_tq_rel_kernel<<<grid((long long)(E + 1) * I), th, 0, st>>>((const uint8_t*)w->s_gate, l.gu, l.gsc, E + 1, I,
+                                                                     H / 32, 2 * mat, 0, code_b, 2, 0);
+      pack_tq_rel_kernel<<<grid((long long)(E + 1) * I), th, 0, st>>>((const uint8_t*)w->s_up, l.gu, l.gsc, E + 1, I,
+                                                                     H / 32, 2 * mat, (int)mat, code_b, 2, 1);
+      pack_tq_rel_kernel<<<grid((long long)(E + 1) * H), th, 0, st>>>((const uint8_t*)w->s_down, l.dn, l.dsc, E + 1, H,
+                                                                     I / 32, mat, 0, code_b, 1, 0);
     }
     cudaError_t e2 = cudaGetLastError();
     cudaSetDevice(prev);
@@ -809,6 +828,8 @@ extern "C" int mono_ffn_get_info(const mono_ffn_plan_t* p, mono_ffn_info* info) 
   info->expert_bytes = p->gu_estride + p->dn_estride;
   if (p->tq && p->wt == W_FP8)   // the FP8 block scales travel in their own arrays
     info->expert_bytes += (int64_t)(p->cfg.inter / 128) * (H / 128) * 256 * 4 + (int64_t)(H / 128) * (p->cfg.inter / 128) * 128 * 4;
+  if (p->tq && p->wt == W_FP4)   // and the MXFP4 row references
+    info->expert_bytes += (int64_t)(2 * p->cfg.inter + H) * 4;
   info->dense_bytes = (int64_t)kS * H * kMixC * 4 + (int64_t)E * H * 4 + (int64_t)E * 4 +
                       (int64_t)H * (p->cfg.norm_dtype == MONO_BF16 ? 2 : 4);
   info->packed_bytes = p->packed_bytes;

@@ -19,10 +19,25 @@
 // each unit's fp32 tile in the epilogue, so every unit gets its own
 // accumulator (four in flight).
 //
-// Packed units as in the converting kernel: [8 chunks][128 rows][16] e4m3,
-// chunk j of row i at [j][i]: K-major core matrices of 8 rows x 16 bytes,
-// 2048 bytes between K-neighbours and 128 between row groups.  A ring stage
-// is one gate/up unit (gate, then up) or two down units, 32 KB.
+// Packed FP8 units as in the converting kernel: [8 chunks][128 rows][16]
+// e4m3, chunk j of row i at [j][i]: K-major core matrices of 8 rows x 16
+// bytes, 2048 bytes between K-neighbours and 128 between row groups.  A ring
+// stage is one gate/up unit (gate, then up) or two down units, 32 KB.
+//
+// MXFP4 takes the same MMAs after one step: warps 4-7 (one thread per weight
+// row) expand each unit's e2m1 codes to e4m3 in shared memory (two A buffers
+// of one ring stage each).  A code times its block scale 2^s is written as
+// the e4m3 value code * 2^(s - s_ref), where s_ref, fixed per weight row at
+// packing, is the row's largest block exponent minus 6: every e2m1 value
+// times 2^d is an e4m3 value for d in [-8, 6] (6 * 2^6 = 384 <= 448; the
+// subnormal step 2^-9 divides 0.5 * 2^-8), so the expansion is exact unless
+// a block's scale lies more than 2^14 below its row's largest, where the
+// values are rounded to e4m3 (an error below 2^-16 of the row's largest
+// scale).  2^s_ref plays the part of the FP8 block scale in the epilogue.
+// Packed MXFP4 units: codes [4 chunks][128 rows][16] (32 e2m1 per chunk, 8
+// a word with the sign bits moved: f4_pack_word), then d = s - s_ref as int8
+// [128 rows][4], 8704 bytes a matrix; the per-row 2^s_ref sit in their own
+// arrays.
 #pragma once
 #include <cuda_fp8.h>
 
@@ -55,6 +70,87 @@ __device__ __forceinline__ void f8_split2(float y0, float y1, uint32_t& hi, uint
       __nv_cvt_float2_to_fp8x2(make_float2(y0 - hf.x, y1 - hf.y), __NV_SATFINITE, __NV_E4M3);
   hi = h;
   lo = l;
+}
+
+// e4m3 of the 8 e2m1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} times 2^d, as
+// bytes 0-3 / 4-7 of a byte-permute table.  For d in [-5, 6] every nonzero
+// entry is a normal e4m3 value and d is added to the exponent field of the
+// d = 0 table (f4_lut_fast); below -5 the values are converted one by one
+// (subnormal, or rounded below -8), out of line since it is rare.
+__device__ __forceinline__ void f4_lut_fast(int d, uint32_t& l0, uint32_t& l1) {
+  const uint32_t de = (uint32_t)(d * 8);
+  l0 = 0x3C383000u + de * 0x01010100u;
+  l1 = 0x4C484440u + de * 0x01010101u;
+}
+__device__ __noinline__ uint2 f4_lut_slow(int d) {
+  const float s = ldexpf(1.0f, max(d, -126));
+  const uint32_t a = __nv_cvt_float2_to_fp8x2(make_float2(0.f, 0.5f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t b = __nv_cvt_float2_to_fp8x2(make_float2(1.0f * s, 1.5f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(2.0f * s, 3.0f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t e = __nv_cvt_float2_to_fp8x2(make_float2(4.0f * s, 6.0f * s), __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(a | (b << 16), c | (e << 16));
+}
+
+// Eight e2m1 codes in the packed word layout of this kernel -> eight e4m3
+// bytes.  The magnitude of code k sits in bits 4k .. 4k + 2 (as in the MXFP4
+// byte stream, two codes a byte, low nibble first); the sign bits are moved at
+// packing (f4_pack_word) to bits 3, 11, 19, 27 for codes 0-3 and 7, 15, 23,
+// 31 for codes 4-7, so that one shift or none puts each on bit 7 of its
+// output byte.  The magnitudes go through the table: one byte permute per
+// four codes.
+__host__ __device__ inline uint32_t f4_pack_word(uint32_t w) {
+  uint32_t o = w & 0x77777777u;
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t sgn = (w >> (4 * k + 3)) & 1u;
+    const int at = k < 4 ? 8 * k + 3 : 8 * (k - 4) + 7;
+    o |= sgn << at;
+  }
+  return o;
+}
+__device__ __forceinline__ void f4x8_to_e4m3(uint32_t w, uint32_t l0, uint32_t l1, uint32_t& o0, uint32_t& o1) {
+  o0 = __byte_perm(l0, l1, w & 0x7777u) | ((w & 0x08080808u) << 4);
+  o1 = __byte_perm(l0, l1, (w >> 16) & 0x7777u) | (w & 0x80808080u);
+}
+
+// One ring stage of MXFP4 (two unit-matrices: gate and up, or two down
+// units; the second is stored only when two), this thread's weight row:
+// codes [4][128 rows][16] and the rows' d [128][4] of each matrix -> e4m3
+// [8][128 rows][16] at dst and dst + 16384.  One copy of the code for every
+// caller (not inlined).
+__device__ __noinline__ void f4_expand_stage(const uint8_t* src, uint8_t* dst, int row, bool two) {
+  constexpr int MAT = 8192 + 512;
+  uint32_t l0[2][4], l1[2][4];
+  uint4 q[2][4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const uint32_t dd = *reinterpret_cast<const uint32_t*>(src + m * MAT + 8192 + row * 4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      q[m][j] = *reinterpret_cast<const uint4*>(src + m * MAT + j * 2048 + row * 16);
+      const int d = (int)(int8_t)((dd >> (8 * j)) & 0xFFu);
+      f4_lut_fast(d, l0[m][j], l1[m][j]);
+      if (d < -5) {
+        const uint2 t = f4_lut_slow(d);
+        l0[m][j] = t.x;
+        l1[m][j] = t.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t w[4] = {q[m][j].x, q[m][j].y, q[m][j].z, q[m][j].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f4x8_to_e4m3(w[k], l0[m][j], l1[m][j], o[2 * k], o[2 * k + 1]);
+      if (m == 0 || two) {
+        uint8_t* t = dst + m * 16384 + row * 16;
+        *reinterpret_cast<uint4*>(t + (2 * j) * 2048) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(t + (2 * j + 1) * 2048) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
 }
 
 // n, bf16 in the layout [H/8][8 rows][8], becomes the e4m3 B operand
@@ -168,10 +264,18 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
   }
 }
 
+// shared memory behind the ring: the MXFP4 kernel's two A buffers of 32 KB
+constexpr int kF4Ab = 2;
+constexpr uint32_t kF4AbBytes = 32768;
+__host__ __device__ inline size_t f4_abuf_off(const SmemLayout& L) { return align_up(L.total, 1024); }
+
+template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_constant__ Params p) {
-  constexpr uint32_t MAT = TqFmt<W_FP8>::MAT_BYTES;   // one unit of one matrix
+  constexpr bool F4 = WT == W_FP4;                    // codes expanded by warps 4-7 first
+  constexpr uint32_t MAT = TqFmt<WT>::MAT_BYTES;      // one unit of one matrix in the ring
   extern __shared__ __align__(1024) uint8_t smem[];
   const SmemLayout L(p.nst, p.slot_bytes, p.regA_bytes, p.ymax);
+  uint8_t* abuf = smem + f4_abuf_off(L);   // MXFP4: e4m3 A tiles, one ring stage each
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + p.nst;
   Ctl* c = reinterpret_cast<Ctl*>(smem + L.ctl);
@@ -192,11 +296,15 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);   // the MMAs' commit
+      mbar_init(&empty[s], F4 ? 4 : 1);   // the expanding warps, or the MMAs' commit
     }
     for (uint32_t b = 0; b < kF8Acc; ++b) {
       mbar_init(&c->accfull[b], 1);
       mbar_init(&c->accempty[b], 4);
+    }
+    for (int b = 0; b < kF4Ab; ++b) {
+      mbar_init(&c->abfull[b], 4);
+      mbar_init(&c->abempty[b], 1);
     }
     mbar_init(&c->drain, 1);
     mbar_init(&c->bfull, 1);
@@ -226,9 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
       const uint8_t* base = gu ? p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT
                                : p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * geo.upb_dn * MAT;
       const uint32_t ub = gu ? 2u * MAT : MAT;
-      const uint32_t sc_unit = gu ? 256u : 128u;   // block scales of one unit
-      const float* sc_base = gu ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * geo.upb_gu) * 256
-                                : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * geo.upb_dn) * 128;
+      // the epilogue's scales: FP8 block scales [unit][gate | up] or [unit]
+      // per block, MXFP4 row references [gate | up] or [rows] per block
+      const uint32_t sc_unit = gu ? 256u : 128u;
+      const float* sc_base = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : geo.upb_gu) * 256
+                                : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : geo.upb_dn) * 128;
+      if (F4) prefetch_l2(sc_base, sc_unit * 4);
       const int per = stage_units(sg);
       for (int u = sg.k0; u < sg.k1; u += per) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
@@ -238,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
           mbar_arrive_expect_tx(&full[slot], bytes);
           tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
           issued = s + 1;
-          prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
+          if (!F4) prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
         }
         ++s;
       }
@@ -314,11 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
       }
       const int per = stage_units(sg);
       for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
-        const uint32_t slot = s % p.nst, q = s / p.nst;
+        // the stage's A: the ring slot (FP8) or the A buffer its codes were
+        // expanded into (MXFP4)
+        const uint32_t slot = F4 ? s % kF4Ab : s % p.nst, q = F4 ? s / kF4Ab : s / p.nst;
         const int n = min(per, sg.k1 - u0);
-        if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
+        if (lane == 0 && ok) ok = wait_bar(p, c, F4 ? &c->abfull[slot] : &full[slot], q & 1);
         ok = warp_ok(ok);
         tc_fence_after();
+        const uint8_t* a_st = F4 ? abuf + (size_t)slot * kF4AbBytes : ring + (size_t)slot * p.slot_bytes;
         if (sg.list == L_RGU && first_rgu) {
           first_rgu = false;
           trace(p, 13, lane == 0);
@@ -332,13 +446,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
           }
           tc_fence_after();
           if (ok) {
-            const uint64_t da = umma_desc(smem_u32(ring + (size_t)slot * p.slot_bytes + (size_t)j * MAT), 2048u, 128u);
+            const uint64_t da = umma_desc(smem_u32(a_st + (size_t)j * 16384), 2048u, 128u);
             umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
           }
           umma_commit_warp(&c->accfull[buf]);
           ++t;
         }
-        umma_commit_warp(&empty[slot]);
+        umma_commit_warp(F4 ? &c->abempty[slot] : &empty[slot]);
         ++s;
       }
     };
@@ -417,10 +531,11 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
 #pragma unroll
       for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
       uint32_t v[16], w2[16];
-      // the units' block scales (brought to L2 by the producer), two units ahead
-      const float* sc = gu ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * upb) * 256
-                           : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * upb) * 128;
-      const int us = gu ? 256 : 128;
+      // the units' scales (brought to L2 by the producer), two units ahead:
+      // FP8 block scales, or the MXFP4 row reference (the same every unit)
+      const float* sc = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : upb) * 256
+                           : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : upb) * 128;
+      const int us = F4 ? 0 : gu ? 256 : 128;
       auto ld_g = [&](int u) { return u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
       auto ld_u = [&](int u) { return gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
       float sg0 = ld_g(sg.k0), su0 = ld_u(sg.k0), sg1 = ld_g(sg.k0 + 1), su1 = ld_u(sg.k0 + 1);
@@ -493,8 +608,39 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tf8_kernel(const __grid_
     }
     tc_fence_before();
     bar_arrive(kBarEnd, 5 * 32);   // the issuer may free the tensor memory
+  } else if (F4) {
+    // ======================================================= expanders
+    // warps 4-7, thread = weight row: each ring stage's codes into an A buffer
+    const int row = (warp - 4) * 32 + lane;
+    uint32_t s = 0;
+    bool cok = true;
+    auto expand = [&](const Seg& sg) {
+      const bool gu = sg.list != L_DN;
+      const int per = stage_units(sg);
+      for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+        const uint32_t slot = s % p.nst, q = s / p.nst;
+        const uint32_t ab = s % kF4Ab, qa = s / kF4Ab;
+        const int n = min(per, sg.k1 - u0);
+        if (lane == 0 && cok) cok = wait_bar(p, c, &full[slot], q & 1);
+        if (lane == 0 && cok && qa > 0) cok = wait_bar(p, c, &c->abempty[ab], (qa - 1) & 1);
+        cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
+        const uint8_t* src = ring + (size_t)slot * p.slot_bytes;
+        uint8_t* dst = abuf + (size_t)ab * kF4AbBytes;
+        if (cok) f4_expand_stage(src, dst, row, gu || n == 2);   // gate and up, or one or two down units
+        fence_proxy_async_smem();   // the MMAs read the tiles through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&c->abfull[ab]);
+          mbar_arrive(&empty[slot]);
+        }
+        ++s;
+      }
+    };
+    tc_segments(p, geo, L_SGU, 0, expand);
+    tc_segments(p, geo, L_RGU, nu, expand);
+    tc_segments(p, geo, L_DN, nu, expand);
   }
-  // warps 4-7 have no part in the main phase
+  // (FP8: warps 4-7 have no part in the main phase)
 
   // ==================================================================== tail
   bar_sync(kBarCons, kCW * 32);

@@ -39,6 +39,7 @@ class Workload:
     route_scale: float = 2.5
     denom_clamp: float = 1e-20
     sinkhorn_iters: int = 20
+    mx_spread: int = 0   # MXFP4: block magnitudes within a row span up to 2^mx_spread
 
     def with_(self, **kw):
         return replace(self, **kw)

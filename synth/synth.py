@@ -61,7 +61,7 @@ def cpu_lib():
         lib.synth_quant_fp8.argtypes = [vp, u64, u64, vp, vp]
         lib.synth_quant_mxfp4.argtypes = [vp, u64, u64, vp, vp]
         lib.synth_fill_fp8.argtypes = [u64, u32, u32, u32, f64, u64, u64, vp, vp]
-        lib.synth_fill_mxfp4.argtypes = [u64, u32, u32, u32, f64, u64, u64, vp, vp]
+        lib.synth_fill_mxfp4.argtypes = [u64, u32, u32, u32, f64, u64, u64, u32, vp, vp]
         lib.synth_ln_probe.argtypes = [f64]
         lib.synth_ln_probe.restype = f64
         _cpu = lib
@@ -78,7 +78,7 @@ def gpu_lib():
                                   ctypes.c_void_p)
         lib.synth_gpu_fill.argtypes = [u64, u32, u32, u32, i32, f64, f64, u64, u64, i32, vp, vp]
         lib.synth_gpu_fill_fp8.argtypes = [u64, u32, u32, u32, f64, u64, u64, vp, vp, vp]
-        lib.synth_gpu_fill_mxfp4.argtypes = [u64, u32, u32, u32, f64, u64, u64, vp, vp, vp]
+        lib.synth_gpu_fill_mxfp4.argtypes = [u64, u32, u32, u32, f64, u64, u64, u32, vp, vp, vp]
         for f in (lib.synth_gpu_fill, lib.synth_gpu_fill_fp8, lib.synth_gpu_fill_mxfp4):
             f.restype = i32
         _gpu = lib
@@ -148,7 +148,7 @@ def cpu_expert(w: Workload, layer: int, slot: int):
         else:
             q = np.empty((rows, cols // 2), np.uint8)
             e = np.empty((rows, cols // 32), np.uint8)
-            lib.synth_fill_mxfp4(w.seed, layer, kind, slot, std, rows, cols,
+            lib.synth_fill_mxfp4(w.seed, layer, kind, slot, std, rows, cols, w.mx_spread,
                                  q.ctypes.data_as(ctypes.c_void_p), e.ctypes.data_as(ctypes.c_void_p))
             res[name] = (q, e)
     return res
@@ -246,7 +246,7 @@ def gpu_experts(w: Workload, layer: int, device="cuda"):
             q = torch.empty((E1, rows, cols // 2), dtype=torch.uint8, device=device)
             s = torch.empty((E1, rows, cols // 32), dtype=torch.uint8, device=device)
             for e in range(E1):
-                _check(lib.synth_gpu_fill_mxfp4(w.seed, layer, kind, e, std, rows, cols,
+                _check(lib.synth_gpu_fill_mxfp4(w.seed, layer, kind, e, std, rows, cols, w.mx_spread,
                                                 ctypes.c_void_p(q[e].data_ptr()),
                                                 ctypes.c_void_p(s[e].data_ptr()), _stream()), "mxfp4")
             res[name] = (q, s)

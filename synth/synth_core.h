@@ -194,6 +194,17 @@ SYNTH_FN uint8_t synth_fp8_encode(float w, float s) {
   return (uint8_t)(sign | synth_e4m3_mag(v < 0.0f ? -v : v));
 }
 
+/* Spread of block magnitudes within a row, for the MXFP4 generator: block b
+ * of an expert's blocks is drawn at std * 2^-k with k = synth_mx_shift(b,
+ * spread) in [0, spread] (0 when spread is 0), so that a row's block scales
+ * span up to 2^spread.  Real checkpoints hold blocks far below their row's
+ * largest; the default workloads use spread 0. */
+SYNTH_FN uint32_t synth_mx_shift(uint64_t b, uint32_t spread) {
+  if (spread == 0u) return 0u;
+  uint64_t h = (b + 1u) * 0x9E3779B97F4A7C15ull;
+  return (uint32_t)((h >> 40) % (uint64_t)(spread + 1u));
+}
+
 /* MXFP4 32-block encoder (OCP MX v1.0 shared-exponent rule):
  * X = floor(log2 amax) - 2 (e2m1's largest exponent), stored as the e8m0 byte
  * X + 127 clamped to [0, 254]; amax == 0 stores byte 0. */

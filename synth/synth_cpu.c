@@ -100,7 +100,7 @@ EXPORT void synth_fill_fp8(uint64_t seed, uint32_t layer, uint32_t kind, uint32_
 }
 
 EXPORT void synth_fill_mxfp4(uint64_t seed, uint32_t layer, uint32_t kind, uint32_t expert, double std,
-                             uint64_t rows, uint64_t cols, uint8_t* q, uint8_t* e) {
+                             uint64_t rows, uint64_t cols, uint32_t spread, uint8_t* q, uint8_t* e) {
   uint64_t key = synth_key(seed, layer, kind, expert);
   uint64_t nb = cols / 32;
 #pragma omp parallel for schedule(static)
@@ -108,7 +108,7 @@ EXPORT void synth_fill_mxfp4(uint64_t seed, uint32_t layer, uint32_t kind, uint3
     float buf[32];
     float amax = 0.0f;
     for (int i = 0; i < 32; ++i) {
-      buf[i] = (float)(std * synth_normal(key, (uint64_t)rb * 32 + i));
+      buf[i] = (float)(ldexp(std, -(int)synth_mx_shift((uint64_t)rb, spread)) * synth_normal(key, (uint64_t)rb * 32 + i));
       float a = buf[i] < 0.0f ? -buf[i] : buf[i];
       if (a > amax) amax = a;
     }

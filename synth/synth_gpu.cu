@@ -52,12 +52,12 @@ __global__ void fill_fp8_kernel(uint64_t key, double std, uint64_t nblocks, uint
 }
 
 /* one warp per 32-block: 1 value per lane, nibbles paired through a shuffle */
-__global__ void fill_mxfp4_kernel(uint64_t key, double std, uint64_t nblocks, uint8_t* q, uint8_t* e) {
+__global__ void fill_mxfp4_kernel(uint64_t key, double std, uint64_t nblocks, uint32_t spread, uint8_t* q, uint8_t* e) {
   const int lane = threadIdx.x & 31;
   uint64_t warp = (blockIdx.x * (uint64_t)blockDim.x + threadIdx.x) >> 5;
   uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
   for (uint64_t b = warp; b < nblocks; b += nwarps) {
-    float v = __double2float_rn(std * synth_normal(key, b * 32 + lane));
+    float v = __double2float_rn(ldexp(std, -(int)synth_mx_shift(b, spread)) * synth_normal(key, b * 32 + lane));
     float amax = fabsf(v);
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     uint8_t sb = synth_mx_scale_byte(amax);
@@ -95,10 +95,10 @@ EXPORT int synth_gpu_fill_fp8(uint64_t seed, uint32_t layer, uint32_t kind, uint
 }
 
 EXPORT int synth_gpu_fill_mxfp4(uint64_t seed, uint32_t layer, uint32_t kind, uint32_t expert, double std,
-                                uint64_t rows, uint64_t cols, uint8_t* q, uint8_t* e, void* stream) {
+                                uint64_t rows, uint64_t cols, uint32_t spread, uint8_t* q, uint8_t* e, void* stream) {
   uint64_t nb = rows * (cols / 32);
   if (nb == 0) return 0;
   uint64_t key = synth_key(seed, layer, kind, expert);
-  fill_mxfp4_kernel<<<grid_for(nb * 32, 256), 256, 0, (cudaStream_t)stream>>>(key, std, nb, q, e);
+  fill_mxfp4_kernel<<<grid_for(nb * 32, 256), 256, 0, (cudaStream_t)stream>>>(key, std, nb, spread, q, e);
   return (int)cudaGetLastError();
 }

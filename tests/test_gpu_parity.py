@@ -166,6 +166,17 @@ def test_cuda_core_mxfp4_hidden_not_multiple_of_128():
     run.close()
 
 
+def test_scaled_mxfp4_wide_block_spread():
+    """MXFP4 rows whose block scales span up to 2^20: the tensor-core path's
+    e4m3 expansion relative to each row's largest scale takes its table, its
+    one-by-one (subnormal) and its rounded branches."""
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=431, mx_spread=20)
+    run = GpuRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
 def test_scaled_mxfp4_single_layer():
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=401)
     run = GpuRun(wl)

@@ -44,12 +44,32 @@ def test_recipe_scales():
     assert abs(nw.mean() - 1) < 0.02 and abs(nw.std() - 0.1) < 0.01
 
 
+def test_mxfp4_block_spread():
+    """mx_spread widens the block scales of a row; spread 0 is the default
+    generator, byte for byte."""
+    wl = C.scaled(C.FLASH_BF16_R1, hidden=512, n_routed=4, top_k=2, inter=256, w_dtype="mxfp4")
+    base = S.cpu_expert(wl, 0, 1)
+    same = S.cpu_expert(wl.with_(mx_spread=0), 0, 1)
+    wide = S.cpu_expert(wl.with_(mx_spread=20), 0, 1)
+    for nm in ("gate", "up", "down"):
+        assert np.array_equal(base[nm][0], same[nm][0]) and np.array_equal(base[nm][1], same[nm][1])
+        e0, e1 = base[nm][1].astype(int), wide[nm][1].astype(int)
+        span0 = (e0.max(axis=1) - e0.min(axis=1)).max()
+        span1 = (e1.max(axis=1) - e1.min(axis=1))
+        assert span0 <= 4
+        # most rows now span more than 2^14, and each block moved down by 0..20
+        assert (span1 > 14).mean() > 0.9 and span1.max() <= 20 + span0
+        assert ((e0 - e1) >= -1).all() and ((e0 - e1) <= 21).all()
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("wdt", ["bf16", "fp8", "mxfp4"])
+@pytest.mark.parametrize("wdt", ["bf16", "fp8", "mxfp4", "mxfp4-spread"])
 def test_device_build_writes_host_bytes(wdt):
     import torch
     S.build(gpu=True)
-    wl = C.scaled(C.FLASH_BF16_R1, hidden=512, n_routed=4, top_k=2, inter=256, w_dtype=wdt)
+    spread = 20 if wdt == "mxfp4-spread" else 0
+    wdt = wdt.split("-")[0]
+    wl = C.scaled(C.FLASH_BF16_R1, hidden=512, n_routed=4, top_k=2, inter=256, w_dtype=wdt, mx_spread=spread)
     dev = S.gpu_experts(wl, 1)
     torch.cuda.synchronize()
     for slot in (0, 4):
