@@ -29,8 +29,7 @@ FLUSH_BYTES = 512 << 20
 N_INPUT_SETS = 4
 KERNEL_SOURCES = ["moe_decode_layer_sm_b200/csrc/mono_ffn.cu", "moe_decode_layer_sm_b200/csrc/common.cuh",
                   "moe_decode_layer_sm_b200/csrc/cc_kernel.cuh", "moe_decode_layer_sm_b200/csrc/tc_kernel.cuh",
-                  "moe_decode_layer_sm_b200/csrc/ptx.cuh", "moe_decode_layer_sm_b200/csrc/tq_kernel.cuh",
-                  "moe_decode_layer_sm_b200/csrc/tf8_kernel.cuh"]
+                  "moe_decode_layer_sm_b200/csrc/ptx.cuh", "moe_decode_layer_sm_b200/csrc/tq_kernel.cuh"]
 
 
 def kernel_sha():

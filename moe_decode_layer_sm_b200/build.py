@@ -10,7 +10,6 @@ SRC = os.path.join(PKG, "csrc", "mono_ffn.cu")
 DEPS = [SRC, os.path.join(PKG, "csrc", "common.cuh"), os.path.join(PKG, "csrc", "cc_kernel.cuh"),
         os.path.join(PKG, "csrc", "tc_kernel.cuh"), os.path.join(PKG, "csrc", "ptx.cuh"),
         os.path.join(PKG, "csrc", "route_noalloc.cuh"), os.path.join(PKG, "csrc", "tq_kernel.cuh"),
-        os.path.join(PKG, "csrc", "tf8_kernel.cuh"),
         os.path.join(ROOT, "include", "mono_ffn.h")]
 SO = os.path.join(PKG, "libmonoffn.so")
 

@@ -41,7 +41,7 @@ constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // warps 0-3, routing hand-over (compute + control), end (epilogue warps + the
 // issuer warp)
 constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6;
-constexpr int kMaxAb = 3;          // A-tile buffers of the quantised tensor-core kernel
+constexpr int kMaxAb = 6;          // A-tile buffers of the quantised tensor-core kernels
 constexpr int kMaxAcc = 4;         // accumulator buffers in tensor memory
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
 
@@ -98,7 +98,6 @@ struct Params {
   uint32_t* xready;  // tensor-core kernel: [R*K+1] finished gate/up blocks per expert entry (0 between steps)
   const float* gsc;  // tensor-core FP8 kernel: [E+1][I/128][H/128][gate 128 | up 128] fp32 block scales
   const float* dsc;  // tensor-core FP8 kernel: [E+1][H/128][I/128][128] fp32 block scales
-  int q_f16;         // tensor-core kernels: B operands (n, activations) in fp16 instead of bf16
   int n_xready;
   uint8_t* actb;     // tensor-core kernel: [R*K+1][I/8][16][8] bf16 down-projection B operands
   float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks

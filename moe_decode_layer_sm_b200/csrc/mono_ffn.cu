@@ -13,7 +13,6 @@
 #include "cc_kernel.cuh"
 #include "tc_kernel.cuh"
 #include "tq_kernel.cuh"
-#include "tf8_kernel.cuh"
 
 using namespace mono;
 
@@ -109,8 +108,8 @@ void* kernel_ptr() {
 
 void* kernel_for(int wt, bool tc, bool tq) {
   if (tc) return reinterpret_cast<void*>(&mono_ffn_tc_kernel<W_BF16>);
-  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tf8_kernel<W_FP8>)
-                             : reinterpret_cast<void*>(&mono_ffn_tf8_kernel<W_FP4>);
+  if (tq) return wt == W_FP8 ? reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP8>)
+                             : reinterpret_cast<void*>(&mono_ffn_tq_kernel<W_FP4>);
   switch (wt) {
     case W_F32: return kernel_ptr<W_F32>();
     case W_BF16: return kernel_ptr<W_BF16>();
@@ -424,9 +423,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->regA_bytes = (int)align_up(regA, 128);
   const int smem_max = prop.sharedMemPerBlockOptin;
   SmemLayout L0(0, p->slot_bytes, p->regA_bytes, p->ymax);
-  // MXFP4 on the tensor cores: two A buffers behind the ring
-  const long long abuf_room = p->tq && dt == MONO_MXFP4 ? (long long)kF4Ab * kF4AbBytes + 1024 : 0;
-  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard - abuf_room;
+  long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard;
   p->nst = (int)std::min<long long>(16, room / p->slot_bytes);
   if (p->nst < 2) {
     std::string m = "shared memory: " + std::to_string(smem_max) + " bytes leave room for " + std::to_string(p->nst) +
@@ -435,10 +432,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     cudaSetDevice(prev);
     return fail(nullptr, MONO_ERR_INVALID_ARG, m);
   }
-  {
-    const SmemLayout L1(p->nst, p->slot_bytes, p->regA_bytes, p->ymax);
-    p->smem = (int)(abuf_room ? f4_abuf_off(L1) + (size_t)kF4Ab * kF4AbBytes : L1.total);
-  }
+  p->smem = (int)SmemLayout(p->nst, p->slot_bytes, p->regA_bytes, p->ymax).total;
   void* kfn = kernel_for(dt, p->tc, p->tq);
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
   int occ = 0;
@@ -731,7 +725,6 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.xready = p->xready;
     prm.gsc = ls.gsc;
     prm.dsc = ls.dsc;
-    prm.q_f16 = p->tq;
     prm.n_xready = p->xready ? rows * p->cfg.top_k + 1 : 0;
     prm.sync = p->sync + l;
     prm.err = p->err;

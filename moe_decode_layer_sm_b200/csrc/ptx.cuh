@@ -184,83 +184,6 @@ __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
       : "memory");
 }
 
-// fp16 A (from tensor memory) and fp16 B (shared-memory descriptor), fp32 D;
-// A's row i is TMEM lane i, 32-bit column c holds K elements 2c (low half)
-// and 2c + 1.  One elected lane of a converged warp issues.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int m, int n) {
-  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-__device__ __forceinline__ void umma_f16_tmem_a_warp(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
-                                                     uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p, e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(db), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// One 128 x 128 unit of the quantised kernels, issued by one elected lane
-// of a converged warp: 8 K-steps of 16, A from tensor memory (columns a, a +
-// 8, ..; pairs: up at a + 64 into d + 16), B from the descriptor db advanced
-// by db_step (16-byte units) per K-step.  acc0: accumulate from the first
-// K-step on (else the first one overwrites D).
-__device__ __forceinline__ void umma_unit_f16(uint32_t d, uint32_t a, uint64_t db, uint32_t db_step, uint32_t idesc,
-                                              uint32_t acc0, bool pair) {
-  if (pair) {
-    asm volatile(
-        "{\n .reg .pred e, p, t;\n .reg .b32 rx, a0, a1, d1;\n .reg .b64 b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %5, 0;\n setp.eq.b32 t, 0, 0;\n"
-        " mov.b32 a0, %1;\n add.u32 a1, %1, 64;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, p;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, p;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [d1], [a1], b, %4, t;\n"
-        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(acc0)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n .reg .pred e, p, t;\n .reg .b32 rx, a0;\n .reg .b64 b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %5, 0;\n setp.eq.b32 t, 0, 0;\n"
-        " mov.b32 a0, %1;\n mov.b64 b, %2;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, p;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], b, %4, t;\n"
-        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(acc0)
-        : "memory");
-  }
-}
-
 // Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0 in both
 // fields), fp32 accumulator, both K-major, M = m, N = n.
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3(int m, int n) {
@@ -308,35 +231,57 @@ __device__ __forceinline__ void umma_unit_e4m3(uint32_t d, uint64_t da, uint64_t
   }
 }
 
-// 32 lanes x 16 consecutive 32-bit columns from registers (thread l of the
-// warp writes its quadrant's lane l)
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
+// One 128 x 128 e4m3 unit with A in tensor memory (lane = row, 32-bit
+// column c = contraction elements 4c .. 4c + 3, lowest byte first), issued
+// by one elected lane: 4 K-steps of 32 (8 columns each), the first
+// overwriting D; B from the descriptor db advanced db_step units a K-step.
+// pair: a second A (up) 32 columns on, into d + 16.
+__device__ __forceinline__ void umma_unit_e4m3_tmem_a(uint32_t d, uint32_t a, uint64_t db, uint32_t db_step,
+                                                      uint32_t idesc, bool pair) {
+  if (pair) {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, a0, a1, d1;\n .reg .b64 b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " mov.b32 a0, %1;\n add.u32 a1, %1, 32;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, f;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, f;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
+        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, a0;\n .reg .b64 b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " mov.b32 a0, %1;\n mov.b64 b, %2;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, f;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
+        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
+        : "memory");
+  }
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// two e4m3 codes (low byte first) -> f16x2 bits (low half first); exact
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two_bytes) {
-  uint32_t h;
-  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(h) : "r"(two_bytes));
-  return h;
+// 32 lanes x 8 consecutive 32-bit columns from registers (thread l of the
+// warp writes its quadrant's lane l)
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
-// two e2m1 codes (low nibble first) -> f16x2 bits (low half first); exact
-__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
-  uint32_t h;
-  asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}\n" : "=r"(h) : "r"(byte));
-  return h;
-}
-__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // arrive once on bar when every tcgen05 operation this thread issued so far is complete
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {

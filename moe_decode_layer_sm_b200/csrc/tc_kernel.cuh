@@ -186,7 +186,7 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
 
 // A complete block.  Gate/up: SwiGLU, written as the down projection's B
 // operand of expert entry x, [I/8][16 rows][8] 16-bit, row 2r = hi, 2r + 1 =
-// lo of token row r (bf16, or fp16 when p.q_f16), zero for rows that do not
+// lo of token row r (bf16), zero for rows that do not
 // use the expert; then the block counts for its expert.  Down: the weighted
 // output of every row that uses the expert into yp.
 __device__ __forceinline__ void epi_store(const Params& p, Ctl* c, const TcGeo& geo, const Seg& sg, bool gu, bool live,
@@ -208,15 +208,9 @@ __device__ __forceinline__ void epi_store(const Params& p, Ctl* c, const TcGeo& 
           uu = round_bf16(uu);
         }
         const float act = gg / (1.0f + expf(-gg)) * uu;
-        if (p.q_f16) {
-          const __half hi = __float2half_rn(act);
-          hb = __half_as_ushort(hi);
-          lb = __half_as_ushort(__float2half_rn(act - __half2float(hi)));
-        } else {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(act);
-          hb = __bfloat16_as_ushort(hi);
-          lb = __bfloat16_as_ushort(__float2bfloat16_rn(act - __bfloat162float(hi)));
-        }
+        const __nv_bfloat16 hi = __float2bfloat16_rn(act);
+        hb = __bfloat16_as_ushort(hi);
+        lb = __bfloat16_as_ushort(__float2bfloat16_rn(act - __bfloat162float(hi)));
       }
       dst[(2 * r) * 8] = hb;
       dst[(2 * r + 1) * 8] = lb;

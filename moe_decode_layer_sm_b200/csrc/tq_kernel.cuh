@@ -1,105 +1,283 @@
-// Tensor-core variant of the persistent kernel for quantised experts: FP8
-// e4m3 with one fp32 scale per 1 x 128 block, and MXFP4 (e2m1 with one e8m0
-// scale per 32 elements).  Same work units, lists, split-block combine and
-// prologue as the bf16 tensor-core kernel; what differs is the A operand.
+// Quantised experts (FP8 e4m3 with 1 x 128 block scales, MXFP4) on the
+// tensor cores: tcgen05.mma of kind::f8f6f4.  FP8 needs no conversion pass:
+// the MMAs read the e4m3 weight codes straight from the ring (A, in shared
+// memory), and the activations as e4m3 as well (B).
 //
-// The weights stream through the ring as codes.  Warps 4-7 (idle in the
-// bf16 kernel's main phase) convert them, one thread per weight row, to fp16
-// and write them into tensor memory with tcgen05.st; the MMA reads A from
-// tensor memory (M = 128 rows, K = 16, fp16) and B (n, or the activations)
-// from shared memory, in fp16.  The conversions are exact: every e4m3 value
-// is an fp16 value, and an e2m1 value times its power-of-two MXFP4 scale is
-// one as long as the scale lies in [2^-22, 2^12] (the plan checks the packed
-// scales).  Only the FP8 block scale is not a power of two: it multiplies
-// the fp32 partial product of its 128-element unit in the epilogue, so each
-// FP8 unit gets its own accumulator.
+// An activation vector y goes into B as two e4m3 terms after a power-of-two
+// scale 2^e that puts its largest magnitude in [128, 256): hi = e4m3(y 2^e)
+// and lo = e4m3(y 2^e - hi).  B rows 0-7 carry hi of the 8 token rows, rows
+// 8-15 lo; the epilogue adds the two halves of the accumulator and multiplies
+// by 2^-e (exact).  A bf16 value has 8 significant bits and hi and lo hold 4
+// each, so n (bf16) is represented exactly down to 2^-9 of its row's largest
+// magnitude; smaller values, and the SwiGLU activations (fp32), keep an
+// absolute error below 2^-10 of the scaled unit, about 2^-17 of the block's
+// largest magnitude.
+//   gate/up B: n, one scale per token row
+//   down B:    the activations, one scale per (token row, 128-block of I),
+//              chosen by the epilogue that completes the gate/up block and
+//              stored behind the expert's codes
+// The FP8 block scales (fp32, one per 1 x 128 block of a weight row) scale
+// each unit's fp32 tile in the epilogue, so every unit gets its own
+// accumulator (four in flight).
 //
-// Packed units (one unit = 128 weight rows x 128 contraction elements of one
-// matrix), 16-byte chunk j of row i at [j][i] so that the 32 converter lanes
-// of a warp read consecutive 16-byte words:
-//   FP8    codes [8 chunks][128 rows][16]                      16384 B
-//   MXFP4  codes [4 chunks][128 rows][16], scales [128 rows][4]  8704 B
-// gate/up units hold gate then up; FP8 scales sit in their own arrays
-// (read by the epilogue), MXFP4 scales travel with the codes.
+// Packed FP8 units: [8 chunks][128 rows][16]
+// e4m3, chunk j of row i at [j][i]: K-major core matrices of 8 rows x 16
+// bytes, 2048 bytes between K-neighbours and 128 between row groups.  A ring
+// stage is one gate/up unit (gate, then up) or two down units, 32 KB.
+//
+// MXFP4 takes the same MMAs after one step: warps 4-7 (one thread per weight
+// row, its tensor-memory lane) expand each ring stage's e2m1 codes to e4m3
+// in tensor memory (six A buffers of one stage, 64 columns each), and the
+// MMAs read A from there.  A code times its block scale 2^s is written as
+// the e4m3 value code * 2^(s - s_ref), where s_ref, fixed per weight row at
+// packing, is the row's largest block exponent minus 6: every e2m1 value
+// times 2^d is an e4m3 value for d in [-8, 6] (6 * 2^6 = 384 <= 448; the
+// subnormal step 2^-9 divides 0.5 * 2^-8), so the expansion is exact unless
+// a block's scale lies more than 2^14 below its row's largest, where the
+// values are rounded to e4m3 (an error below 2^-16 of the row's largest
+// scale).  2^s_ref plays the part of the FP8 block scale in the epilogue.
+// Packed MXFP4 units: codes [4 chunks][128 rows][16] (32 e2m1 per chunk, 8
+// a word with the sign bits moved: f4_pack_word), then d = s - s_ref as int8
+// [128 rows][4], 8704 bytes a matrix; the per-row 2^s_ref sit in their own
+// arrays.
 #pragma once
+#include <cuda_fp8.h>
+
 #include "tc_kernel.cuh"
 
 namespace mono {
 
-constexpr int kTqTmemCols = 512;   // 2 accumulators of 32 columns, then 3 A buffers of 128
-constexpr uint32_t kAbCol = 64;    // first A buffer; buffer b at kAbCol + 128 b (gate 64 | up 64)
-constexpr int kAb = kMaxAb;        // A buffers: the converters run up to 3 units ahead of the MMAs
-// accumulator buffer b: columns 32 b for b < 2, behind the A buffers for b >= 2
-__device__ __forceinline__ uint32_t acc_col(uint32_t b) { return b < 2 ? 32u * b : 448u + 32u * (b - 2); }
-static_assert(kTqTmemCols >= (int)kAbCol + 128 * kAb, "A buffers fit in the tensor memory");
-
+// one 128 x 128 unit of one matrix in the ring: codes (and MXFP4 d bytes)
 template <int WT> struct TqFmt;
 template <> struct TqFmt<W_FP8> {
-  static constexpr int CHUNKS = 8, CODE_BYTES = 16384, MAT_BYTES = 16384;
+  static constexpr int MAT_BYTES = 16384;
 };
 template <> struct TqFmt<W_FP4> {
-  static constexpr int CHUNKS = 4, CODE_BYTES = 8192, MAT_BYTES = 8192 + 512;
+  static constexpr int MAT_BYTES = 8192 + 512;
 };
 
-// fp16 bits of 2^(e - 127) for an e8m0 code e with e - 127 in [-22, 12]
-__device__ __forceinline__ uint32_t e8m0_to_h(uint32_t e) {
-  const int k = (int)e - 127;
-  return k >= -14 ? (uint32_t)(k + 15) << 10 : 1u << (k + 24);
+constexpr int kF8TmemCols = 128;   // four accumulators of 32 columns (gate 16 | up 16)
+constexpr int kF4TmemCols = 512;   // the accumulators, then the MXFP4 A buffers
+constexpr int kF4Ab = 6;           // MXFP4 A buffers of one ring stage (64 columns) in tensor memory
+static_assert(kF4Ab <= kMaxAb && kF8TmemCols + 64 * kF4Ab <= kF4TmemCols, "A buffers fit");
+constexpr uint32_t kF8Acc = 4;
+static_assert(kF8Acc <= (uint32_t)kMaxAcc, "accumulator barriers");
+
+// bytes of one expert entry's down B operand: [I/16][16 rows][16] e4m3 codes,
+// then [I/128][8] fp32 inverse scales
+__host__ __device__ inline size_t f8_act_stride(int I) { return (size_t)I * 16 + (size_t)(I / 128) * 32; }
+
+// e with m 2^e in [128, 256) for m > 0 (0 for m = 0), within [-126, 126] so
+// that 2^e and 2^-e are normal floats
+__device__ __forceinline__ int f8_exp(float m) {
+  if (!(m > 0.f)) return 0;
+  const int ex = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;   // floor(log2 m) for normal m
+  return max(-126, min(126, 7 - ex));
+}
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// two scaled values -> e4m3 hi and lo code pairs (the first value in the low byte)
+__device__ __forceinline__ void f8_split2(float y0, float y1, uint32_t& hi, uint32_t& lo) {
+  const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
+  const float2 hf = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3)));
+  const __nv_fp8x2_storage_t l =
+      __nv_cvt_float2_to_fp8x2(make_float2(y0 - hf.x, y1 - hf.y), __NV_SATFINITE, __NV_E4M3);
+  hi = h;
+  lo = l;
 }
 
-// Chunks [j0, j1) of one matrix of one unit from the ring slot to this
-// thread's lane (row) of tensor memory, from column taddr on (64 columns
-// for the whole matrix).
-template <int WT>
-__device__ __forceinline__ void tq_convert(const uint8_t* mat, int row, uint32_t taddr, int j0, int j1) {
-  using F = TqFmt<WT>;
-  if (WT == W_FP8) {
+// e4m3 of the 8 e2m1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} times 2^d, as
+// bytes 0-3 / 4-7 of a byte-permute table.  For d in [-5, 6] every nonzero
+// entry is a normal e4m3 value and d is added to the exponent field of the
+// d = 0 table (f4_lut_fast); below -5 the values are converted one by one
+// (subnormal, or rounded below -8), out of line since it is rare.
+__device__ __forceinline__ void f4_lut_fast(int d, uint32_t& l0, uint32_t& l1) {
+  const uint32_t de = (uint32_t)(d * 8);
+  l0 = 0x3C383000u + de * 0x01010100u;
+  l1 = 0x4C484440u + de * 0x01010101u;
+}
+__device__ __noinline__ uint2 f4_lut_slow(int d) {
+  const float s = ldexpf(1.0f, max(d, -126));
+  const uint32_t a = __nv_cvt_float2_to_fp8x2(make_float2(0.f, 0.5f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t b = __nv_cvt_float2_to_fp8x2(make_float2(1.0f * s, 1.5f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(2.0f * s, 3.0f * s), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t e = __nv_cvt_float2_to_fp8x2(make_float2(4.0f * s, 6.0f * s), __NV_SATFINITE, __NV_E4M3);
+  return make_uint2(a | (b << 16), c | (e << 16));
+}
+
+// Eight e2m1 codes in the packed word layout of this kernel -> eight e4m3
+// bytes.  The magnitude of code k sits in bits 4k .. 4k + 2 (as in the MXFP4
+// byte stream, two codes a byte, low nibble first); the sign bits are moved at
+// packing (f4_pack_word) to bits 3, 11, 19, 27 for codes 0-3 and 7, 15, 23,
+// 31 for codes 4-7, so that one shift or none puts each on bit 7 of its
+// output byte.  The magnitudes go through the table: one byte permute per
+// four codes.
+__host__ __device__ inline uint32_t f4_pack_word(uint32_t w) {
+  uint32_t o = w & 0x77777777u;
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t sgn = (w >> (4 * k + 3)) & 1u;
+    const int at = k < 4 ? 8 * k + 3 : 8 * (k - 4) + 7;
+    o |= sgn << at;
+  }
+  return o;
+}
+__device__ __forceinline__ void f4x8_to_e4m3(uint32_t w, uint32_t l0, uint32_t l1, uint32_t& o0, uint32_t& o1) {
+  o0 = __byte_perm(l0, l1, w & 0x7777u) | ((w & 0x08080808u) << 4);
+  o1 = __byte_perm(l0, l1, (w >> 16) & 0x7777u) | (w & 0x80808080u);
+}
+
+// One ring stage of MXFP4 (two unit-matrices: gate and up, or two down
+// units; the second is stored only when two), this thread's weight row:
+// codes [4][128 rows][16] and the rows' d [128][4] of each matrix -> e4m3 in
+// the 32 tensor-memory columns from taddr and taddr + 32 (column c = four
+// contraction elements).  Whole warps (tcgen05.st); not inlined.
+__device__ __noinline__ void f4_expand_stage(const uint8_t* src, uint32_t taddr, int row, bool two) {
+  constexpr int MAT = 8192 + 512;
+  uint32_t l0[2][4], l1[2][4];
+  uint4 q[2][4];
 #pragma unroll
-    for (int j = 0; j < F::CHUNKS; j += 2) {
-      if (j < j0 || j >= j1) continue;
-      uint32_t v[16];
+  for (int m = 0; m < 2; ++m) {
+    const uint32_t dd = *reinterpret_cast<const uint32_t*>(src + m * MAT + 8192 + row * 4);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4 q = *reinterpret_cast<const uint4*>(mat + (size_t)(j + h) * 2048 + row * 16);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          v[8 * h + 2 * m] = e4m3x2_to_h2(w[m] & 0xFFFFu);
-          v[8 * h + 2 * m + 1] = e4m3x2_to_h2(w[m] >> 16);
-        }
+    for (int j = 0; j < 4; ++j) {
+      q[m][j] = *reinterpret_cast<const uint4*>(src + m * MAT + j * 2048 + row * 16);
+      const int d = (int)(int8_t)((dd >> (8 * j)) & 0xFFu);
+      f4_lut_fast(d, l0[m][j], l1[m][j]);
+      if (d < -5) {
+        const uint2 t = f4_lut_slow(d);
+        l0[m][j] = t.x;
+        l1[m][j] = t.y;
       }
-      tmem_st16(taddr + 8u * j, v);
     }
-  } else {
-    const uint32_t sc = *reinterpret_cast<const uint32_t*>(mat + F::CODE_BYTES + row * 4);
+  }
 #pragma unroll
-    for (int j = 0; j < F::CHUNKS; ++j) {
-      if (j < j0 || j >= j1) continue;
-      const uint32_t s1 = e8m0_to_h((sc >> (8 * j)) & 0xFFu);
-      const uint32_t s2 = s1 | (s1 << 16);
-      const uint4 q = *reinterpret_cast<const uint4*>(mat + (size_t)j * 2048 + row * 16);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-      uint32_t v[16];
+  for (int m = 0; m < 2; ++m) {
 #pragma unroll
-      for (int m = 0; m < 16; ++m) v[m] = hmul2_bits(e2m1x2_to_h2((w[m >> 2] >> (8 * (m & 3))) & 0xFFu), s2);
-      tmem_st16(taddr + 16u * j, v);
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t w[4] = {q[m][j].x, q[m][j].y, q[m][j].z, q[m][j].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f4x8_to_e4m3(w[k], l0[m][j], l1[m][j], o[2 * k], o[2 * k + 1]);
+      if (m == 0 || two) tmem_st8(taddr + 32u * m + 8u * j, o);
     }
+  }
+}
+
+// n, bf16 in the layout [H/8][8 rows][8], becomes the e4m3 B operand
+// [H/16][16 rows][16] (rows 0-7 hi, 8-15 lo) in place, one 128-column block
+// per warp at a time (the two layouts put a block in the same 2 KB); c->nsc
+// gets each row's inverse scale.  Compute warps.
+__device__ void f8_convert_n(const Params& p, Ctl* c, uint8_t* regA) {
+  const int H = p.H, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // row maxima: 16-byte item q of the bf16 layout holds row q & 7, and this
+  // thread's items all have row tid & 7
+  float m = 0.f;
+  for (int q = tid; q < H; q += kCW * 32) {
+    const uint4 v = *reinterpret_cast<const uint4*>(regA + (size_t)q * 16);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x))), fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y)))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))), fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w)))));
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+  if (lane < 8) c->sq[warp][lane] = m;
+  bar_sync(kBarCons, kCW * 32);
+  const int r = lane & 7, q = lane >> 3;
+  float mr = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCW; ++w) mr = fmaxf(mr, c->sq[w][r]);
+  const int e = f8_exp(mr);
+  if (tid < 8) c->nsc[tid] = pow2i(-e);
+  const float sc = pow2i(e);
+  // lane (r, q): columns 32 q .. 32 q + 31 of row r of the block, i.e. bf16
+  // chunks 4q .. 4q + 3 in, e4m3 chunks 2q and 2q + 1 out
+  for (int kb = warp; kb < H / 128; kb += kCW) {
+    uint8_t* blk = regA + (size_t)kb * 2048;
+    uint4 v[4];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) v[cc] = *reinterpret_cast<const uint4*>(blk + (4 * q + cc) * 128 + r * 16);
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int m2 = 0; m2 < 4; ++m2) {
+        const uint4 s = v[2 * h + (m2 >> 1)];
+        const uint32_t w0 = (m2 & 1) ? s.z : s.x, w1 = (m2 & 1) ? s.w : s.y;
+        uint32_t h01, l01, h23, l23;
+        f8_split2(bf16lo(w0) * sc, bf16hi(w0) * sc, h01, l01);
+        f8_split2(bf16lo(w1) * sc, bf16hi(w1) * sc, h23, l23);
+        hi[m2] = h01 | (h23 << 16);
+        lo[m2] = l01 | (l23 << 16);
+      }
+      *reinterpret_cast<uint4*>(blk + (2 * q + h) * 256 + r * 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(blk + (2 * q + h) * 256 + (8 + r) * 16) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+}
+
+// A complete gate/up block: SwiGLU, then each token row's 128 activations of
+// the block as e4m3 hi/lo under the block's power-of-two scale, into the
+// down B operand of expert entry x, with the inverse scale behind the codes;
+// zero for rows that do not use the expert.  Then the block counts for its
+// expert.  Every epilogue thread, live or not.
+__device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg& sg, bool live, int i,
+                                             const float (&a)[8], const float (&b)[8]) {
+  const int R = p.R, K = p.K, I = p.I, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int x = sg.x;
+  float act[8];
+#pragma unroll
+  for (int r = 0; r < kMaxR; ++r) {
+    const int sl = x == 0 ? K : c->uslot[x - 1][r];
+    act[r] = 0.f;
+    if (live && r < R && sl >= 0) {
+      float gg = a[r], uu = b[r];
+      if (p.round_bf16) {
+        gg = round_bf16(gg);
+        uu = round_bf16(uu);
+      }
+      act[r] = gg / (1.0f + expf(-gg)) * uu;
+    }
+    const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(act[r])));
+    if (lane == 0) c->amax[warp][r] = __uint_as_float(mb);
+  }
+  bar_sync(kBarEpi, 4 * 32);
+  uint8_t* base = p.actb + (size_t)x * f8_act_stride(I);
+  const int ch = sg.blk * 128 + i;
+  uint8_t* dst = base + (size_t)(ch >> 4) * 256 + (ch & 15);
+#pragma unroll
+  for (int r = 0; r < kMaxR; r += 2) {
+    int e[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int rr = r + k;
+      e[k] = f8_exp(fmaxf(fmaxf(c->amax[0][rr], c->amax[1][rr]), fmaxf(c->amax[2][rr], c->amax[3][rr])));
+    }
+    uint32_t hb, lb;
+    f8_split2(act[r] * pow2i(e[0]), act[r + 1] * pow2i(e[1]), hb, lb);
+    if (live) {
+      dst[r * 16] = (uint8_t)(hb & 0xFFu);
+      dst[(r + 1) * 16] = (uint8_t)(hb >> 8);
+      dst[(8 + r) * 16] = (uint8_t)(lb & 0xFFu);
+      dst[(9 + r) * 16] = (uint8_t)(lb >> 8);
+      float* inv = reinterpret_cast<float*>(base + (size_t)I * 16) + sg.blk * 8;
+      if (i == r) inv[r] = pow2i(-e[0]);
+      if (i == r + 1) inv[r + 1] = pow2i(-e[1]);
+    }
+  }
+  // the block's activations are out: count it for its expert (the codes are
+  // read by a bulk copy, the async proxy; the scales by the epilogues)
+  __threadfence();
+  bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
+  if (tid == 0 && live) {
+    fence_proxy_async_global();
+    red_release_add(&p.xready[x], 1u);
   }
 }
 
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_constant__ Params p) {
-  using F = TqFmt<WT>;
-  constexpr uint32_t MAT = F::MAT_BYTES;
-  constexpr bool PER_UNIT = WT == W_FP8;   // a non-power-of-two block scale per unit
-  // MXFP4 (two codes a byte, a scale multiply each) needs the conversion
-  // throughput of all eight compute warps; its epilogue runs once a segment
-  // on warps 0-3 between their conversions.  FP8 converts on warps 4-7.
-  constexpr int NCV = WT == W_FP4 ? 8 : 4;
-  // FP8 hands every unit to the epilogue: four accumulators keep the MMAs
-  // three units ahead of it; MXFP4 hands over once per segment
-  constexpr uint32_t NACC = PER_UNIT ? 4 : 2;
-  static_assert(NACC <= kMaxAcc && 448 + 32 * 2 <= kTqTmemCols, "accumulators fit");
+  constexpr bool F4 = WT == W_FP4;                    // codes expanded by warps 4-7 first
+  constexpr uint32_t MAT = TqFmt<WT>::MAT_BYTES;      // one unit of one matrix in the ring
   extern __shared__ __align__(1024) uint8_t smem[];
   const SmemLayout L(p.nst, p.slot_bytes, p.regA_bytes, p.ymax);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -110,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int R = p.R, H = p.H, I = p.I, K = p.K, G = p.G;
+  const int H = p.H, I = p.I, K = p.K, G = p.G;
   const TcGeo geo(p);
 
   if (tid == 0) {
@@ -122,14 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NCV);   // the converter warps
+      mbar_init(&empty[s], F4 ? 4 : 1);   // the expanding warps, or the MMAs' commit
     }
-    for (uint32_t b = 0; b < NACC; ++b) {
+    for (uint32_t b = 0; b < kF8Acc; ++b) {
       mbar_init(&c->accfull[b], 1);
       mbar_init(&c->accempty[b], 4);
     }
-    for (int b = 0; b < kAb; ++b) {
-      mbar_init(&c->abfull[b], NCV);
+    for (int b = 0; b < kF4Ab; ++b) {
+      mbar_init(&c->abfull[b], 4);
       mbar_init(&c->abempty[b], 1);
     }
     mbar_init(&c->drain, 1);
@@ -138,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   }
   __syncthreads();
   if (c->dead) return;
-  if (warp == kMmaWarp) tmem_alloc(&c->tmem_base, kTqTmemCols);
+  constexpr int kCols = F4 ? kF4TmemCols : kF8TmemCols;
+  if (warp == kMmaWarp) tmem_alloc(&c->tmem_base, kCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -146,16 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   const uint32_t tmem = c->tmem_base;
   trace(p, 0, tid == 0);
 
-  // unit bytes in the ring and the first byte of a segment's block; a ring
-  // stage holds one gate/up unit or two down units (one copy of 2 MAT bytes:
-  // a single down unit of MXFP4 would be a copy too small to stream well)
-  auto unit_bytes = [&](const Seg& sg) { return sg.list != L_DN ? 2u * MAT : MAT; };
+  // a ring stage: one gate/up unit (gate, up) or two down units
   auto stage_units = [&](const Seg& sg) { return sg.list != L_DN ? 1 : 2; };
-  auto block_base = [&](const Seg& sg) -> const uint8_t* {
-    const int e = seg_expert(p, c, sg.x);
-    if (sg.list != L_DN) return p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT;
-    return p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * geo.upb_dn * MAT;
-  };
 
   // ================================================================ producer
   if (warp == kProdWarp) {
@@ -163,15 +334,17 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     bool ok = true;
     auto seg = [&](const Seg& sg) {
       if (lane != 0) return;
-      const uint8_t* base = block_base(sg);
-      const uint32_t ub = unit_bytes(sg);
-      const uint32_t sc_unit = sg.list != L_DN ? 256u : 128u;   // FP8 scales of one unit
-      const float* sc_base = nullptr;
-      if (PER_UNIT) {
-        const int e = seg_expert(p, c, sg.x);
-        sc_base = sg.list != L_DN ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * geo.upb_gu) * 256
-                                  : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * geo.upb_dn) * 128;
-      }
+      const int e = seg_expert(p, c, sg.x);
+      const bool gu = sg.list != L_DN;
+      const uint8_t* base = gu ? p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT
+                               : p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * geo.upb_dn * MAT;
+      const uint32_t ub = gu ? 2u * MAT : MAT;
+      // the epilogue's scales: FP8 block scales [unit][gate | up] or [unit]
+      // per block, MXFP4 row references [gate | up] or [rows] per block
+      const uint32_t sc_unit = gu ? 256u : 128u;
+      const float* sc_base = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : geo.upb_gu) * 256
+                                : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : geo.upb_dn) * 128;
+      if (F4) prefetch_l2(sc_base, sc_unit * 4);
       const int per = stage_units(sg);
       for (int u = sg.k0; u < sg.k1; u += per) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
@@ -181,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           mbar_arrive_expect_tx(&full[slot], bytes);
           tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
           issued = s + 1;
-          if (PER_UNIT) prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
+          if (!F4) prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
         }
         ++s;
       }
@@ -215,26 +388,18 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
 
   // =========================================================== MMA issuer
   if (warp == kMmaWarp) {
-    uint32_t t = 0, ua = 0, ndrain = 0, nb = 0;
+    uint32_t s = 0, t = 0, ndrain = 0, nb = 0;
     int prev_x = -1;
-    bool b_pending = false;
+    bool first_rgu = true, b_pending = false;
     auto warp_ok = [&](bool v) { return __shfl_sync(0xffffffffu, (int)v, 0) != 0; };
     bool ok = true;
     if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
     ok = warp_ok(ok);
-    const uint32_t b_addr = smem_u32(regA);
-    const uint32_t idesc = umma_idesc_f16(128, 16);
-    const uint32_t b_bytes = (uint32_t)I * 32u;
-    const uint64_t bdesc_gu = umma_desc(b_addr, 128u, 0u), bdesc_dn = umma_desc(b_addr, 256u, 128u);
-    auto acc_claim = [&]() {   // the accumulator buffer for the next tile
-      const uint32_t buf = t % NACC;
-      if (t >= NACC) {
-        if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / NACC) - 1) & 1u);
-        ok = warp_ok(ok);
-      }
-      tc_fence_after();
-      return tmem + acc_col(buf);
-    };
+    const uint32_t idesc = umma_idesc_e4m3(128, 16);
+    const uint32_t b_bytes = (uint32_t)I * 16u;
+    // B (n, or a down expert's activations): [K/16][16 rows][16], 256 bytes
+    // between K-neighbours, rows 8-15 128 bytes on; a unit is 2048 bytes
+    const uint64_t bdesc = umma_desc(smem_u32(regA), 256u, 128u);
     auto seg = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
       if (!gu && sg.x != prev_x) {
@@ -253,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         if (ok) {   // (a copy whose wait failed is waited for again at exit)
           if (lane == 0) {
             mbar_arrive_expect_tx(&c->bfull, b_bytes);
-            tma_load_1d(regA, p.actb + (size_t)sg.x * b_bytes, b_bytes, &c->bfull);
+            tma_load_1d(regA, p.actb + (size_t)sg.x * f8_act_stride(I), b_bytes, &c->bfull);
             ok = wait_bar(p, c, &c->bfull, nb & 1u);
           }
           ok = warp_ok(ok);
@@ -263,32 +428,42 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         tc_fence_after();
         trace(p, 15, nb == 1 && lane == 0);
       }
-      uint32_t d0 = PER_UNIT ? 0u : acc_claim();
-      for (int u = sg.k0; u < sg.k1; ++u) {
-        if (PER_UNIT) d0 = acc_claim();
-        const uint32_t ab = ua % kAb;
-        if (lane == 0 && ok) ok = wait_bar(p, c, &c->abfull[ab], (ua / kAb) & 1u);
+      const int per = stage_units(sg);
+      for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+        // the stage's A: the ring slot (FP8) or the A buffer its codes were
+        // expanded into (MXFP4)
+        const uint32_t slot = F4 ? s % kF4Ab : s % p.nst, q = F4 ? s / kF4Ab : s / p.nst;
+        const int n = min(per, sg.k1 - u0);
+        if (lane == 0 && ok) ok = wait_bar(p, c, F4 ? &c->abfull[slot] : &full[slot], q & 1);
         ok = warp_ok(ok);
         tc_fence_after();
-        if (ok) {
-          // the unit's 8 K-steps (gate and up as a pair) from one elected lane
-          const uint32_t a0 = tmem + kAbCol + 128u * ab;
-          const int kg0 = u * kKS;   // contraction group of the B operand
-          // a fresh accumulator per FP8 unit; MXFP4 adds the segment's units up
-          const uint32_t acc0 = (!PER_UNIT && u > sg.k0) ? 1u : 0u;
-          if (gu) umma_unit_f16(d0, a0, bdesc_gu + (uint64_t)(kg0 * 8), 16u, idesc, acc0, true);   // 2 groups of 128 B a step
-          else umma_unit_f16(d0, a0, bdesc_dn + (uint64_t)(kg0 * 16), 32u, idesc, acc0, false);   // 2 groups of 256 B
+        const uint8_t* a_st = ring + (size_t)slot * p.slot_bytes;   // FP8
+        const uint32_t a_tm = tmem + (uint32_t)kF8TmemCols + 64u * slot;   // MXFP4
+        if (sg.list == L_RGU && first_rgu) {
+          first_rgu = false;
+          trace(p, 13, lane == 0);
         }
-        umma_commit_warp(&c->abempty[ab]);
-        ++ua;
-        if (PER_UNIT) {
-          umma_commit_warp(&c->accfull[t % NACC]);
+        for (int j = 0; j < n; ++j) {
+          const int u = u0 + j;
+          const uint32_t buf = t % kF8Acc;
+          if (t >= kF8Acc) {
+            if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / kF8Acc) - 1) & 1u);
+            ok = warp_ok(ok);
+          }
+          tc_fence_after();
+          if (ok) {
+            if (F4) {
+              umma_unit_e4m3_tmem_a(tmem + 32u * buf, a_tm + 32u * j, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
+            } else {
+              const uint64_t da = umma_desc(smem_u32(a_st + (size_t)j * MAT), 2048u, 128u);
+              umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
+            }
+          }
+          umma_commit_warp(&c->accfull[buf]);
           ++t;
         }
-      }
-      if (!PER_UNIT) {
-        umma_commit_warp(&c->accfull[t % NACC]);
-        ++t;
+        umma_commit_warp(F4 ? &c->abempty[slot] : &empty[slot]);
+        ++s;
       }
     };
     tc_segments(p, geo, L_SGU, 0, seg);
@@ -299,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     trace(p, 14, lane == 0);
     tc_segments(p, geo, L_DN, nu, seg);
     trace(p, 16, lane == 0);
+    // every MMA of this CTA is complete before the tensor memory goes away,
+    // and no bulk copy still targets shared memory at exit
     umma_commit_warp(&c->drain);
     if (lane == 0) {
       const uint64_t t0 = globaltimer();
@@ -307,9 +484,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         __nanosleep(64);
     }
     __syncwarp();
-    bar_sync(kBarEnd, 9 * 32);
+    bar_sync(kBarEnd, 5 * 32);
     tc_fence_after();
-    tmem_dealloc(tmem, kTqTmemCols);
+    tmem_dealloc(tmem, kCols);
     return;
   }
 
@@ -321,22 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   }
   collapse_norm<true>(p, c, regA, ep1);
   // the router reads n as bf16 (the layer's values); the MMAs then take it
-  // as fp16 (exact for normal values; below 2^-14 fp16 keeps 2^-24 steps)
+  // as e4m3 hi/lo
   router_logits<true>(p, c, regA, false);
-  {
-    const int H8 = H / 8;
-    for (int q = tid; q < R * H8; q += kCW * 32) {
-      uint4* w = reinterpret_cast<uint4*>(regA + n_off<true>(q / H8, (q % H8) * 8, H, true));
-      uint4 v = *w;
-      uint32_t* u = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __half2 h = __floats2half2_rn(bf16lo(u[k]), bf16hi(u[k]));
-        u[k] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      *w = v;
-    }
-  }
+  f8_convert_n(p, c, regA);
   fence_proxy_async_smem();   // n is read by the tensor cores (async proxy)
   bar_sync(kBarCons, kCW * 32);
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
@@ -351,153 +515,101 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   bar_sync(kBarCons, kCW * 32);
   const int nu = c->nu_comp;
 
-  // ==================================================== converters, epilogue
-  // Converter warp w: its lane quadrant (w & 3) of tensor memory, thread =
-  // weight row.  With eight converter warps (MXFP4) warps 4-7 take the gate
-  // matrix (or the first half of the chunks of a down unit) and warps 0-3
-  // the up matrix (or the second half); with four (FP8), warps 4-7 take all.
-  const bool converts = NCV == 8 || warp >= 4;
-  const int row = (warp & 3) * 32 + lane;
-  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-  uint32_t s = 0, ua = 0;
-  bool cok = true;
-  auto convert_units = [&](const Seg& sg) {
-    const bool gu = sg.list != L_DN;
-    const int per = stage_units(sg);
-    for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
-      const uint32_t slot = s % p.nst, q = s / p.nst;
-      const int n = min(per, sg.k1 - u0);
-      // lane 0 waits; the warp follows its answer (tcgen05.st is warp-wide)
-      if (lane == 0 && cok) cok = wait_bar(p, c, &full[slot], q & 1);
-      cok = __shfl_sync(0xffffffffu, (int)cok, 0) != 0;
-      for (int j = 0; j < n; ++j) {
-        const uint32_t ab = ua % kAb;
-        if (lane == 0 && ua >= kAb && cok) cok = wait_bar(p, c, &c->abempty[ab], ((ua / kAb) - 1) & 1u);
-        cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
-        tc_fence_after();
-        const uint8_t* st = ring + (size_t)slot * p.slot_bytes + (size_t)j * MAT;
-        const uint32_t col = lane_base + kAbCol + 128u * ab;
-        if (cok) {
-          if (NCV == 4) {
-            tq_convert<WT>(st, row, col, 0, F::CHUNKS);
-            if (gu) tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
-          } else if (gu) {
-            if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS);
-            else tq_convert<WT>(st + MAT, row, col + 64u, 0, F::CHUNKS);
-          } else {
-            if (warp >= 4) tq_convert<WT>(st, row, col, 0, F::CHUNKS / 2);
-            else tq_convert<WT>(st, row, col, F::CHUNKS / 2, F::CHUNKS);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c->abfull[ab]);
-        ++ua;
-      }
-      if (lane == 0) mbar_arrive(&empty[slot]);   // every unit of the stage is read
-      ++s;
-    }
-  };
-
   if (warp < 4) {
     // ============================================================ epilogue
     // thread <-> row i = 32 w + l of the 128-row tile (its TMEM lane)
     const int i = tid;
     uint32_t t = 0;
     bool ok = true;
-    auto take = [&](uint32_t* v, uint32_t* w2) {   // the next accumulator tile
-      const uint32_t buf = t % NACC;
-      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / NACC) & 1u);
+    auto take = [&](uint32_t* v, uint32_t* w2, bool gu) {   // the next unit's tile
+      const uint32_t buf = t % kF8Acc;
+      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / kF8Acc) & 1u);
       tc_fence_after();
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + acc_col(buf), v);
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + acc_col(buf) + 16u, w2);
+      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf;
+      tmem_ld16(ta, v);
+      if (gu) tmem_ld16(ta + 16u, w2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c->accempty[buf]);
       ++t;
     };
-    // the accumulator work of a segment (its conversion is done)
-    auto finish = [&](const Seg& sg) {
+    auto seg = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
       const int upb = gu ? geo.upb_gu : geo.upb_dn;
+      const int e = seg_expert(p, c, sg.x);
       float a[8], b[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
       uint32_t v[16], w2[16];
-      if (PER_UNIT) {
-        // FP8: scale each unit's fp32 tile by its row's block scale (the
-        // producer brought the scales to L2); two units' scales in flight
-        const int e = seg_expert(p, c, sg.x);
-        const float* sc = gu ? p.gsc + ((size_t)(e * geo.nbi + sg.blk) * upb) * 256
-                             : p.dsc + ((size_t)(e * geo.nbh + sg.blk) * upb) * 128;
-        const int us = gu ? 256 : 128;
-        auto ld_g = [&](int u) { return u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
-        auto ld_u = [&](int u) { return gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
-        float sg0 = ld_g(sg.k0), su0 = ld_u(sg.k0), sg1 = ld_g(sg.k0 + 1), su1 = ld_u(sg.k0 + 1);
+      // the units' scales (brought to L2 by the producer), two units ahead:
+      // FP8 block scales, or the MXFP4 row reference (the same every unit)
+      const float* sc = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : upb) * 256
+                           : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : upb) * 128;
+      const int us = F4 ? 0 : gu ? 256 : 128;
+      auto ld_g = [&](int u) { return u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
+      auto ld_u = [&](int u) { return gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
+      float sg0 = ld_g(sg.k0), su0 = ld_u(sg.k0), sg1 = ld_g(sg.k0 + 1), su1 = ld_u(sg.k0 + 1);
+      if (gu) {
         for (int u = sg.k0; u < sg.k1; ++u) {
           const float sg2 = ld_g(u + 2), su2 = ld_u(u + 2);
-          take(v, w2);
+          take(v, w2, true);
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
-            if (gu) {
-              a[r] = fmaf(sg0, __uint_as_float(v[r]), a[r]);
-              b[r] = fmaf(su0, __uint_as_float(w2[r]), b[r]);
-            } else {
-              a[r] = fmaf(sg0, __uint_as_float(v[2 * r]) + __uint_as_float(v[2 * r + 1]), a[r]);
-            }
+            a[r] = fmaf(sg0, __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
+            b[r] = fmaf(su0, __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]), b[r]);
           }
           sg0 = sg1;
           su0 = su1;
           sg1 = sg2;
           su1 = su2;
         }
-      } else {
-        take(v, w2);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (gu) {
-            a[r] = __uint_as_float(v[r]);
-            b[r] = __uint_as_float(w2[r]);
-          } else {
-            a[r] = __uint_as_float(v[2 * r]) + __uint_as_float(v[2 * r + 1]);
-          }
+        for (int r = 0; r < 8; ++r) {   // n's row scale, a power of two
+          a[r] *= c->nsc[r];
+          b[r] *= c->nsc[r];
+        }
+      } else {
+        // this expert's activation scales were published with its block
+        // counts: acquire them once (the issuer has seen them complete)
+        if (tid == 0 && ok) ok = wait_count(p, c, &p.xready[sg.x], (uint32_t)geo.nbi, 4u);
+        bar_sync(kBarEpi, 4 * 32);
+        const float4* asc =
+            reinterpret_cast<const float4*>(p.actb + (size_t)sg.x * f8_act_stride(I) + (size_t)I * 16);
+        auto ld_a = [&](int u, float4& lo4, float4& hi4) {
+          const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+          lo4 = u < sg.k1 ? __ldcg(asc + 2 * u) : z;
+          hi4 = u < sg.k1 ? __ldcg(asc + 2 * u + 1) : z;
+        };
+        float4 a0l, a0h, a1l, a1h;
+        ld_a(sg.k0, a0l, a0h);
+        ld_a(sg.k0 + 1, a1l, a1h);
+        for (int u = sg.k0; u < sg.k1; ++u) {
+          const float sg2 = ld_g(u + 2);
+          float4 a2l, a2h;
+          ld_a(u + 2, a2l, a2h);
+          take(v, w2, false);
+          const float k8[8] = {a0l.x, a0l.y, a0l.z, a0l.w, a0h.x, a0h.y, a0h.z, a0h.w};
+#pragma unroll
+          for (int r = 0; r < 8; ++r) a[r] = fmaf(sg0 * k8[r], __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
+          sg0 = sg1;
+          sg1 = sg2;
+          a0l = a1l;
+          a0h = a1h;
+          a1l = a2l;
+          a1h = a2h;
         }
       }
       trace(p, 20, t == 1 && tid == 0);
-      const bool live = ok && cok && !c->dead;
+      const bool live = ok && !c->dead;
       if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
-      epi_store(p, c, geo, sg, gu, live, i, a, b);
-    };
-    // When these warps also convert (MXFP4), a segment's accumulator work
-    // waits until the next segment of the list is converted: the MMAs of
-    // that segment run meanwhile (the accumulators alternate).  The last
-    // segment of a list is finished before the next list starts converting
-    // (a down expert may wait for this CTA's own gate/up block).
-    Seg pend;
-    bool has_pend = false;
-    auto seg = [&](const Seg& sg) {
-      if (!converts) {
-        finish(sg);
-        return;
-      }
-      convert_units(sg);
-      if (has_pend) finish(pend);
-      pend = sg;
-      has_pend = true;
-    };
-    auto flush = [&]() {
-      if (has_pend) finish(pend);
-      has_pend = false;
+      if (gu) f8_store_act(p, c, sg, live, i, a, b);
+      else epi_store(p, c, geo, sg, false, live, i, a, b);
     };
     tc_segments(p, geo, L_SGU, 0, seg);
-    flush();
     trace(p, 6, tid == 0);
     tc_segments(p, geo, L_RGU, nu, seg);
-    flush();
     trace(p, 7, tid == 0);
     tc_segments(p, geo, L_DN, nu, seg);
-    flush();
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
     if (tid == 0) {
@@ -505,15 +617,42 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       red_release_add(&p.sync->cnt_y, 1u);
     }
     tc_fence_before();
-    bar_arrive(kBarEnd, 9 * 32);   // the issuer may free the tensor memory
-  } else {
-    // ============================================================ converters
-    tc_segments(p, geo, L_SGU, 0, convert_units);
-    tc_segments(p, geo, L_RGU, nu, convert_units);
-    tc_segments(p, geo, L_DN, nu, convert_units);
-    tc_fence_before();
-    bar_arrive(kBarEnd, 9 * 32);   // the issuer may free the tensor memory
+    bar_arrive(kBarEnd, 5 * 32);   // the issuer may free the tensor memory
+  } else if (F4) {
+    // ======================================================= expanders
+    // warps 4-7, thread = weight row: each ring stage's codes into an A buffer
+    const int row = (warp - 4) * 32 + lane;
+    uint32_t s = 0;
+    bool cok = true;
+    auto expand = [&](const Seg& sg) {
+      const bool gu = sg.list != L_DN;
+      const int per = stage_units(sg);
+      for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+        const uint32_t slot = s % p.nst, q = s / p.nst;
+        const uint32_t ab = s % kF4Ab, qa = s / kF4Ab;
+        const int n = min(per, sg.k1 - u0);
+        if (lane == 0 && cok) cok = wait_bar(p, c, &full[slot], q & 1);
+        if (lane == 0 && cok && qa > 0) cok = wait_bar(p, c, &c->abempty[ab], (qa - 1) & 1);
+        cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
+        const uint8_t* src = ring + (size_t)slot * p.slot_bytes;
+        const uint32_t dst = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)kF8TmemCols + 64u * ab;
+        tc_fence_after();
+        if (cok) f4_expand_stage(src, dst, row, gu || n == 2);   // gate and up, or one or two down units
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&c->abfull[ab]);
+          mbar_arrive(&empty[slot]);
+        }
+        ++s;
+      }
+    };
+    tc_segments(p, geo, L_SGU, 0, expand);
+    tc_segments(p, geo, L_RGU, nu, expand);
+    tc_segments(p, geo, L_DN, nu, expand);
   }
+  // (FP8: warps 4-7 have no part in the main phase)
 
   // ==================================================================== tail
   bar_sync(kBarCons, kCW * 32);
