@@ -4,8 +4,10 @@
 One step = one fused MoE layer-step of the chosen workload (all rows, every
 stage of the layer, n_layers persistent launches).  Inputs are seeded and
 synthetic; the weights are generated on the device and packed before timing.
-L2 is flushed (512 MiB write) before every timed step, and four hc_in sets
-rotate so the routed experts change from step to step.
+L2 is flushed before every timed step (a 512 MiB write, then a 512 MiB read,
+so that the write-back of the flush's dirty lines is not charged to the
+step), and four hc_in sets rotate so the routed experts change from step to
+step.
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload instead.
@@ -59,7 +61,9 @@ def wl_config(wl, extra=None):
     cfg = {"workload": wl.name, "rows": wl.rows, "hidden": wl.hidden, "hc_streams": wl.hc,
            "routed_experts": wl.n_routed, "top_k": wl.top_k, "shared_experts": 1, "inter": wl.inter,
            "layers_per_step": wl.n_layers, "expert_format": wl.w_dtype, "hc_format": wl.hc_dtype,
-           "l2": "flushed before every timed step (512 MiB write)" if L2_MODE[0] == "flush" else
+           "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so that the "
+                 "written lines are back in HBM and L2 holds only clean lines of an unrelated buffer)"
+                 if L2_MODE[0] == "flush" else
                  "not flushed: every step streams its weights (larger than the 126 MB L2) through it",
            "inputs": f"{N_INPUT_SETS} rotating seeded hc_in sets"}
     if extra:
@@ -185,7 +189,7 @@ TRACE_NAMES = ["start", "mix published", "mix totals seen", "n ready", "logits p
 TRACE_POINTS = 32
 
 
-def print_trace(plan, wl, sets, out, flush):
+def print_trace(plan, wl, sets, out, flush_l2):
     """One extra traced step: stage timestamps relative to the earliest CTA
     start, min / median / max over CTAs (µs), to stderr."""
     import numpy as np
@@ -194,7 +198,7 @@ def print_trace(plan, wl, sets, out, flush):
     G = info["grid"]
     buf = torch.zeros(wl.n_layers * G * TRACE_POINTS, dtype=torch.int64, device="cuda")
     plan.set_trace(buf)
-    flush.zero_()
+    flush_l2()
     plan.step(wl.rows, sets[0], out)
     torch.cuda.synchronize()
     plan.set_trace(None)
@@ -268,11 +272,16 @@ def run_gpu(args):
     bytes_per_set = [sum(info["dense_bytes"] + (u + 1) * info["expert_bytes"] + 2 * hc_bytes for u in us)
                      for us in uniq]
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros((), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
     def flush_l2():
+        # a write pass evicts everything, a read pass then writes the dirty
+        # lines back before the timed region instead of inside it
         if args.l2 == "flush":
             flush.zero_()
+            torch.sum(flush_rd, dim=0, out=flush_acc)
 
     for k in range(args.warmup):
         flush_l2()
@@ -314,7 +323,7 @@ def run_gpu(args):
     e2e_ms = [a.elapsed_time(b) for a, b in ev2]
     clk = clocks.stop()
     if args.trace:
-        print_trace(plan, wl, sets, out, flush)
+        print_trace(plan, wl, sets, out, flush_l2)
     rc, st = plan.query_error()
     if rc != 0:
         raise SystemExit(f"device error {rc} stage {st.stage}")
@@ -376,7 +385,8 @@ def main():
     ap.add_argument("--trace-dump", default=None, help="with --trace: save the raw [layers][grid][32] stamps (.npy)")
     ap.add_argument("--trace", action="store_true", help="print per-stage device timestamps (stderr) after the run")
     ap.add_argument("--l2", default="flush", choices=["flush", "none"],
-                    help="flush: write 512 MiB before every step; none: rely on the step's weights exceeding L2")
+                    help="flush: write, then read, 512 MiB before every step; none: rely on the step's weights "
+                         "exceeding L2")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

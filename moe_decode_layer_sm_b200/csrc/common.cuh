@@ -40,7 +40,7 @@ constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // named barriers: prologue (compute + control), compute, control, epilogue
 // warps 0-3, routing hand-over (compute + control), end (epilogue warps + the
 // issuer warp)
-constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6;
+constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6, kBarTop = 7;
 constexpr int kMaxAb = 6;          // A-tile buffers of the quantised tensor-core kernels
 constexpr int kMaxAcc = 4;         // accumulator buffers in tensor memory
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
@@ -650,7 +650,8 @@ __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_
 // when ctl_topk; otherwise the compute warps do it in route_rows and hand
 // over at the routing barrier), then the list of unique routed experts with
 // their rows and act slots.
-__device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint32_t ep1, bool ctl_topk) {
+__device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint32_t ep1, bool ctl_topk,
+                              bool split = false) {
   const int R = p.R, E = p.E, K = p.K, G = p.G;
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kCtlWarp0;
   const int ct = threadIdx.x - kCtlWarp0 * 32;
@@ -695,8 +696,9 @@ __device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint
     // core kernel is the only caller of this branch)
     router_logits<true>(p, c, regA, true);
     if (cw == 0) topk_dispatch(p, c, 0, true);
-    // the compute warps' top-k rows (route_rows) are in c->idx / c->wt after this
-    bar_sync(kBarRoute, kPreThreads);
+    // the compute warps' top-k rows (route_rows) are in c->idx / c->wt after
+    // this (split: warps 4-7 alone took them)
+    bar_sync(kBarRoute, split ? (4 + kCtlWarps) * 32 : kPreThreads);
   }
   for (int i = ct; i < R * K; i += kCtlWarps * 32) {
     const int e = c->idx[i / K][i % K];
@@ -941,17 +943,21 @@ __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_
   trace(p, 4, ctid == 0);
 }
 
-// A6 on the compute warps, one row per warp: wait for every CTA's logits,
-// then the canonical top-k and weights of each row; the control warps take
-// over (expert lists) at the routing barrier.
-__device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1) {
-  const int R = p.R, E = p.E, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
-  bar_sync(kBarCons, kCW * 32);
-  trace(p, 21, threadIdx.x == 0);
-  for (int r = warp; r < R; r += kCW) topk_dispatch(p, c, r, false);
-  trace(p, 22, threadIdx.x == 0);
-  bar_sync(kBarRoute, kPreThreads);
+// A6, one row per warp: wait for every CTA's logits, then the canonical
+// top-k and weights of each row; the control warps take over (expert lists)
+// at the routing barrier.  On all compute warps, or (split, R <= 4) on warps
+// 4-7 alone while warps 0-3 go on with the shared expert.
+__device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1, bool split) {
+  const int R = p.R, warp = threadIdx.x >> 5;
+  const int w0 = split ? 4 : 0, nw = kCW - w0;
+  const bool lead = (int)threadIdx.x == w0 * 32;
+  if (lead) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
+  if (split) bar_sync(kBarTop, 4 * 32);
+  else bar_sync(kBarCons, kCW * 32);
+  trace(p, 21, lead);
+  for (int r = warp - w0; r < R; r += nw) topk_dispatch(p, c, r, false);
+  trace(p, 22, lead);
+  bar_sync(kBarRoute, (nw + kCtlWarps) * 32);
 }
 
 // Tail on the CTA's h-range: y = bf16(routed + shared) from yfun(r, h), then

@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   // ================================================================ prologue
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, regA, ep1, false);
+    control_warps(p, c, regA, ep1, false, !F4 && p.R <= 4);
     return;
   }
   collapse_norm<true>(p, c, regA, ep1);
@@ -505,15 +505,23 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   bar_sync(kBarCons, kCW * 32);
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
   trace(p, 3, tid == 0);
-  route_rows(p, c, ep1);
-
-  // the compute warps agree on the expert list once
-  if (tid == 0) {
-    const bool ok = wait_flag(p, c, &c->lists_ready);
-    c->nu_comp = (ok && !c->dead) ? c->nu : 0;
+  // R <= 4: warps 4-7 take the top-k while warps 0-3 start on the shared
+  // expert's tiles, which need no routing (MXFP4: warps 4-7 expand)
+  const bool split = !F4 && p.R <= 4;
+  if (!split || warp >= 4) route_rows(p, c, ep1, split);
+  // the warps that need it agree on the expert list once
+  int nu = 0;
+  auto agree = [&]() {
+    if (tid == 0) {
+      const bool ok = wait_flag(p, c, &c->lists_ready);
+      c->nu_comp = (ok && !c->dead) ? c->nu : 0;
+    }
+  };
+  if (!split) {
+    agree();
+    bar_sync(kBarCons, kCW * 32);
+    nu = c->nu_comp;
   }
-  bar_sync(kBarCons, kCW * 32);
-  const int nu = c->nu_comp;
 
   if (warp < 4) {
     // ============================================================ epilogue
@@ -607,6 +615,11 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     };
     tc_segments(p, geo, L_SGU, 0, seg);
     trace(p, 6, tid == 0);
+    if (split) {
+      agree();
+      bar_sync(kBarEpi, 4 * 32);
+      nu = c->nu_comp;
+    }
     tc_segments(p, geo, L_RGU, nu, seg);
     trace(p, 7, tid == 0);
     tc_segments(p, geo, L_DN, nu, seg);
