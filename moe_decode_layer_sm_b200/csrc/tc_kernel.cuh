@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     uint32_t s = 0, issued = 0;
     bool ok = true;
     uint32_t first_copy = 0u;
+    bool dry = false;
     auto seg = [&](const Seg& sg) {
       if (lane != 0) return;
       size_t kgb;
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       const uint32_t bytes = (uint32_t)(kgs * kgb);
       for (int kg = kg0; kg < kg1; kg += kgs) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
-        if (ok) {
+        if (ok && !dry) {
           if (q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
           if (ok) {
             mbar_arrive_expect_tx(&full[slot], bytes);
@@ -323,6 +324,16 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       prefetch_l2_span(p.bias, (size_t)p.E * 4);
     }
     tc_segments(p, geo, L_SGU, 0, seg);
+    {
+      // the routed list's loop once with no waits or copies (one expert's
+      // worth of stages, addresses never used), so that its code is in the
+      // instruction cache when the lists arrive
+      const uint32_t s0 = s;
+      dry = true;
+      tc_segments(p, geo, L_RGU, 1, seg);
+      dry = false;
+      s = s0;
+    }
     if (ok && lane == 0) ok = wait_flag(p, c, &c->lists_ready);
     ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
     const int nu = ok ? *(volatile int*)&c->nu : 0;

@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   // ================================================================ producer
   if (warp == kProdWarp) {
     uint32_t s = 0, issued = 0;
-    bool ok = true;
+    bool ok = true, dry = false;
     auto seg = [&](const Seg& sg) {
       if (lane != 0) return;
       const int e = seg_expert(p, c, sg.x);
@@ -344,13 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       const uint32_t sc_unit = gu ? 256u : 128u;
       const float* sc_base = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : geo.upb_gu) * 256
                                 : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : geo.upb_dn) * 128;
-      if (F4) prefetch_l2(sc_base, sc_unit * 4);
+      if (F4 && !dry) prefetch_l2(sc_base, sc_unit * 4);
       const int per = stage_units(sg);
       for (int u = sg.k0; u < sg.k1; u += per) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
         const uint32_t n = (uint32_t)min(per, sg.k1 - u), bytes = n * ub;
-        if (ok && q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
-        if (ok) {
+        if (ok && !dry && q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
+        if (ok && !dry) {
           mbar_arrive_expect_tx(&full[slot], bytes);
           tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
           issued = s + 1;
@@ -366,6 +366,16 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       prefetch_l2_span(p.bias, (size_t)p.E * 4);
     }
     tc_segments(p, geo, L_SGU, 0, seg);
+    {
+      // the routed list's loop once with no waits or copies (one expert's
+      // worth of stages, addresses never used), so that its code is in the
+      // instruction cache when the lists arrive
+      const uint32_t s0 = s;
+      dry = true;
+      tc_segments(p, geo, L_RGU, 1, seg);
+      dry = false;
+      s = s0;
+    }
     if (ok && lane == 0) ok = wait_flag(p, c, &c->lists_ready);
     ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
     const int nu = ok ? *(volatile int*)&c->nu : 0;
