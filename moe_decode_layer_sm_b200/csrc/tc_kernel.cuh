@@ -70,9 +70,39 @@ struct TcGeo {
   }
 };
 
+// The shared gate/up list is cut along its blocks: block b goes to CTAs
+// [sgu_c0(b), sgu_c0(b + 1)), which split its units evenly, so that no CTA
+// holds parts of two blocks.  (A CTA that holds a block's end and the next
+// block's start finishes two blocks; the second one then completes while
+// the routed weights saturate HBM, where every round trip of its combine
+// takes microseconds, and stalls that CTA's MMAs.)  Used when every block
+// has a CTA of its own.
+__device__ __forceinline__ bool sgu_by_block(const Params& p, const TcGeo& g) { return p.G >= g.nbi; }
+__device__ __forceinline__ int sgu_c0(const Params& p, const TcGeo& g, int b) { return (b * p.G + g.nbi - 1) / g.nbi; }
+// units [k0, k1) of block b for the j-th of its m CTAs
+__device__ __forceinline__ void sgu_share(const TcGeo& g, int j, int m, int& k0, int& k1) {
+  k0 = j * g.upb_gu / m;
+  k1 = (j + 1) * g.upb_gu / m;
+}
+
 // Walk this CTA's segments of one list; f(const Seg&).
 template <class F>
 __device__ __forceinline__ void tc_segments(const Params& p, const TcGeo& g, int list, int nu, F f) {
+  if (list == L_SGU && sgu_by_block(p, g)) {
+    const int b = (int)(((long long)blockIdx.x * g.nbi) / p.G);
+    const int c0 = sgu_c0(p, g, b), m = sgu_c0(p, g, b + 1) - c0;
+    Seg s;
+    sgu_share(g, (int)blockIdx.x - c0, m, s.k0, s.k1);
+    if (s.k0 < s.k1) {
+      s.list = L_SGU;
+      s.x = 0;
+      s.blk = b;
+      s.gblk = b;
+      s.N = (long long)g.nbi * g.upb_gu;
+      f(s);
+    }
+    return;
+  }
   const int upb = list == L_DN ? g.upb_dn : g.upb_gu;
   const int nb = list == L_DN ? g.nbh : g.nbi;
   const long long nexp = list == L_SGU ? 1 : list == L_RGU ? nu : nu + 1;
@@ -121,13 +151,23 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
   const int G = p.G, R = p.R, tid = threadIdx.x;
   volatile int* bcast = &c->bcast;
   const long long u0 = sg.gblk * upb, u1 = u0 + upb;
-  const int c_lo = part_owner(sg.N, G, u0), c_hi = part_owner(sg.N, G, u1 - 1);
+  const bool by_block = sg.list == L_SGU && sgu_by_block(p, geo);   // one segment per CTA, slot 0
+  const int c_lo = by_block ? sgu_c0(p, geo, sg.blk) : part_owner(sg.N, G, u0);
+  const int c_hi = by_block ? sgu_c0(p, geo, sg.blk + 1) - 1 : part_owner(sg.N, G, u1 - 1);
+  // does CTA cc hold a part of this block, and in which slot
+  auto holds = [&](int cc) {
+    if (!by_block) return part_start(sg.N, G, cc) != part_start(sg.N, G, cc + 1);
+    int k0, k1;
+    sgu_share(geo, cc - c_lo, c_hi - c_lo + 1, k0, k1);
+    return k0 < k1;
+  };
+  auto slot_of = [&](int cc, int sl0) { return by_block ? 0 : sl0 + (part_start(sg.N, G, cc) >= u0 ? 0 : 1); };
   if (c_lo == c_hi) return true;
   // part slots: a CTA's first and last segment of a list (0 / 1), the
   // routed gate/up list after the shared one (2 / 3)
   const int nsl = gu ? 4 : 2, sl0 = sg.list == L_RGU ? 2 : 0;
   const bool q1 = R > 4;
-  const int slot = sl0 + (part_start(sg.N, G, blockIdx.x) >= u0 ? 0 : 1);
+  const int slot = slot_of((int)blockIdx.x, sl0);
   float4* mine = reinterpret_cast<float4*>((gu ? p.gpart : p.dpart) + (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16);
   if (live) {
     __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
@@ -140,7 +180,7 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
   if (tid == 0) {
     uint32_t* cnt = (gu ? p.gcnt : p.dcnt) + (size_t)sg.x * (gu ? geo.nbi : geo.nbh) + sg.blk;
     int parts = 0;
-    for (int cc = c_lo; cc <= c_hi; ++cc) parts += part_start(sg.N, G, cc) != part_start(sg.N, G, cc + 1);
+    for (int cc = c_lo; cc <= c_hi; ++cc) parts += holds(cc) ? 1 : 0;
     const uint32_t old = live ? atomicAdd(cnt, 1u) : 0u;
     const bool last = live && old == (uint32_t)(parts - 1);
     if (last) atomicExch(cnt, 0u);   // ready for the next step
@@ -159,9 +199,8 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int cc = cb + j;
-        const long long ps = part_start(sg.N, G, cc);
-        use[j] = cc <= c_hi && ps != part_start(sg.N, G, cc + 1);   // skip empty ranges
-        const int sl = sl0 + (ps >= u0 ? 0 : 1);
+        use[j] = cc <= c_hi && holds(cc);   // skip empty ranges
+        const int sl = slot_of(cc, sl0);
         const float4* src =
             reinterpret_cast<const float4*>((gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + sl) * 128 + i) * 16);
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
