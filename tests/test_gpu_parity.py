@@ -177,6 +177,25 @@ def test_scaled_mxfp4_wide_block_spread():
     run.close()
 
 
+def test_mxfp4_nan_scale_refused_at_packing():
+    """e8m0 code 255 is NaN: the tensor-core path's packing refuses it with
+    INVALID_ARG before any step, instead of expanding a NaN scale."""
+    import torch
+    from moe_decode_layer_sm_b200 import Plan
+    from moe_decode_layer_sm_b200.binding import MonoError
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=451)
+    plan = Plan.for_workload(wl)
+    d = S.gpu_dense(wl, 0)
+    ex = S.gpu_experts(wl, 0)
+    ex["up"][1][3, 17, 2] = 255
+    torch.cuda.synchronize()
+    with pytest.raises(MonoError) as err:
+        plan.pack(0, d["mix_w"], d["norm_w"], d["router_w"], d["router_bias"], ex["gate"][0], ex["up"][0],
+                  ex["down"][0], ex["gate"][1], ex["up"][1], ex["down"][1])
+    assert "NaN" in str(err.value) and "INVALID_ARG" in str(err.value)
+    plan.close()
+
+
 def test_scaled_mxfp4_single_layer():
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=401)
     run = GpuRun(wl)
