@@ -180,11 +180,22 @@ typedef struct mono_ffn_plan_s mono_ffn_plan_t;
 int mono_ffn_plan(const mono_ffn_config* cfg, mono_ffn_plan_t** out);
 
 /* Repack one layer's weights (logical layouts above) into the plan's kernel
- * layout: expert rows cut into contraction chunks with their block scales
- * interleaved, gate and up chunks of a channel adjacent, router transposed to
- * [E][H].  A one-time conversion (vLLM MonoKernel page, Weights: "packed
- * once").  Asynchronous on `stream`; the inputs may be freed after the
- * stream reaches this point. */
+ * layout, router transposed to [E][H].  A one-time conversion (vLLM
+ * MonoKernel page, Weights: "packed once").  Expert layouts:
+ *   - bf16 on the tensor cores (hidden, inter multiples of 128): blocks of 128
+ *     rows of K-major core matrices, gate and up interleaved per row group;
+ *   - FP8 / MXFP4 on the tensor cores (bf16-rounded layers, multiples of 128):
+ *     units of 128 rows x 128 inputs, 16-byte chunk j of row i at [j][i];
+ *     FP8 block scales in arrays of their own; MXFP4 with the sign bits moved
+ *     inside each 32-bit word of 8 codes, each block's exponent stored
+ *     relative to its row's largest minus 6, and 2^(that reference) per row
+ *     in arrays of their own;
+ *   - otherwise rows cut into contraction chunks with their block scales
+ *     interleaved, gate and up chunks of a channel adjacent.
+ * Asynchronous on `stream`; the inputs may be freed after the stream reaches
+ * this point.  MXFP4 on the tensor cores first reads the scale codes
+ * (synchronising `stream`) and refuses code 255 (NaN) with
+ * MONO_ERR_INVALID_ARG. */
 int mono_ffn_pack_weights(mono_ffn_plan_t* plan, int layer, const mono_ffn_layer_weights* w, void* stream);
 
 /* Run one step: n_layers persistent launches on `stream`.  hc_in, hc_out:
