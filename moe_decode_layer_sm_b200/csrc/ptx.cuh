@@ -159,17 +159,10 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(da), "l"(db), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// The same from a converged warp: one elected lane issues (the same lane
-// every time, so its commits track all of its MMAs); the operands stay
-// warp-uniform, which keeps the descriptor arithmetic cheap.
+// One tcgen05.mma (kind::f16) from a converged warp: one elected lane issues
+// (the same lane every time, so its commits track all of its MMAs); the
+// operands stay warp-uniform, which keeps the descriptor arithmetic cheap.
+// acc: accumulate into D (else overwrite).
 __device__ __forceinline__ void umma_bf16_warp(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n .reg .pred p, e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
@@ -177,6 +170,8 @@ __device__ __forceinline__ void umma_bf16_warp(uint32_t tmem_d, uint64_t da, uin
       "l"(da), "l"(db), "r"(idesc), "r"(acc)
       : "memory");
 }
+// Arrive once on bar when every tcgen05 operation the elected lane issued so
+// far is complete (from a converged warp).
 __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n .reg .pred e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
@@ -282,12 +277,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// arrive once on bar when every tcgen05 operation this thread issued so far is complete
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
