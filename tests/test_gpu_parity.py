@@ -204,13 +204,14 @@ def test_scaled_mxfp4_single_layer():
     run.close()
 
 
-@pytest.mark.parametrize("wdt", ["bf16", "mxfp4"])
-def test_scaled_chain_four_layers(wdt):
+@pytest.mark.parametrize("wdt, rows", [("bf16", 8), ("mxfp4", 8), ("bf16", 2), ("mxfp4", 1)])
+def test_scaled_chain_four_layers(wdt, rows):
     """Each layer of the chain checked on the residual streams the kernel
     materialised for it (x tap): routing exact (near-tie exemption), y and the
     next layer's streams within tolerance, and the final output.  Then the
-    whole chain against the oracle's own chain."""
-    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, w_dtype=wdt, seed=402)
+    whole chain against the oracle's own chain, at 8, 2 and 1 rows (R <= 4
+    also moves the top-k to warps 4-7 on the bf16 path)."""
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, w_dtype=wdt, seed=402, rows=rows)
     run = GpuRun(wl)
     got = run.step()
     lws = [O.LayerWeights(wl, S.cpu_dense(wl, l), all_experts(wl, l)) for l in range(wl.n_layers)]
