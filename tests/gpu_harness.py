@@ -15,7 +15,7 @@ BF16_MAX_ABS = 5e-2
 TIE_REL = 1e-5
 
 
-class GpuRun:
+class LayerRun:
     """Generate a workload's inputs on the device, pack, and run steps."""
 
     def __init__(self, wl, dense_override=None, hc_in=None, **plan_kw):

@@ -10,7 +10,7 @@ import pytest
 from oracle import oracle as O
 from synth import configs as C
 from synth import synth as S
-from tests.gpu_harness import GpuRun, compare_out, routing_ok
+from tests.gpu_harness import LayerRun, compare_out, routing_ok
 from tests.oracle_helpers import touched_experts
 
 pytestmark = pytest.mark.gpu
@@ -65,7 +65,7 @@ def _all_rows_routing(wl, run):
 @pytest.mark.parametrize("wl, rows", [(C.FLASH_BF16_R1, [0]), (C.FLASH_BF16_R8, [0, 7]), (C.FLASH_BF16_R6, [2]),
                                       (C.FLASH_FP8_R4, [0, 3])], ids=lambda x: getattr(x, "name", str(x)))
 def test_full_size_single_layer(wl, rows):
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     got = run.step()
     _all_rows_routing(wl, run)
     out, t, keep = _check_rows(wl, run, rows)
@@ -81,7 +81,7 @@ def test_full_size_single_layer(wl, rows):
 
 def test_full_size_mxfp4_chain_row_sample():
     wl = C.FLASH_MXFP4_CHAIN4_R8
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     got = run.step()
     _all_rows_routing(wl, run)
     r = [5]

@@ -9,7 +9,7 @@ import pytest
 from oracle import oracle as O
 from synth import configs as C
 from synth import synth as S
-from tests.gpu_harness import GpuRun, compare_out, oracle_rows, raw_hc, routing_ok, select_weights
+from tests.gpu_harness import LayerRun, compare_out, oracle_rows, raw_hc, routing_ok, select_weights
 from tests.oracle_helpers import all_experts
 
 pytestmark = pytest.mark.gpu
@@ -60,7 +60,7 @@ def _check_layer(wl, run, rows, layer=0, hc_in=None, dense=None):
 
 def test_tiny_fp32_all_rows():
     wl = C.TINY_FP32
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, [0])
     run.close()
@@ -69,7 +69,7 @@ def test_tiny_fp32_all_rows():
 @pytest.mark.parametrize("rows", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_tiny_fp32_rows_sweep(rows):
     wl = C.TINY_FP32.with_(rows=rows, seed=100 + rows)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, list(range(rows)))
     run.close()
@@ -80,7 +80,7 @@ def test_rows_zero_is_noop_and_rows_above_max_refused():
 
     from moe_decode_layer_sm_b200 import MonoError
     wl = C.TINY_FP32.with_(rows=2)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.out.fill_(7.0)
     run.plan.step(0, run.hc, run.out)
     torch.cuda.synchronize()
@@ -101,7 +101,7 @@ def test_zero_input_tie_rounds(bias):
         levels = np.array([-0.075, -0.025, 0.025, 0.075], np.float32)
         b = levels[np.minimum(3, np.floor((d["router_bias"] + 0.1) / 0.05).astype(int))]
     hc = torch.zeros((2, 4, wl.hidden), dtype=torch.float32, device="cuda")
-    run = GpuRun(wl, dense_override=lambda l: {"router_bias": b}, hc_in=hc)
+    run = LayerRun(wl, dense_override=lambda l: {"router_bias": b}, hc_in=hc)
     run.step()
     d["router_bias"] = b
     t = _check_layer(wl, run, [0, 1], hc_in=np.zeros((2, 4, wl.hidden), np.float32), dense=d)
@@ -114,7 +114,7 @@ def test_zero_input_tie_rounds(bias):
 @pytest.mark.parametrize("rows", [1, 3, 8])
 def test_scaled_bf16(rows):
     wl = C.scaled(C.FLASH_BF16_R8, rows=rows, seed=200 + rows)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, list(range(rows)))
     # a second step on the same plan (epoch-tagged counters, no reset) gives the same bytes
@@ -126,7 +126,7 @@ def test_scaled_bf16(rows):
 
 def test_scaled_fp8_rows4():
     wl = C.scaled(C.FLASH_FP8_R4, seed=301)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
     run.close()
@@ -136,7 +136,7 @@ def test_cuda_core_bf16_hidden_not_multiple_of_128():
     """bf16 experts with hidden 1056 and inter 544: not whole 128-row blocks,
     so the CUDA-core kernel."""
     wl = C.scaled(C.FLASH_BF16_R8, seed=221, hidden=1056, inter=544, rows=5)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     assert run.plan.info()["ring_slot_bytes"] != 16384   # not the tensor-core layout
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
@@ -148,7 +148,7 @@ def test_cuda_core_fp8_fp32_streams():
     CUDA-core kernel (the tensor-core kernels take only the rounded layer);
     compared at the fp32 tolerance."""
     wl = C.scaled(C.FLASH_FP8_R4, seed=311, hc_dtype="f32", norm_dtype="f32", round_bf16=False)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     assert run.plan.info()["ring_slot_bytes"] != 2 * 16384   # not the tensor-core layout
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
@@ -159,7 +159,7 @@ def test_cuda_core_mxfp4_hidden_not_multiple_of_128():
     """MXFP4 with hidden 1056 and inter 544 (multiples of 32, not of 128): the
     CUDA-core kernel."""
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=411, hidden=1056, inter=544, rows=3)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     assert run.plan.info()["ring_slot_bytes"] != 2 * (8192 + 512)
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
@@ -171,7 +171,7 @@ def test_scaled_mxfp4_wide_block_spread():
     e4m3 expansion relative to each row's largest scale takes its table, its
     one-by-one (subnormal) and its rounded branches."""
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=431, mx_spread=20)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
     run.close()
@@ -198,7 +198,7 @@ def test_mxfp4_nan_scale_refused_at_packing():
 
 def test_scaled_mxfp4_single_layer():
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=401)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
     run.close()
@@ -212,7 +212,7 @@ def test_scaled_chain_four_layers(wdt, rows):
     whole chain against the oracle's own chain, at 8, 2 and 1 rows (R <= 4
     also moves the top-k to warps 4-7 on the bf16 path)."""
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, w_dtype=wdt, seed=402, rows=rows)
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     got = run.step()
     lws = [O.LayerWeights(wl, S.cpu_dense(wl, l), all_experts(wl, l)) for l in range(wl.n_layers)]
     assert np.array_equal(run.tap(0, "x"), O.decode_hc(wl, S.cpu_hc_in(wl)))
@@ -240,7 +240,7 @@ def test_device_timeout_is_reported_and_recovers():
     wait expires, the step reports DEVICE_TIMEOUT, and the next step on the
     same plan is correct again."""
     wl = C.TINY_FP32.with_(rows=1)
-    run = GpuRun(wl, wait_timeout_us=20000)
+    run = LayerRun(wl, wait_timeout_us=20000)
     run.plan.debug_skip_arrival(3)
     run.plan.step(1, run.hc, run.out)
     rc, st = run.plan.query_error()

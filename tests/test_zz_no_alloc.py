@@ -10,7 +10,7 @@ import pytest
 from moe_decode_layer_sm_b200 import binding
 from synth import configs as C
 from synth import synth as S
-from tests.gpu_harness import FP32_MAX_ABS, GpuRun, routing_ok
+from tests.gpu_harness import FP32_MAX_ABS, LayerRun, routing_ok
 
 
 def _sel(wl, logits, bias):
@@ -31,7 +31,7 @@ CASES = {
 def test_route_noalloc_matches_fused_step(case):
     import torch
     wl = CASES[case]()
-    run = GpuRun(wl)
+    run = LayerRun(wl)
     run.step()
     R, K = wl.rows, wl.top_k
     d = S.gpu_dense(wl, 0)
