@@ -157,7 +157,7 @@ class Plan:
         return rc, st
 
     def set_trace(self, buf):
-        """buf: int64 device tensor of n_layers * grid * 16 entries, or None."""
+        """buf: int64 device tensor of n_layers * grid * 32 entries, or None."""
         self._check(self._lib.mono_ffn_set_trace(self.handle, _ptr(buf)))
 
     def debug_skip_arrival(self, cta):
