@@ -217,6 +217,24 @@ def print_trace(plan, wl, sets, out, flush_l2):
             print(f"  {i:2d} {nm:22s} {d.min():9.2f} {statistics.median(d):9.2f} {d.max():9.2f}  (n={len(col)})",
                   file=sys.stderr)
 
+def job_times(tot_ms, tot_e2e, world, device):
+    """Max over ranks of each rank's timed totals (ms).  Every rank calls it,
+    at the same point, on the initialised process group."""
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([tot_ms, tot_e2e], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, tot_e2e = t.tolist()
+    return tot_ms, tot_e2e
+
+
+def job_value(tot_ms, steps, layers, world):
+    """µs per layer-step of the whole job: the layer-steps of all ranks in the
+    max-over-ranks time (replicas: the work grows with the ranks)."""
+    return tot_ms * 1000.0 / steps / layers / world
+
+
 def run_gpu(args):
     import numpy as np
     import torch
@@ -330,12 +348,8 @@ def run_gpu(args):
 
     tot_ms = sum(step_ms)
     tot_e2e = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms, tot_e2e], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, tot_e2e = t.tolist()
-    us_per_step = tot_ms * 1000.0 / K
-    value = us_per_step / wl.n_layers / world       # whole job: layer-steps of all ranks per unit time
+    tot_ms, tot_e2e = job_times(tot_ms, tot_e2e, world, "cuda")
+    value = job_value(tot_ms, K, wl.n_layers, world)
     mean_bytes = sum(bytes_per_set[k % N_INPUT_SETS] for k in range(K)) / K
     achieved = mean_bytes / (tot_ms / 1000.0 / K) / 1e9
     pk, pk_kind = peaks()
@@ -355,7 +369,7 @@ def run_gpu(args):
                      "peak_kind": f"{pk_kind} HBM copy", "frac_of_8tbs_nominal": achieved / 8000.0,
                      "algorithmic_bytes_per_step": mean_bytes,
                      "unique_routed_experts_per_layer": statistics.mean(x for us in uniq for x in us)},
-        "e2e": {"value": tot_e2e * 1000.0 / KE / wl.n_layers / world, "unit": UNIT, "h2d_bytes_per_step": hc_bytes,
+        "e2e": {"value": job_value(tot_e2e, KE, wl.n_layers, world), "unit": UNIT, "h2d_bytes_per_step": hc_bytes,
                 "d2h_bytes_per_step": hc_bytes},
         "gpu_launches": K * wl.n_layers,
         "clocks": clk,
