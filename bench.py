@@ -9,8 +9,13 @@ so that the write-back of the flush's dirty lines is not charged to the
 step), and four hc_in sets rotate so the routed experts change from step to
 step.
 
-Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle on a
-bounded sample of the same workload instead.
+Prints ONE JSON line (rank 0).  Its headline (`value`, `roofline`, `e2e`)
+is the --config workload (default: the bf16 layer at one row); `per_config`
+then holds every configuration of the metric (rows 1, 6 and 8 bf16, FP8 at
+4 rows, the 4-layer MXFP4 chain at 8 rows), each timed the same way, with
+the CPU oracle on a bounded sample at one thread and on every host core.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead.
 """
 
 import argparse
@@ -125,39 +130,75 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU baseline --
 
-def cpu_oracle_sample(wl, budget_s=12.0):
-    """Time the CPU oracle (as it stands) on one full layer-step of the
-    workload's first input set; weights of the touched experts are generated
-    before the clock starts.  Repeats while the budget lasts."""
+def _omp_threads(n):
+    """Thread count of the oracle's OpenMP regions started from this thread."""
+    import ctypes
+    try:
+        ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+        return True
+    except OSError:
+        return False
+
+
+def _oracle_case(wl):
+    """The oracle's inputs for a bounded sample of the workload: the whole
+    step when it has one row and one layer, else row 0 of layer 0 (the
+    oracle works row by row, so a row's time times the rows is the step's,
+    per layer).  Only the experts the sample touches are generated, before
+    any clock starts.  Returns (layer weights, hc rows, scale, description)."""
     from oracle import oracle as O
     from synth import synth as S
     hc = S.cpu_hc_in(wl)
-    lws = []
-    x = hc
-    for l in range(wl.n_layers):
-        dense = S.cpu_dense(wl, l)
-        t = O.route(wl, O.LayerWeights(wl, dense, {}), x)
-        slots = sorted(set(int(e) for e in t.idx.ravel()) | {wl.n_routed})
-        lw = O.LayerWeights(wl, dense, {e: S.cpu_expert(wl, l, e) for e in slots})
-        lws.append(lw)
-        if l + 1 < wl.n_layers:
-            x, _ = O.layer(wl, lw, x)
+    scale = 1
+    what = f"one full layer-step of {wl.name} ({wl.rows} rows)"
+    if wl.rows > 1 or wl.n_layers > 1:
+        hc = hc[:1]
+        scale = wl.rows
+        what = (f"row 0 of layer 0 of {wl.name}, times {wl.rows} rows (the oracle computes rows one by one)")
+    w1 = wl.with_(rows=hc.shape[0])
+    dense = S.cpu_dense(wl, 0)
+    t = O.route(w1, O.LayerWeights(w1, dense, {}), hc)
+    slots = sorted(set(int(e) for e in t.idx.ravel()) | {wl.n_routed})
+    lw = O.LayerWeights(w1, dense, {e: S.cpu_expert(wl, 0, e) for e in slots})
+    return w1, lw, hc, scale, what
+
+
+def cpu_oracle_sample(wl, budget_s=12.0, threads=None, case=None):
+    """Time the CPU oracle (as it stands) on a bounded sample of the
+    workload (_oracle_case), in µs per layer-step.  threads: None = every
+    host core, else that many OpenMP threads.  Repeats (up to 5) while the
+    budget lasts; the median counts."""
+    from oracle import oracle as O
+    w1, lw, hc, scale, what = case if case is not None else _oracle_case(wl)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    if threads is not None and _omp_threads(threads):
+        cores = threads
+    elif threads is None:
+        _omp_threads(cores)
+    O.layer(w1, lw, hc)   # untimed: first touch of the weights
     times = []
     t_end = time.time() + budget_s
     while time.time() < t_end or not times:
         t0 = time.perf_counter()
-        if wl.n_layers == 1:
-            O.layer(wl, lws[0], hc)
-        else:
-            O.chain(wl, lws, hc, deferred=True)
+        O.layer(w1, lw, hc)
         times.append(time.perf_counter() - t0)
         if len(times) >= 5:
             break
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    us = statistics.median(times) * 1e6 / wl.n_layers
+    _omp_threads(int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)))
+    us = statistics.median(times) * 1e6 * scale
     return {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(times)} full layer-step(s) of {wl.name} ({wl.rows} rows, {wl.n_layers} layer(s)), "
-                      f"median; touched experts generated before timing"}
+            "sample": f"{what}; median of {len(times)}; touched experts generated before timing"}
+
+
+def cpu_baselines(wl, budget_s=12.0):
+    """The oracle on every host core and on one thread, same sample."""
+    case = _oracle_case(wl)
+    return {"all_cores": cpu_oracle_sample(wl, budget_s, None, case),
+            "one_thread": cpu_oracle_sample(wl, budget_s, 1, case)}
+
+
+def parallelism(world):
+    return "replicas" if world > 1 else "none (one replica)"
 
 
 def run_reference(args):
@@ -171,7 +212,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": cb["value"] / 1000.0, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-            "config": wl_config(wl, {"parallelism": "single host process"}), "impl": "reference",
+            "config": wl_config(wl, {"parallelism": parallelism(args.gpus)}), "impl": "reference",
             "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -235,33 +276,31 @@ def job_value(tot_ms, steps, layers, world):
     return tot_ms * 1000.0 / steps / layers / world
 
 
-def run_gpu(args):
+PER_CONFIG = ["v41flash-bf16-r1", "v41flash-bf16-r6", "v41flash-bf16-r8", "v41flash-fp8b128-r4",
+              "v41flash-mxfp4-chain4-r8"]
+
+
+def traffic_of(wl):
+    """ncu DRAM bytes per launch from profiles/, if captured at these sources."""
+    tr_path = os.path.join(ROOT, "profiles", f"traffic_{wl.name}.json")
+    if os.path.exists(tr_path):
+        tr = json.load(open(tr_path))
+        if tr.get("kernel_sha") == kernel_sha():
+            return tr.get("dram_bytes_per_launch")
+    return None
+
+
+def measure(wl, args, ctx):
+    """Plan, pack and time one workload: K steps with inputs resident (CUDA
+    events on the launching stream, L2 flushed before each), then K steps
+    end to end through mono_ffn_step_host.  Every rank runs it at the same
+    point (the barriers and the max over ranks)."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     from moe_decode_layer_sm_b200 import Plan
     from synth import synth as S
-
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    wl = workload(args.config)
-    if args.routed:
-        wl = wl.with_(name=f"{wl.name}-e{args.routed}", n_routed=args.routed)
-    if args.inter:
-        wl = wl.with_(name=f"{wl.name}-i{args.inter}", inter=args.inter)
+    rank, world, local, barrier, flush_l2 = ctx["rank"], ctx["world"], ctx["local"], ctx["barrier"], ctx["flush"]
     plan = Plan.for_workload(wl, device=local)
     info = plan.info()
     for l in range(wl.n_layers):
@@ -286,21 +325,12 @@ def run_gpu(args):
         if rc != 0:
             raise SystemExit(f"device error {rc} stage {st.stage}")
         uniq.append([len(set(t.cpu().numpy().ravel().tolist())) for t in idx_taps])
+    for l in range(wl.n_layers):
+        plan.clear_taps(l)
     hc_bytes = wl.rows * wl.hc * wl.hidden * (2 if wl.hc_dtype == "bf16" else 4)
     bytes_per_set = [sum(info["dense_bytes"] + (u + 1) * info["expert_bytes"] + 2 * hc_bytes for u in us)
                      for us in uniq]
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    flush_rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    flush_acc = torch.zeros((), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
-
-    def flush_l2():
-        # a write pass evicts everything, a read pass then writes the dirty
-        # lines back before the timed region instead of inside it
-        if args.l2 == "flush":
-            flush.zero_()
-            torch.sum(flush_rd, dim=0, out=flush_acc)
-
     for k in range(args.warmup):
         flush_l2()
         plan.step(wl.rows, sets[k % N_INPUT_SETS], out)
@@ -325,7 +355,7 @@ def run_gpu(args):
 
     # end to end through the host-buffer entry point: H2D of the step's hc_in
     # from pinned memory, the step, D2H of the result, per step
-    host_in = [s.cpu().pin_memory() for s in sets]
+    host_in = [x.cpu().pin_memory() for x in sets]
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     KE = min(K, args.e2e_steps)
     ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KE)]
@@ -345,27 +375,20 @@ def run_gpu(args):
     rc, st = plan.query_error()
     if rc != 0:
         raise SystemExit(f"device error {rc} stage {st.stage}")
+    plan.close()
+    del plan, sets, out, host_in, host_out
+    torch.cuda.empty_cache()
 
-    tot_ms = sum(step_ms)
-    tot_e2e = sum(e2e_ms)
-    tot_ms, tot_e2e = job_times(tot_ms, tot_e2e, world, "cuda")
-    value = job_value(tot_ms, K, wl.n_layers, world)
+    tot_ms, tot_e2e = job_times(sum(step_ms), sum(e2e_ms), world, "cuda")
     mean_bytes = sum(bytes_per_set[k % N_INPUT_SETS] for k in range(K)) / K
     achieved = mean_bytes / (tot_ms / 1000.0 / K) / 1e9
     pk, pk_kind = peaks()
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", f"traffic_{wl.name}.json")
-    if os.path.exists(tr_path):
-        tr = json.load(open(tr_path))
-        if tr.get("kernel_sha") == kernel_sha():
-            traffic = tr.get("dram_bytes_per_launch")
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": tot_ms / K, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": dtype_of(wl), "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
-        "config": wl_config(wl, {"parallelism": "replicas" if world > 1 else "single GPU"}),
+    return {
+        "workload": wl.name, "rows": wl.rows, "layers_per_step": wl.n_layers, "expert_format": wl.w_dtype,
+        "value": job_value(tot_ms, K, wl.n_layers, world), "unit": UNIT, "ms_per_step": tot_ms / K,
+        "step_us_p10_p50_p90": [float(np.percentile(step_ms, q)) * 1000.0 for q in (10, 50, 90)],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic_of(wl),
                      "peak_kind": f"{pk_kind} HBM copy", "frac_of_8tbs_nominal": achieved / 8000.0,
                      "algorithmic_bytes_per_step": mean_bytes,
                      "unique_routed_experts_per_layer": statistics.mean(x for us in uniq for x in us)},
@@ -373,12 +396,77 @@ def run_gpu(args):
                 "d2h_bytes_per_step": hc_bytes},
         "gpu_launches": K * wl.n_layers,
         "clocks": clk,
-        "step_us_p10_p50_p90": [float(np.percentile(step_ms, q)) * 1000.0 for q in (10, 50, 90)],
         "plan": {k: info[k] for k in ("grid", "threads", "smem_bytes", "ring_stages", "ring_slot_bytes")},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(wl)
-    plan.close()
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros((), dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        # a write pass evicts everything, a read pass then writes the dirty
+        # lines back before the timed region instead of inside it
+        if args.l2 == "flush":
+            flush.zero_()
+            torch.sum(flush_rd, dim=0, out=flush_acc)
+
+    ctx = {"rank": rank, "world": world, "local": local, "barrier": barrier, "flush": flush_l2}
+    wl = workload(args.config)
+    if args.routed:
+        wl = wl.with_(name=f"{wl.name}-e{args.routed}", n_routed=args.routed)
+    if args.inter:
+        wl = wl.with_(name=f"{wl.name}-i{args.inter}", inter=args.inter)
+    head = measure(wl, args, ctx)
+    others = []
+    if not args.no_per_config and not args.routed and not args.inter:
+        # every configuration of the metric (rows = 1..8, each expert format),
+        # in the same run, each with its own plan
+        for name in PER_CONFIG:
+            if name != wl.name:
+                others.append(measure(workload(name), args, ctx))
+    cpu_on = rank == 0 and world == 1 and not args.no_cpu_baseline
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": dtype_of(wl),
+        "data": "synthetic (seeded generator, random-init weights of the layer's shape)",
+        "config": wl_config(wl, {"parallelism": parallelism(world)}),
+        "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"], "step_us_p10_p50_p90": head["step_us_p10_p50_p90"], "plan": head["plan"],
+    }
+    if cpu_on:
+        cb = cpu_baselines(wl)
+        line["cpu_baseline"] = cb["all_cores"]
+        line["cpu_baseline_one_thread"] = cb["one_thread"]
+    if others or cpu_on:
+        per = {}
+        for m in [head] + others:
+            entry = {k: m[k] for k in ("rows", "layers_per_step", "expert_format", "value", "unit",
+                                       "step_us_p10_p50_p90", "roofline", "e2e", "clocks")}
+            if cpu_on:
+                entry["cpu_baseline"] = cpu_baselines(workload(m["workload"])) if m is not head else \
+                    {"all_cores": line["cpu_baseline"], "one_thread": line["cpu_baseline_one_thread"]}
+            per[m["workload"]] = entry
+        line["per_config"] = per
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -388,12 +476,14 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mono", choices=["mono", "reference"])
     ap.add_argument("--config", default="v41flash-bf16-r1")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only --config (by default every configuration of the metric follows it)")
     ap.add_argument("--routed", type=int, default=0, help="override the routed-expert count (small profiling cases)")
     ap.add_argument("--inter", type=int, default=0, help="override the expert width (small profiling cases)")
     ap.add_argument("--trace-dump", default=None, help="with --trace: save the raw [layers][grid][32] stamps (.npy)")

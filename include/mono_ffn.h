@@ -240,9 +240,28 @@ int mono_ffn_get_info(const mono_ffn_plan_t* plan, mono_ffn_info* info);
  * NULL turns it off (the default). */
 int mono_ffn_set_trace(mono_ffn_plan_t* plan, unsigned long long* buf);
 
-/* Fault injection for tests: CTA `cta` (-1 = none) withholds its arrival at
- * the router-logits counter, so every CTA's bounded wait expires. */
-int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* plan, int cta);
+/* Fault injection for tests (no GPU fault: every wait is bounded).  CTA
+ * `cta` (-1 = none) withholds its arrival at one grid stage, so the other
+ * CTAs' bounded waits there expire and mono_ffn_query_error reports
+ * MONO_ERR_DEVICE_TIMEOUT with that stage:
+ *   MONO_STAGE_MIX, MONO_STAGE_COLLAPSE, MONO_STAGE_LOGITS: the prologue's
+ *     grid stages;
+ *   MONO_STAGE_ACT: the CUDA-core kernel's activation counter; on the
+ *     tensor-core kernels the per-expert activation count of the shared
+ *     expert's first gate/up block (withheld by whichever CTA completes that
+ *     block; `cta` only enables it);
+ *   MONO_STAGE_Y: the expert-output counter (tensor-core kernels only).
+ * Other stages, or cta >= grid, are MONO_ERR_INVALID_ARG.  Stays in force
+ * until called with cta = -1. */
+int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* plan, int cta, int stage);
+
+/* Race detection for tests: with max_ns > 0 (at most 100000) every thread
+ * that publishes a grid-visible arrival (the stage counters, the split-block
+ * arrivals of the tensor-core kernels, the per-expert activation counts)
+ * first sleeps a pseudo-random hash(CTA, step epoch, point) % max_ns
+ * nanoseconds, so the order in which CTAs arrive changes from step to step;
+ * results must not change.  0 turns it off (the default). */
+int mono_ffn_debug_jitter(mono_ffn_plan_t* plan, unsigned max_ns);
 
 /* Router select without a plan and without allocating anything.
  *

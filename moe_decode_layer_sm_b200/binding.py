@@ -15,12 +15,15 @@ SO = os.path.join(PKG, "libmonoffn.so")
 F32, BF16, FP8E4M3_B128, MXFP4 = 0, 1, 2, 3
 DTYPE = {"f32": F32, "bf16": BF16, "fp8": FP8E4M3_B128, "mxfp4": MXFP4}
 
+STAGE = {"MIX": 1, "LOGITS": 2, "LISTS": 3, "ACT": 4, "RING": 5, "Y": 6, "COLLAPSE": 7}
+
 ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED_ARCH", -3: "NOT_CORESIDENT", -4: "OOM",
           -5: "NOT_PACKED", -6: "CUDA", -7: "DEVICE_TIMEOUT", -8: "DEVICE_ABORTED"}
 
 SYMBOLS = ["mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
            "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_last_error",
-           "mono_ffn_destroy", "mono_ffn_abi_version", "mono_ffn_set_trace", "mono_ffn_route_noalloc"]
+           "mono_ffn_destroy", "mono_ffn_abi_version", "mono_ffn_set_trace", "mono_ffn_route_noalloc",
+           "mono_ffn_debug_jitter"]
 
 
 class Config(ctypes.Structure):
@@ -72,7 +75,8 @@ def lib():
         L.mono_ffn_set_taps.argtypes = [vp, i32, ctypes.POINTER(TapsStruct)]
         L.mono_ffn_query_error.argtypes = [vp, ctypes.POINTER(Status)]
         L.mono_ffn_get_info.argtypes = [vp, ctypes.POINTER(Info)]
-        L.mono_ffn_debug_skip_arrival.argtypes = [vp, i32]
+        L.mono_ffn_debug_skip_arrival.argtypes = [vp, i32, i32]
+        L.mono_ffn_debug_jitter.argtypes = [vp, ctypes.c_uint]
         L.mono_ffn_set_trace.argtypes = [vp, vp]
         L.mono_ffn_last_error.argtypes = [vp]
         L.mono_ffn_last_error.restype = ctypes.c_char_p
@@ -82,7 +86,7 @@ def lib():
         L.mono_ffn_route_noalloc.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, f32, f32, vp, vp, vp]
         for f in ("mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
                   "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_abi_version",
-                  "mono_ffn_set_trace", "mono_ffn_route_noalloc"):
+                  "mono_ffn_set_trace", "mono_ffn_route_noalloc", "mono_ffn_debug_jitter"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -160,8 +164,13 @@ class Plan:
         """buf: int64 device tensor of n_layers * grid * 32 entries, or None."""
         self._check(self._lib.mono_ffn_set_trace(self.handle, _ptr(buf)))
 
-    def debug_skip_arrival(self, cta):
-        self._check(self._lib.mono_ffn_debug_skip_arrival(self.handle, cta))
+    def debug_skip_arrival(self, cta, stage=STAGE["LOGITS"]):
+        """Tests: CTA `cta` (-1: none) withholds its arrival at `stage`."""
+        self._check(self._lib.mono_ffn_debug_skip_arrival(self.handle, cta, stage))
+
+    def debug_jitter(self, max_ns):
+        """Tests: publishing threads sleep hash(CTA, epoch, point) % max_ns first."""
+        self._check(self._lib.mono_ffn_debug_jitter(self.handle, max_ns))
 
     def info(self):
         inf = Info()
@@ -186,8 +195,28 @@ def route_noalloc(n, router_w, router_bias, top_k, route_scale, denom_clamp, idx
     router_bias [n_routed] fp32, idx [rows][top_k] int32 and w [rows][top_k]
     fp32 written in place; all CUDA tensors on the current device."""
     import torch
+    if n.dim() != 2 or router_w.dim() != 2 or router_bias.dim() != 1:
+        raise ValueError("route_noalloc: n [rows][hidden], router_w [hidden][n_routed], router_bias [n_routed]")
     rows, hidden = n.shape
     n_routed = router_w.shape[1]
+    why = []
+    if n.dtype not in (torch.bfloat16, torch.float32):
+        why.append("n must be bf16 or fp32")
+    if router_w.dtype != torch.float32 or router_bias.dtype != torch.float32 or w.dtype != torch.float32:
+        why.append("router_w, router_bias and w must be fp32")
+    if idx.dtype != torch.int32:
+        why.append("idx must be int32")
+    if router_w.shape[0] != hidden or router_bias.numel() != n_routed:
+        why.append("router_w must be [hidden][n_routed] and router_bias [n_routed]")
+    if tuple(idx.shape) != (rows, top_k) or tuple(w.shape) != (rows, top_k):
+        why.append("idx and w must be [rows][top_k]")
+    ts = (n, router_w, router_bias, idx, w)
+    if not all(t.is_contiguous() for t in ts):
+        why.append("every tensor must be contiguous")
+    if not all(t.is_cuda for t in ts) or any(t.device.index != torch.cuda.current_device() for t in ts):
+        why.append("every tensor must be on the current CUDA device")
+    if why:
+        raise ValueError("route_noalloc: " + "; ".join(why))
     rc = lib().mono_ffn_route_noalloc(rows, hidden, n_routed, top_k, _ptr(n), 1 if n.dtype == torch.bfloat16 else 0,
                                       _ptr(router_w), _ptr(router_bias), route_scale, denom_clamp, _ptr(idx), _ptr(w),
                                       _stream(stream))

@@ -452,8 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
   // publish this CTA's activations, then wait for everyone's
   bar_sync(kBarCons, kCW * 32);
   if (ctid == 0) {
-    __threadfence();
-    red_release_add(&p.sync->cnt_act, 1u);
+    if (may_publish(p, c->epoch, 4, 4)) {
+      __threadfence();
+      red_release_add(&p.sync->cnt_act, 1u);
+    }
     wait_count(p, c, &p.sync->cnt_act, ep1 * (uint32_t)G, 4u);
   }
   int h0, h1;

@@ -109,7 +109,9 @@ struct Params {
   Taps taps;
   int nst, slot_bytes, regA_bytes, ymax;
   unsigned long long timeout_ns;
-  int fault_cta;
+  int fault_cta;      // tests: this CTA withholds its arrival at fault_stage (-1: none)
+  int fault_stage;    // MONO_STAGE_* of the withheld arrival
+  unsigned jitter_ns; // tests: every publishing thread first sleeps up to this long (0: off)
   unsigned long long* trace;   // optional [G][kTracePoints] globaltimer stamps
 };
 
@@ -117,6 +119,22 @@ constexpr int kTracePoints = 32;
 // stage timestamps (one writer per point and CTA)
 __device__ __forceinline__ void trace(const Params& p, int point, bool who = true) {
   if (p.trace && who) p.trace[blockIdx.x * kTracePoints + point] = globaltimer();
+}
+
+// Before a grid-visible arrival (a counter other CTAs wait on) at `stage`:
+// in the race-detection mode the publishing thread first sleeps a pseudo-
+// random time hash(CTA, epoch, point) % jitter_ns, so that arrival orders
+// change from step to step; returns false when this CTA is the one told to
+// withhold its arrival at this stage (fault injection of the tests).
+__device__ __forceinline__ bool may_publish(const Params& p, uint32_t epoch, int stage, uint32_t point) {
+  if (p.jitter_ns) {
+    uint32_t h = blockIdx.x * 0x9E3779B1u ^ (epoch + 0x7F4A7C15u) * 0x85EBCA77u ^ point * 0xC2B2AE3Du;
+    h ^= h >> 15;
+    h *= 0x2C1B3C6Du;
+    h ^= h >> 12;
+    __nanosleep(h % p.jitter_ns);
+  }
+  return !((int)blockIdx.x == p.fault_cta && stage == p.fault_stage);
 }
 
 // per-CTA control block in shared memory
@@ -586,7 +604,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       p.mix_part[(size_t)o * G + blockIdx.x] = acc;
     }
     bar_sync(kBarPre, kPreThreads);
-    if (ptid == 0) {
+    if (ptid == 0 && may_publish(p, c->epoch, 1, 0)) {
       __threadfence();
       red_release_add(&p.sync->cnt_mix, 1u);
     }
@@ -796,7 +814,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
       p.sq_part[(size_t)ctid * G + blockIdx.x] = t;
     }
     bar_sync(kBarCons, kCW * 32);
-    if (ctid == 0) {
+    if (ctid == 0 && may_publish(p, c->epoch, 7, 1)) {
       __threadfence();
       red_release_add(&p.sync->cnt_a, 1u);
     }
@@ -936,7 +954,7 @@ __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_
     bar_sync(kBarCons, kCW * 32);
   }
   if (dry) return;
-  if (ctid == 0 && (int)blockIdx.x != p.fault_cta) {
+  if (ctid == 0 && may_publish(p, c->epoch, 2, 2)) {
     __threadfence();
     red_release_add(&p.sync->cnt_logit, 1u);
   }
@@ -999,6 +1017,7 @@ __device__ void tail(const Params& p, Ctl* c, YF yfun) {
 // layer's epoch.  Compute thread 0.
 __device__ __forceinline__ void finish_step(const Params& p, Ctl* c, uint32_t ep1) {
   if (threadIdx.x == 0 && !c->dead) {
+    may_publish(p, c->epoch, 0, 3);
     __threadfence();
     const uint32_t old = atomicAdd(&p.sync->cnt_done, 1u);
     if (old == ep1 * (uint32_t)p.G - 1u) {

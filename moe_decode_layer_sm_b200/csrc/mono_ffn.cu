@@ -65,6 +65,8 @@ struct mono_ffn_plan_s {
   void* stage_out = nullptr;
   int64_t packed_bytes = 0, scratch_bytes = 0;
   int fault_cta = -1;
+  int fault_stage = 0;
+  unsigned jitter_ns = 0;
   unsigned long long* trace = nullptr;
   std::string last_error;
 };
@@ -279,7 +281,7 @@ int dalloc(mono_ffn_plan_t* p, T** ptr, size_t bytes, int64_t* acct) {
 
 // ================================================================ the C ABI
 
-extern "C" int mono_ffn_abi_version(void) { return 1; }
+extern "C" int mono_ffn_abi_version(void) { return 2; }
 
 extern "C" const char* mono_ffn_last_error(const mono_ffn_plan_t* plan) {
   return plan ? plan->last_error.c_str() : g_plan_error.c_str();
@@ -735,6 +737,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.ymax = p->ymax;
     prm.timeout_ns = (unsigned long long)p->cfg.wait_timeout_us * 1000ull;
     prm.fault_cta = p->fault_cta;
+    prm.fault_stage = p->fault_cta >= 0 ? p->fault_stage : 0;
+    prm.jitter_ns = p->jitter_ns;
     prm.trace = p->trace ? p->trace + (size_t)l * p->G * kTracePoints : nullptr;
 
     cudaLaunchConfig_t lc{};
@@ -836,9 +840,29 @@ extern "C" int mono_ffn_set_trace(mono_ffn_plan_t* p, unsigned long long* buf) {
   return MONO_OK;
 }
 
-extern "C" int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* p, int cta) {
-  if (!p) return MONO_ERR_INVALID_ARG;
+extern "C" int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* p, int cta, int stage) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "debug_skip_arrival: NULL plan");
+  if (cta < 0) {
+    p->fault_cta = -1;
+    p->fault_stage = 0;
+    return MONO_OK;
+  }
+  const bool known = stage == MONO_STAGE_MIX || stage == MONO_STAGE_LOGITS || stage == MONO_STAGE_ACT ||
+                     stage == MONO_STAGE_Y || stage == MONO_STAGE_COLLAPSE;
+  if (!known || cta >= p->G)
+    return fail(p, MONO_ERR_INVALID_ARG, "debug_skip_arrival: cta must be < grid and stage one of MIX, LOGITS, "
+                                         "ACT, Y, COLLAPSE");
+  if (stage == MONO_STAGE_Y && !(p->tc || p->tq))
+    return fail(p, MONO_ERR_INVALID_ARG, "debug_skip_arrival: the CUDA-core kernel has no Y stage");
   p->fault_cta = cta;
+  p->fault_stage = stage;
+  return MONO_OK;
+}
+
+extern "C" int mono_ffn_debug_jitter(mono_ffn_plan_t* p, unsigned max_ns) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "debug_jitter: NULL plan");
+  if (max_ns > 100000u) return fail(p, MONO_ERR_INVALID_ARG, "debug_jitter: max_ns above 100000");
+  p->jitter_ns = max_ns;
   return MONO_OK;
 }
 

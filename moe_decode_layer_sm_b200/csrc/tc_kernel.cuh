@@ -181,6 +181,7 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
     uint32_t* cnt = (gu ? p.gcnt : p.dcnt) + (size_t)sg.x * (gu ? geo.nbi : geo.nbh) + sg.blk;
     int parts = 0;
     for (int cc = c_lo; cc <= c_hi; ++cc) parts += holds(cc) ? 1 : 0;
+    if (live) may_publish(p, c->epoch, 0, 5 + (uint32_t)sg.list);
     const uint32_t old = live ? atomicAdd(cnt, 1u) : 0u;
     const bool last = live && old == (uint32_t)(parts - 1);
     if (last) atomicExch(cnt, 0u);   // ready for the next step
@@ -258,7 +259,9 @@ __device__ __forceinline__ void epi_store(const Params& p, Ctl* c, const TcGeo& 
     // read by bulk copies, the async proxy)
     __threadfence();
     bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
-    if (tid == 0 && live) {
+    // (fault injection at the activation stage: the arrival of the shared
+    // expert's first block is withheld, whichever CTA completes it)
+    if (tid == 0 && live && may_publish(p, c->epoch, 0, 8) && !(p.fault_stage == 4 && x == 0 && sg.blk == 0)) {
       fence_proxy_async_global();
       red_release_add(&p.xready[x], 1u);
     }
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     tc_segments(p, geo, L_DN, nu, seg);
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
-    if (tid == 0) {
+    if (tid == 0 && may_publish(p, c->epoch, 6, 9)) {
       __threadfence();
       red_release_add(&p.sync->cnt_y, 1u);
     }

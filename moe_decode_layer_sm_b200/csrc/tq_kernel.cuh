@@ -268,7 +268,7 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
   // read by a bulk copy, the async proxy; the scales by the epilogues)
   __threadfence();
   bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
-  if (tid == 0 && live) {
+  if (tid == 0 && live && may_publish(p, c->epoch, 0, 8) && !(p.fault_stage == 4 && x == 0 && sg.blk == 0)) {
     fence_proxy_async_global();
     red_release_add(&p.xready[x], 1u);
   }
@@ -635,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     tc_segments(p, geo, L_DN, nu, seg);
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
-    if (tid == 0) {
+    if (tid == 0 && may_publish(p, c->epoch, 6, 9)) {
       __threadfence();
       red_release_add(&p.sync->cnt_y, 1u);
     }

@@ -4,6 +4,7 @@ leg are the only callers; the product path never imports this module.
 """
 
 import ctypes
+import hashlib
 import os
 import subprocess
 
@@ -19,9 +20,22 @@ _DT = {"f32": F32, "bf16": BF16, "fp8": FP8, "mxfp4": MXFP4}
 
 
 def build():
-    if (not os.path.exists(SO) or os.path.getmtime(SO) < max(os.path.getmtime(SRC), os.path.getmtime(HDR))):
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared", "-o", SO,
-                               SRC, "-lm"])
+    """Compile the oracle unless its stamp file records the SHA-256 of the
+    sources and the compile command."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared", "-o", SO, SRC, "-lm"]
+    h = hashlib.sha256()
+    for s in (SRC, HDR):
+        with open(s, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(cmd).encode())
+    stamp = SO + ".sha256"
+    if os.path.exists(SO) and os.path.exists(stamp) and open(stamp).read().strip() == h.hexdigest():
+        return
+    if os.path.exists(stamp):
+        os.unlink(stamp)
+    subprocess.check_call(cmd)
+    with open(stamp, "w") as f:
+        f.write(h.hexdigest() + "\n")
 
 
 class Cfg(ctypes.Structure):

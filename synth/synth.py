@@ -8,6 +8,7 @@ Nothing here computes any step of the layer.
 """
 
 import ctypes
+import hashlib
 import math
 import os
 import subprocess
@@ -25,24 +26,33 @@ _OUT = {"f32": 0, "bf16": 1, "f64": 2}
 
 
 def build(gpu=True):
-    """Compile the generator (CPU with gcc; device with nvcc for sm_100a)."""
+    """Compile the generator (CPU with gcc; device with nvcc for sm_100a).
+    Each library is rebuilt unless its stamp file records the SHA-256 of its
+    sources and compile command."""
     src = os.path.join(HERE, "synth_cpu.c")
-    if _stale(CPU_SO, [src, os.path.join(HERE, "synth_core.h")]):
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
-                               "-o", CPU_SO, src, "-lm"])
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared", "-o", CPU_SO, src, "-lm"]
+    _build_stamped(CPU_SO, [src, os.path.join(HERE, "synth_core.h")], cmd)
     if gpu:
         src = os.path.join(HERE, "synth_gpu.cu")
-        if _stale(GPU_SO, [src, os.path.join(HERE, "synth_core.h")]):
-            subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
-                                   "-fmad=false", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-                                   "-o", GPU_SO, src])
+        cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-fmad=false", "-std=c++17",
+               "-Xcompiler", "-fPIC", "-shared", "-o", GPU_SO, src]
+        _build_stamped(GPU_SO, [src, os.path.join(HERE, "synth_core.h")], cmd)
 
 
-def _stale(out, srcs):
-    if not os.path.exists(out):
-        return True
-    t = os.path.getmtime(out)
-    return any(os.path.getmtime(s) > t for s in srcs)
+def _build_stamped(out, srcs, cmd):
+    h = hashlib.sha256()
+    for s in srcs:
+        with open(s, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(cmd).encode())
+    stamp = out + ".sha256"
+    if os.path.exists(out) and os.path.exists(stamp) and open(stamp).read().strip() == h.hexdigest():
+        return
+    if os.path.exists(stamp):
+        os.unlink(stamp)
+    subprocess.check_call(cmd)
+    with open(stamp, "w") as f:
+        f.write(h.hexdigest() + "\n")
 
 
 _cpu = None

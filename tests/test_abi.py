@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     missing = [n for n in names if not hasattr(L, n)]
     assert not missing, missing
     assert set(names) == set(binding.SYMBOLS)
-    assert L.mono_ffn_abi_version() == 1
+    assert L.mono_ffn_abi_version() == 2
     assert __graft_entry__.ROOT == ROOT
 
 
@@ -41,3 +41,19 @@ def test_plan_refusal_lists_every_reason_without_a_gpu():
     msg = L.mono_ffn_last_error(None).decode()
     for frag in ("hc must be 4", "n_routed", "top_k", "max_rows", "n_layers", "hc_dtype"):
         assert frag in msg, (frag, msg)
+
+
+def test_build_is_keyed_on_the_source_hash(tmp_path, monkeypatch):
+    """build() trusts the library only when the stamp beside it holds the
+    hash of the current sources and nvcc command; a later modification time
+    alone does not count."""
+    from moe_decode_layer_sm_b200 import build as b
+    b.build()
+    assert b.up_to_date()
+    stamp = tmp_path / "stamp"
+    stamp.write_text("0" * 64 + "\n")
+    monkeypatch.setattr(b, "STAMP", str(stamp))
+    os.utime(b.SO, None)   # the binary is newer than every source
+    assert not b.up_to_date()
+    stamp.write_text(b.source_hash() + "\n")
+    assert b.up_to_date()

@@ -1,8 +1,9 @@
 """Parity at the full sizes of the five target configurations, in the launch
 configuration the benchmark times (one persistent CTA per SM).  The device
-runs every row; the oracle recomputes sampled rows completely (rows are
-independent, so a sampled row's output is exact to check), and the routing
-of every row."""
+runs every row and the oracle recomputes every row (rows are independent;
+the oracle generates only the experts the rows touch).  The chain is
+checked layer by layer on the residual streams the kernel materialised,
+every row, and end to end in relative L2."""
 
 import numpy as np
 import pytest
@@ -10,7 +11,8 @@ import pytest
 from oracle import oracle as O
 from synth import configs as C
 from synth import synth as S
-from tests.gpu_harness import LayerRun, compare_out, routing_ok
+from tests.gpu_harness import (LayerRun, check_chain_layer, check_logits, compare_out, compare_rel_l2, raw_hc,
+                               routing_divergence, routing_ok)
 from tests.oracle_helpers import touched_experts
 
 pytestmark = pytest.mark.gpu
@@ -30,68 +32,74 @@ def _free():
     torch.cuda.empty_cache()
 
 
-def _check_rows(wl, run, rows, layer=0, hc_rows=None):
-    """Oracle for `rows` of one layer on hc_rows (host raw [len(rows)][S][H])."""
-    hc = S.cpu_hc_in(wl)[rows] if hc_rows is None else hc_rows
-    w1 = wl.with_(rows=len(rows))
-    dense = S.cpu_dense(wl, layer)
-    ex, _ = touched_experts(w1, dense, hc, layer)
-    out, t = O.layer(w1, O.LayerWeights(w1, dense, ex), hc)
-    exempt = []
-    idx = run.tap(layer, "idx")[rows]
-    for i in range(len(rows)):
-        ok, ex_ = routing_ok(idx[i], t.idx[i], t.sel[i], wl.top_k)
-        assert ok, f"layer {layer} row {rows[i]}: gpu {idx[i]} oracle {t.idx[i]}"
-        if ex_:
-            exempt.append(i)
-    keep = [i for i in range(len(rows)) if i not in exempt]
-    # later chain layers see the kernel's own (bf16-rounded) residual streams
-    tol = 1e-4 if layer == 0 else 2e-2
-    assert np.allclose(run.tap(layer, "mix")[rows], t.mix, rtol=tol, atol=tol)
-    compare_out(wl, run.tap(layer, "n")[rows][keep], t.n[keep], "n")
-    compare_out(wl, run.tap(layer, "y")[rows][keep], t.y[keep], "y")
-    return out, t, keep
-
-
-def _all_rows_routing(wl, run):
-    lw = O.LayerWeights(wl, S.cpu_dense(wl, 0), {})
-    t = O.route(wl, lw, S.cpu_hc_in(wl))
-    gidx = run.tap(0, "idx")
-    for r in range(wl.rows):
-        assert routing_ok(gidx[r], t.idx[r], t.sel[r], wl.top_k)[0], f"row {r}"
-    return t
-
-
-@pytest.mark.parametrize("wl, rows", [(C.FLASH_BF16_R1, [0]), (C.FLASH_BF16_R8, [0, 7]), (C.FLASH_BF16_R6, [2]),
-                                      (C.FLASH_FP8_R4, [0, 3])], ids=lambda x: getattr(x, "name", str(x)))
-def test_full_size_single_layer(wl, rows):
+@pytest.mark.parametrize("wl", [C.FLASH_BF16_R1, C.FLASH_BF16_R6, C.FLASH_BF16_R8, C.FLASH_FP8_R4],
+                         ids=lambda x: x.name)
+def test_full_size_single_layer_all_rows(wl):
     run = LayerRun(wl)
     got = run.step()
-    _all_rows_routing(wl, run)
-    out, t, keep = _check_rows(wl, run, rows)
-    if keep:
-        compare_out(wl, got[rows][keep], O.decode_hc(wl, out)[keep], "hc_out")
+    hc = S.cpu_hc_in(wl)
+    dense = S.cpu_dense(wl, 0)
+    ex, _ = touched_experts(wl, dense, hc, 0)
+    out, t = O.layer(wl, O.LayerWeights(wl, dense, ex), hc)
+    rows = list(range(wl.rows))
+    keep = []
+    idx = run.tap(0, "idx")
+    for r in rows:
+        ok, exempt = routing_ok(idx[r], t.idx[r], t.sel[r], wl.top_k)
+        assert ok, f"row {r}: gpu {idx[r]} oracle {t.idx[r]}"
+        if not exempt:
+            keep.append(r)
+    assert np.allclose(run.tap(0, "mix"), t.mix, rtol=1e-4, atol=1e-4)
+    check_logits(run, 0, t, rows)
+    compare_out(wl, run.tap(0, "n")[keep], t.n[keep], "n")
+    compare_out(wl, run.tap(0, "y")[keep], t.y[keep], "y")
+    compare_out(wl, got[keep], O.decode_hc(wl, out)[keep], "hc_out")
     if wl.rows >= 6:
-        uniq = len(set(run.tap(0, "idx").ravel().tolist()))
+        uniq = len(set(idx.ravel().tolist()))
         assert uniq > 5 * wl.top_k   # rows select mostly disjoint experts
     run.close()
     del run
     _free()
 
 
-def test_full_size_mxfp4_chain_row_sample():
+def test_full_size_mxfp4_chain_all_rows():
+    """Every layer and every row of the 4-layer MXFP4 chain on the kernel's
+    own residual streams, then the chain end to end in relative L2 against
+    the oracle's chain, on the rows where both chains take the same routing
+    decisions in every layer (the others are printed with the cause)."""
     wl = C.FLASH_MXFP4_CHAIN4_R8
     run = LayerRun(wl)
     got = run.step()
-    _all_rows_routing(wl, run)
-    r = [5]
-    x = S.cpu_hc_in(wl)[r]
-    w1 = wl.with_(rows=1)
+    cache = {}
+
+    def experts(dense, x, l):   # the experts the rows of x touch in layer l, generated once
+        t = O.route(wl, O.LayerWeights(wl, dense, {}), x)
+        for e in sorted(set(int(i) for i in t.idx.ravel()) | {wl.n_routed}):
+            if (l, e) not in cache:
+                cache[(l, e)] = S.cpu_expert(wl, l, e)
+        return {e: m for (ll, e), m in cache.items() if ll == l}
+
+    ties = {}
     for l in range(wl.n_layers):
-        out, t, keep = _check_rows(wl, run, r, layer=l, hc_rows=x)
-        x = out
-    compare_out(wl, got[r], O.decode_hc(wl, x), "chain hc_out", layers=wl.n_layers)
-    del w1
+        dense = S.cpu_dense(wl, l)
+        ex = experts(dense, raw_hc(wl, run.tap(l, "x")), l)
+        nxt = run.tap(l + 1, "x") if l + 1 < wl.n_layers else got
+        for r, cause in check_chain_layer(wl, run, l, O.LayerWeights(wl, dense, ex), nxt).items():
+            ties.setdefault(r, cause)
+    # the oracle's own chain from hc_in (its own routing, so its own experts)
+    x, otaps = S.cpu_hc_in(wl), []
+    for l in range(wl.n_layers):
+        dense = S.cpu_dense(wl, l)
+        x, t = O.layer(wl, O.LayerWeights(wl, dense, experts(dense, x, l)), x)
+        otaps.append(t)
+    want = O.decode_hc(wl, x)
+    for r, cause in routing_divergence(wl, run, otaps).items():
+        ties.setdefault(r, cause)
+    keep = [r for r in range(wl.rows) if r not in ties]
+    assert 2 * len(keep) >= wl.rows, f"rows left out: {ties}"
+    for r in keep:
+        compare_rel_l2(got[r], want[r], f"chain hc_out row {r}")
+    print(f"chain end to end: max-abs {np.abs(got[keep] - want[keep]).max():.4e}; rows left out: {ties}")
     run.close()
     del run
     _free()

@@ -1,8 +1,9 @@
 """mono_ffn_route_noalloc (router select with no plan and no allocation)
 against the fused step's own routing: same normed rows n, same router
-weights and bias, two calls in a row.  The file name puts it last in
-collection, so it also runs after every other GPU test (the static scratch's
-arrival counter must still be zero then)."""
+weights and bias, two calls in a row; and at its size limits against a
+float64 restatement of the select.  The file name puts it last in
+collection, so that a run stopping at the first failure has run every other
+test first; it passes alone in a fresh process and after the others."""
 
 import numpy as np
 import pytest
@@ -70,3 +71,51 @@ def test_route_noalloc_refuses_sizes_beyond_its_scratch():
         assert rc == -1
         assert what in L.mono_ffn_last_error(None)
     assert L.mono_ffn_route_noalloc(0, 5120, 256, 8, null, 1, null, null, 2.5, 1e-20, null, null, null) == 0
+
+
+@pytest.mark.gpu
+def test_route_noalloc_at_its_limits_against_float64():
+    """n_routed 1000 (not a multiple of 32: a partial last lane block, 32 keys
+    a lane), top_k 16 and 8 rows, the largest sizes the static scratch takes,
+    against the select restated in float64: logits, sqrt(softplus) scores,
+    canonical (selection desc, index asc) top-k, weights.  The device
+    allocator's free memory is the same before and after the calls."""
+    import torch
+    g = torch.Generator().manual_seed(1000)
+    R, H, E, K = 8, 512, 1000, 16
+    n = torch.randn(R, H, generator=g).to(torch.bfloat16)
+    rw = (torch.randn(H, E, generator=g) / H ** 0.5).float()
+    rb = (torch.rand(E, generator=g) * 0.2 - 0.1).float()
+    lg = n.double() @ rw.double()
+    sc = torch.sqrt(torch.nn.functional.softplus(lg))
+    sel = (sc + rb.double()).numpy()
+    want_idx = np.stack([sorted(range(E), key=lambda e: (-sel[r, e], e))[:K] for r in range(R)])
+    want_w = np.stack([sc[r, want_idx[r]].numpy() / sc[r, want_idx[r]].numpy().sum() * 2.5 for r in range(R)])
+    nd, rwd, rbd = n.cuda(), rw.cuda(), rb.cuda()
+    idx = torch.full((R, K), -1, dtype=torch.int32, device="cuda")
+    w = torch.zeros((R, K), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(2):
+        binding.route_noalloc(nd, rwd, rbd, K, 2.5, 1e-20, idx, w)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+    for r in range(R):
+        ok, exempt = routing_ok(gi[r], want_idx[r], sel[r].astype(np.float32), K)
+        assert ok, f"row {r}: {gi[r]} vs {want_idx[r]}"
+        if not exempt:
+            assert np.allclose(gw[r], want_w[r], rtol=1e-5, atol=1e-6), (gw[r], want_w[r])
+
+
+def test_route_noalloc_binding_checks_its_arguments():
+    """Wrong dtypes or shapes are refused in Python before any pointer goes
+    to the library (no device needed: the checks come first)."""
+    import torch
+    n = torch.zeros(2, 64, dtype=torch.bfloat16)
+    rw = torch.zeros(64, 32)
+    rb = torch.zeros(32)
+    with pytest.raises(ValueError, match="idx must be int32"):
+        binding.route_noalloc(n, rw, rb, 4, 2.5, 1e-20, torch.zeros(2, 4), torch.zeros(2, 4))
+    with pytest.raises(ValueError, match=r"\[rows\]\[top_k\]"):
+        binding.route_noalloc(n, rw, rb, 4, 2.5, 1e-20, torch.zeros(2, 3, dtype=torch.int32), torch.zeros(2, 3))
