@@ -96,6 +96,10 @@ typedef struct {
   unsigned wait_timeout_us; /* bound of every device-side wait; 0 = 250000 */
   int device;       /* CUDA device ordinal */
   int grid;         /* persistent CTAs; 0 = one per SM */
+  int dense;        /* 1: a dense layer: no router; its SwiGLU MLP of width (n_routed + 1) * inter is
+                       the n_routed + 1 slots in slot order, run as expert-shaped slices each taken
+                       with weight 1 (vLLM MonoKernel page, Weights); top_k must equal n_routed, and
+                       router_w / router_bias may be NULL at packing */
 } mono_ffn_config;
 
 /* One layer's weights, device pointers in logical (caller) layouts, read only
@@ -203,6 +207,38 @@ int mono_ffn_pack_weights(mono_ffn_plan_t* plan, int layer, const mono_ffn_layer
  * no-op; rows > max_rows is MONO_ERR_INVALID_ARG.  Allocates nothing and does
  * not synchronise the host. */
 int mono_ffn_step(mono_ffn_plan_t* plan, int rows, const void* hc_in, void* hc_out, void* stream);
+
+/* One step at a fixed launch width with padding rows (vLLM "[ROCm][Perf]
+ * [GLM-5] Fused sparse-layer decode via AITER MonoKernel", when the path
+ * runs: batches are padded to the captured widths and pad rows carry a slot
+ * below zero).  row_slot: device int32 [width]; row r is a padding row when
+ * row_slot[r] < 0: its hc_in is never used (it may hold anything, NaN
+ * included), it selects no expert (no weight bytes are read for it) and its
+ * hc_out is left as it was.  Live rows compute exactly as in mono_ffn_step.
+ * So one width (a CUDA graph captured at 1, 2, 4 or 8 rows) serves every
+ * batch up to it.  width == 0 is a no-op; width > max_rows or overlapping
+ * hc_in / hc_out is MONO_ERR_INVALID_ARG.  Asynchronous; allocates nothing. */
+int mono_ffn_step_padded(mono_ffn_plan_t* plan, int width, const int* row_slot, const void* hc_in, void* hc_out,
+                         void* stream);
+
+/* One step opened by the attention sublayer's pending post / expand (the
+ * within-layer boundary: SGLang "[DeepSeek-V4] Add mhc_fused_post_pre
+ * kernel", Modifications, "attention hc_post + FFN hc_pre" inside one layer):
+ * for each row r the FFN's residual streams are
+ *   X_i = round(sum_j attn_comb[r][i][j] x_attn[r][j] + attn_post[r][i] y_attn[r])
+ * (round = to hc_dtype), materialised in the opening pass together with the
+ * mix products, then the layer (and, with n_layers > 1, the chain) as in
+ * mono_ffn_step.  So a caller hands over exactly what the attention sublayer
+ * leaves pending instead of closing its expand in a kernel of its own.
+ *   x_attn   [rows][S][H] hc_dtype: the residual streams before the attention sublayer
+ *   attn_post [rows][S] fp32, attn_comb [rows][S][S] fp32 (row-major (i, j))
+ *   y_attn   [rows][H] hc_dtype: the attention sublayer's output
+ *   hc_out   [rows][S][H] hc_dtype; must not overlap any input
+ * All device memory on the plan's device, caller-owned.  rows == 0 is a
+ * no-op; rows > max_rows or overlapping buffers are MONO_ERR_INVALID_ARG.
+ * Asynchronous; allocates nothing. */
+int mono_ffn_step_pending(mono_ffn_plan_t* plan, int rows, const void* x_attn, const float* attn_post,
+                          const float* attn_comb, const void* y_attn, void* hc_out, void* stream);
 
 /* The same step with HOST buffers: copies hc_in (pinned or pageable host
  * memory) to the plan's device staging buffer, runs the step, copies the

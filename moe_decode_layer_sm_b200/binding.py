@@ -23,7 +23,7 @@ ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED_ARCH", -3: "NOT_CORESIDEN
 SYMBOLS = ["mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
            "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_last_error",
            "mono_ffn_destroy", "mono_ffn_abi_version", "mono_ffn_set_trace", "mono_ffn_route_noalloc",
-           "mono_ffn_debug_jitter"]
+           "mono_ffn_debug_jitter", "mono_ffn_step_pending", "mono_ffn_step_padded"]
 
 
 class Config(ctypes.Structure):
@@ -31,7 +31,7 @@ class Config(ctypes.Structure):
                                             "hc_dtype", "norm_dtype", "expert_dtype", "round_bf16")] + \
                [(n, ctypes.c_float) for n in ("rms_eps", "pre_eps", "post_mult", "route_scale", "denom_clamp")] + \
                [("sinkhorn_iters", ctypes.c_int), ("wait_timeout_us", ctypes.c_uint), ("device", ctypes.c_int),
-                ("grid", ctypes.c_int)]
+                ("grid", ctypes.c_int), ("dense", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -72,6 +72,8 @@ def lib():
         L.mono_ffn_pack_weights.argtypes = [vp, i32, ctypes.POINTER(LayerWeights), vp]
         L.mono_ffn_step.argtypes = [vp, i32, vp, vp, vp]
         L.mono_ffn_step_host.argtypes = [vp, i32, vp, vp, vp]
+        L.mono_ffn_step_pending.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp]
+        L.mono_ffn_step_padded.argtypes = [vp, i32, vp, vp, vp, vp]
         L.mono_ffn_set_taps.argtypes = [vp, i32, ctypes.POINTER(TapsStruct)]
         L.mono_ffn_query_error.argtypes = [vp, ctypes.POINTER(Status)]
         L.mono_ffn_get_info.argtypes = [vp, ctypes.POINTER(Info)]
@@ -86,7 +88,8 @@ def lib():
         L.mono_ffn_route_noalloc.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, f32, f32, vp, vp, vp]
         for f in ("mono_ffn_plan", "mono_ffn_pack_weights", "mono_ffn_step", "mono_ffn_step_host", "mono_ffn_set_taps",
                   "mono_ffn_query_error", "mono_ffn_get_info", "mono_ffn_debug_skip_arrival", "mono_ffn_abi_version",
-                  "mono_ffn_set_trace", "mono_ffn_route_noalloc", "mono_ffn_debug_jitter"):
+                  "mono_ffn_set_trace", "mono_ffn_route_noalloc", "mono_ffn_debug_jitter", "mono_ffn_step_pending",
+                  "mono_ffn_step_padded"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -107,13 +110,14 @@ class Plan:
 
     def __init__(self, hidden, n_routed, top_k, inter, max_rows, n_layers=1, hc_dtype="bf16", norm_dtype="bf16",
                  expert_dtype="bf16", round_bf16=True, rms_eps=1e-6, pre_eps=1e-6, post_mult=2.0, route_scale=2.5,
-                 denom_clamp=1e-20, sinkhorn_iters=20, wait_timeout_us=0, device=0, grid=0):
+                 denom_clamp=1e-20, sinkhorn_iters=20, wait_timeout_us=0, device=0, grid=0, dense=False):
         self._lib = lib()
         self.cfg = Config(hidden=hidden, hc=4, n_routed=n_routed, top_k=top_k, inter=inter, max_rows=max_rows,
                           n_layers=n_layers, hc_dtype=DTYPE[hc_dtype], norm_dtype=DTYPE[norm_dtype],
                           expert_dtype=DTYPE[expert_dtype], round_bf16=int(round_bf16), rms_eps=rms_eps,
                           pre_eps=pre_eps, post_mult=post_mult, route_scale=route_scale, denom_clamp=denom_clamp,
-                          sinkhorn_iters=sinkhorn_iters, wait_timeout_us=wait_timeout_us, device=device, grid=grid)
+                          sinkhorn_iters=sinkhorn_iters, wait_timeout_us=wait_timeout_us, device=device, grid=grid,
+                          dense=int(dense))
         h = ctypes.c_void_p()
         rc = self._lib.mono_ffn_plan(ctypes.byref(self.cfg), ctypes.byref(h))
         if rc != 0:
@@ -126,7 +130,8 @@ class Plan:
         return cls(wl.hidden, wl.n_routed, wl.top_k, wl.inter, max_rows=wl.rows, n_layers=wl.n_layers,
                    hc_dtype=wl.hc_dtype, norm_dtype=wl.norm_dtype, expert_dtype=wl.w_dtype,
                    round_bf16=wl.round_bf16, rms_eps=wl.rms_eps, pre_eps=wl.pre_eps, post_mult=wl.post_mult,
-                   route_scale=wl.route_scale, denom_clamp=wl.denom_clamp, sinkhorn_iters=wl.sinkhorn_iters, **kw)
+                   route_scale=wl.route_scale, denom_clamp=wl.denom_clamp, sinkhorn_iters=wl.sinkhorn_iters,
+                   dense=getattr(wl, "dense", False), **kw)
 
     def _check(self, rc):
         if rc != 0:
@@ -140,6 +145,19 @@ class Plan:
 
     def step(self, rows, hc_in, hc_out, stream=None):
         self._check(self._lib.mono_ffn_step(self.handle, rows, _ptr(hc_in), _ptr(hc_out), _stream(stream)))
+
+    def step_padded(self, width, row_slot, hc_in, hc_out, stream=None):
+        """A step at a fixed width: row_slot int32 [width] CUDA tensor, rows
+        with a slot below zero are padding (input ignored, output untouched)."""
+        self._check(self._lib.mono_ffn_step_padded(self.handle, width, _ptr(row_slot), _ptr(hc_in), _ptr(hc_out),
+                                                   _stream(stream)))
+
+    def step_pending(self, rows, x_attn, attn_post, attn_comb, y_attn, hc_out, stream=None):
+        """A step opened by the attention sublayer's pending expand: x_attn
+        [rows][4][H] and y_attn [rows][H] in the hc dtype, attn_post [rows][4]
+        and attn_comb [rows][4][4] fp32, all CUDA tensors."""
+        self._check(self._lib.mono_ffn_step_pending(self.handle, rows, _ptr(x_attn), _ptr(attn_post), _ptr(attn_comb),
+                                                    _ptr(y_attn), _ptr(hc_out), _stream(stream)))
 
     def step_host(self, rows, hc_in, hc_out, stream=None):
         """hc_in / hc_out are CPU tensors (pinned for asynchronous copies)."""

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
     c->lists_ready = 0;
     c->nu = 0;
     c->epoch = ld_relaxed(&p.sync->epoch);
+    c->live = live_rows(p);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);

@@ -17,6 +17,8 @@
 // raises the abort flag and runs the rest of its control flow without waiting
 // (so every named barrier is still reached), then returns.
 #pragma once
+#include <cuda.h>
+
 #include <type_traits>
 
 #include "ptx.cuh"
@@ -41,7 +43,6 @@ constexpr int kPreThreads = (kCW + kCtlWarps) * 32;    // compute + control
 // warps 0-3, routing hand-over (compute + control), end (epilogue warps + the
 // issuer warp)
 constexpr int kBarPre = 1, kBarCons = 2, kBarCtl = 3, kBarEpi = 4, kBarRoute = 5, kBarEnd = 6, kBarTop = 7;
-constexpr int kMaxAb = 6;          // A-tile buffers of the quantised tensor-core kernels
 constexpr int kMaxAcc = 4;         // accumulator buffers in tensor memory
 constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core tile may read past its stage
 
@@ -63,15 +64,20 @@ struct Taps {
 struct Params {
   int H, I, E, K, R, G;
   int layer, first, last;
+  int dense;            // no router: every slot is a slice of one dense MLP, weight 1
   int mix_ctas;
   int hc_bf16, norm_bf16, round_bf16;
   float rms_eps, pre_eps, post_mult, route_scale, denom_clamp;
   int sink_iters;
   // residual streams
-  const void* x_prev;   // first: this layer's X (hc_in); else the previous layer's X
+  const void* x_prev;   // first: this layer's X (hc_in); else the residual streams before the
+                        // pending expand (the previous layer's X, or the attention sublayer's input)
   void* xbuf;           // this layer's X when not first (written by the mix CTAs)
   void* hc_out;         // written when last
-  const float* pend_in; // previous layer's pending post [R][4] | comb [R][16] | y [R][H]
+  const float* pend_post; // the pending expand (not first): post [R][4] and comb [R][16] fp32,
+  const float* pend_comb; // and y [R][H] (fp32, or bf16 when pend_y_bf16), of the previous layer
+  const void* pend_y;     // or of the attention sublayer
+  int pend_y_bf16;
   float* pend_out;      // this layer's pending state (when not last)
   // packed weights
   const float* mix_w;
@@ -96,8 +102,12 @@ struct Params {
   float* sq_part;    // [R][G] per-CTA partial sums of a^2
   float* yp;         // tensor-core kernel: [R][K+1][H] weighted expert outputs
   uint32_t* xready;  // tensor-core kernel: [R*K+1] finished gate/up blocks per expert entry (0 between steps)
-  const float* gsc;  // tensor-core FP8 kernel: [E+1][I/128][H/128][gate 128 | up 128] fp32 block scales
-  const float* dsc;  // tensor-core FP8 kernel: [E+1][H/128][I/128][128] fp32 block scales
+  const float* gsc;  // tensor-core FP8 kernel: [E+1][I/128][H/128][gate 128 | up 128] fp32 block scales;
+                     // MXFP4: [E+1][I/128][H/128][gate | up] 512-byte e8m0 scale chunks
+  const float* dsc;  // tensor-core FP8 kernel: [E+1][H/128][I/128][128] fp32 block scales;
+                     // MXFP4: [E+1][H/128][I/128] 512-byte e8m0 scale chunks
+  CUtensorMap tm_gu; // MXFP4 tensor-core kernel: 2-D maps of the packed gate/up and down codes,
+  CUtensorMap tm_dn; // rows of 128 e2m1 codes, unpacked into 16-byte slots, 128-byte swizzle
   int n_xready;
   uint8_t* actb;     // tensor-core kernel: [R*K+1][I/8][16][8] bf16 down-projection B operands
   float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks
@@ -109,6 +119,7 @@ struct Params {
   Taps taps;
   int nst, slot_bytes, regA_bytes, ymax;
   unsigned long long timeout_ns;
+  const int* row_slot;  // [R] int32: row r is padding when row_slot[r] < 0 (NULL: every row live)
   int fault_cta;      // tests: this CTA withholds its arrival at fault_stage (-1: none)
   int fault_stage;    // MONO_STAGE_* of the withheld arrival
   unsigned jitter_ns; // tests: every publishing thread first sleeps up to this long (0: off)
@@ -142,6 +153,7 @@ struct Ctl {
   volatile int dead;
   volatile int lists_ready;
   uint32_t epoch;
+  uint32_t live;                // bit r: row r is a live row (not padding)
   volatile int nu;              // unique routed experts (control warps' copy)
   int nu_comp;                  // the compute warps' agreed copy
   float smix[kMaxR][kMixP];     // mix partial totals, then the scaled mix
@@ -162,7 +174,6 @@ struct Ctl {
   volatile int n_ready;         // n is in shared memory (B operand of gate/up)
   uint64_t accfull[kMaxAcc], accempty[kMaxAcc], drain;
   uint64_t bfull;               // the down projection's B operand has landed
-  uint64_t abfull[kMaxAb], abempty[kMaxAb];   // quantised tensor-core kernel: converted A tiles in tensor memory
   volatile int bcast;           // epilogue: "this CTA completes the block"
   // FP8 tensor-core kernel: inverse power-of-two scale of each row of n, and
   // the epilogue warps' per-row maxima of a block's activations
@@ -184,6 +195,15 @@ struct SmemLayout {
     total = ring + (size_t)nst * slot_bytes + kRingGuard;
   }
 };
+
+// Rows of the launch that are live (bit r), from the optional row slots: a
+// padding row (slot < 0) reads as zero, selects no expert and writes nothing.
+__device__ __forceinline__ uint32_t live_rows(const Params& p) {
+  uint32_t m = 0u;
+  for (int r = 0; r < p.R; ++r)
+    if (!p.row_slot || __ldg(p.row_slot + r) >= 0) m |= 1u << r;
+  return m;
+}
 
 // ------------------------------------------------------------ bounded waits --
 
@@ -462,6 +482,21 @@ __device__ __noinline__ void topk_row(const Params& p, Ctl* c, int r, bool dry) 
   __syncwarp();
 }
 
+// A dense layer's "routing" of row r (one warp): every routed slot, in slot
+// order, with weight 1 (the shared slot joins as always).
+__device__ __forceinline__ void dense_row(const Params& p, Ctl* c, int r) {
+  const int lane = threadIdx.x & 31;
+  if (lane < p.K) {
+    c->idx[r][lane] = lane;
+    c->wt[r][lane] = 1.0f;
+    if (blockIdx.x == 0) {
+      if (p.taps.idx) p.taps.idx[r * p.K + lane] = lane;
+      if (p.taps.w) p.taps.w[r * p.K + lane] = 1.0f;
+    }
+  }
+  __syncwarp();
+}
+
 // the top-k of row r with the lane layout that fits E
 __device__ __forceinline__ void topk_dispatch(const Params& p, Ctl* c, int r, bool dry) {
   const int E = p.E;
@@ -544,9 +579,8 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       cp_async16(reinterpret_cast<float4*>(ws) + i, reinterpret_cast<const float4*>(p.mix_w + ((size_t)sgm * H + h0) * kMixC) + j);
     }
     cp_async_commit();
-    const float* ppost = p.pend_in;
-    const float* pcomb = p.pend_in + R * kS;
-    const float* py = p.pend_in + R * kS + R * kS * kS;
+    const float* ppost = p.pend_post;
+    const float* pcomb = p.pend_comb;
     const int nx = R * kS * nh;
     constexpr int kXU = 4;   // elements per thread in flight
     for (int i0 = ptid; i0 < nx; i0 += kXU * kPreThreads) {
@@ -557,7 +591,9 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
         v[u] = 0.f;
         if (i < nx) {
           const int r = i / (kS * nh), sg = (i / nh) % kS, h = h0 + i % nh;
-          if (p.first) {
+          if (!((c->live >> r) & 1u)) {
+            v[u] = 0.f;   // padding row: its input is ignored
+          } else if (p.first) {
             v[u] = load_x(p.x_prev, ((size_t)r * kS + sg) * H + h, p.hc_bf16);
           } else {
             // the previous layer's deferred post: X_s = sum_j comb_sj Xprev_j + post_s y
@@ -565,7 +601,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
 #pragma unroll
             for (int j = 0; j < kS; ++j)
               acc = fmaf(pcomb[(r * kS + sg) * kS + j], load_x(p.x_prev, ((size_t)r * kS + j) * H + h, p.hc_bf16), acc);
-            acc = fmaf(ppost[r * kS + sg], py[(size_t)r * H + h], acc);
+            acc = fmaf(ppost[r * kS + sg], load_x(p.pend_y, (size_t)r * H + h, p.pend_y_bf16), acc);
             v[u] = p.hc_bf16 ? round_bf16(acc) : acc;
           }
         }
@@ -699,10 +735,13 @@ __device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint
   }
   if (ctl_topk) {
     // the top-k rows here, two warps over the rows
-    if (ct == 0) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
+    if (ct == 0 && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
     trace(p, 21, ct == 0);
     bar_sync(kBarCtl, kCtlWarps * 32);
-    for (int r = cw; r < R; r += kCtlWarps) topk_dispatch(p, c, r, false);
+    for (int r = cw; r < R; r += kCtlWarps) {
+      if (p.dense) dense_row(p, c, r);
+      else topk_dispatch(p, c, r, false);
+    }
     for (int i = ct; i < kMaxE / 32; i += kCtlWarps * 32) c->bm[i] = 0u;
     bar_sync(kBarCtl, kCtlWarps * 32);
     trace(p, 22, ct == 0);
@@ -720,7 +759,7 @@ __device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint
   }
   for (int i = ct; i < R * K; i += kCtlWarps * 32) {
     const int e = c->idx[i / K][i % K];
-    if (e >= 0 && e < E) atomicOr(&c->bm[e >> 5], 1u << (e & 31));
+    if (e >= 0 && e < E && ((c->live >> (i / K)) & 1u)) atomicOr(&c->bm[e >> 5], 1u << (e & 31));
   }
   bar_sync(kBarCtl, kCtlWarps * 32);
   if (cw == 0) {
@@ -748,7 +787,7 @@ __device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint
     uint32_t mask = 0u;
     for (int r = 0; r < kMaxR; ++r) {
       signed char sl = -1;
-      if (r < R)
+      if (r < R && ((c->live >> r) & 1u))
         for (int j = 0; j < K; ++j)
           if (c->idx[r][j] == e) sl = (signed char)j;
       c->uslot[u][r] = sl;
@@ -901,6 +940,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
 // both calls share the code).
 template <bool CANON>
 __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_t* n_s, bool dry) {
+  if (p.dense) return;   // no router (and no logits stage) in a dense layer
   const int R = p.R, H = p.H, E = p.E, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
   const bool nbf = CANON || p.round_bf16;
   const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
@@ -969,11 +1009,14 @@ __device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1, bool split) {
   const int R = p.R, warp = threadIdx.x >> 5;
   const int w0 = split ? 4 : 0, nw = kCW - w0;
   const bool lead = (int)threadIdx.x == w0 * 32;
-  if (lead) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
+  if (lead && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
   if (split) bar_sync(kBarTop, 4 * 32);
   else bar_sync(kBarCons, kCW * 32);
   trace(p, 21, lead);
-  for (int r = warp - w0; r < R; r += nw) topk_dispatch(p, c, r, false);
+  for (int r = warp - w0; r < R; r += nw) {
+    if (p.dense) dense_row(p, c, r);
+    else topk_dispatch(p, c, r, false);
+  }
   trace(p, 22, lead);
   bar_sync(kBarRoute, (nw + kCtlWarps) * 32);
 }
@@ -991,6 +1034,7 @@ __device__ void tail(const Params& p, Ctl* c, YF yfun) {
   float* pend_y = p.pend_out + R * kS + R * kS * kS;
   for (int i = ctid; i < R * nh; i += kCW * 32) {
     const int r = i / nh, h = h0 + i % nh;
+    if (!((c->live >> r) & 1u)) continue;   // padding row: its output is left as it is
     // all loads (the residual streams and the expert outputs) before any store
     float xv[kS];
 #pragma unroll

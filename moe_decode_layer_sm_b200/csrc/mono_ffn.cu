@@ -1,6 +1,8 @@
 // Host side of libmonoffn: the C ABI declared in include/mono_ffn.h — plan
 // validation and allocation, the one-time weight repack, the per-step
 // launches and the device error word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -27,8 +29,9 @@ struct LayerSlot {
   float* bias = nullptr;
   uint8_t* gu = nullptr;
   uint8_t* dn = nullptr;
-  float* gsc = nullptr;   // quantised tensor-core path, FP8: packed block scales
+  float* gsc = nullptr;   // quantised tensor-core path: packed block scales (FP8 fp32, MXFP4 e8m0 chunks)
   float* dsc = nullptr;
+  CUtensorMap tm_gu{}, tm_dn{};   // MXFP4: tensor maps of the packed codes
   bool packed = false;
   Taps taps{};
 };
@@ -142,45 +145,16 @@ __global__ void pack_tc_kernel(const uint16_t* src, uint8_t* dst, long long e1, 
 // j of unit-row i at j * 2048 + i * 16 inside the unit's matrix slot msub:
 //   dst[((e * rows/128 + row/128) * nu + u) * ustride + msub + j * 2048 + (row % 128) * 16]
 __global__ void pack_tq_codes_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int row_bytes, int ub,
-                                     long long ustride, int msub, int f4) {
+                                     long long ustride, int msub) {
   const int nch = row_bytes / 16, nu = row_bytes / ub, cpu = ub / 16, NB = rows / 128;
   const long long n = e1 * rows * nch;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int ch = (int)(i % nch);
     const long long row = (i / nch) % rows, e = i / ((long long)nch * rows);
     const int u = ch / cpu, j = ch % cpu;
-    uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)ch * 16);
-    if (f4) v = make_uint4(f4_pack_word(v.x), f4_pack_word(v.y), f4_pack_word(v.z), f4_pack_word(v.w));
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)ch * 16);
     const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + (long long)j * 2048 + (row % 128) * 16;
     *reinterpret_cast<uint4*>(dst + off) = v;
-  }
-}
-
-// MXFP4 e8m0 scales [E+1][rows][ns] -> per weight row the reference
-// exponent s_ref = (largest scale exponent) - 6, stored as 2^s_ref in
-// ref[E+1][rows/128][nm * 128] (slot m as below), and per block d = s - s_ref
-// as int8 (at least -127) after each unit's codes, 4 per unit-row:
-// dst[unit * ustride + msub + code_bytes + (row % 128) * 4 + jj]
-__global__ void pack_tq_rel_kernel(const uint8_t* src, uint8_t* dst, float* ref, long long e1, int rows, int ns,
-                                   long long ustride, int msub, int code_bytes, int nm, int m) {
-  const int nu = ns / 4, NB = rows / 128;
-  const long long n = e1 * rows;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long row = i % rows, e = i / rows;
-    const uint8_t* sc = src + (e * rows + row) * ns;
-    int mx = 0;
-    for (int k = 0; k < ns; ++k) mx = max(mx, (int)sc[k]);
-    const int sref = mx - 127 - 6;
-    ref[(e * NB + row / 128) * (nm * 128) + m * 128 + row % 128] = ldexpf(1.0f, sref);
-    for (int u = 0; u < nu; ++u) {
-      uint32_t v = 0;
-      for (int jj = 0; jj < 4; ++jj) {
-        const int d = max(-127, (int)sc[u * 4 + jj] - 127 - sref);
-        v |= (uint32_t)(uint8_t)(int8_t)d << (8 * jj);
-      }
-      const long long off = ((e * NB + row / 128) * nu + u) * ustride + msub + code_bytes + (row % 128) * 4;
-      *reinterpret_cast<uint32_t*>(dst + off) = v;
-    }
   }
 }
 
@@ -193,6 +167,44 @@ __global__ void pack_tq_scales_kernel(const float* src, float* dst, long long e1
     const int u = (int)(i % nu);
     const long long row = (i / nu) % rows, e = i / ((long long)nu * rows);
     dst[((e * NB + row / 128) * nu + u) * (nm * 128) + m * 128 + row % 128] = src[(e * rows + row) * nu + u];
+  }
+}
+
+// MXFP4 on the block-scaled tensor-core path, codes: one [E+1][rows][K/2]
+// byte matrix set -> unit-matrices of 128 rows x 128 contraction elements,
+// each 128 rows x 64 bytes row-major (the e2m1 stream as given, two codes a
+// byte), unit-matrix (e, row block, unit u, slot msub of nm) at
+//   dst[(((e * rows/128 + row/128) * nu + u) * nm + msub) * 8192 + (row % 128) * 64]
+// so a 2-D tensor map of 64-byte rows reads a unit-matrix as one box.
+__global__ void pack_mx_codes_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int row_bytes, int nm,
+                                     int msub) {
+  const int nu = row_bytes / 64, NB = rows / 128;
+  const long long n = e1 * rows * nu * 4;   // 16-byte chunks
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int q = (int)(i & 3), u = (int)((i >> 2) % nu);
+    const long long row = (i >> 2) / nu % rows, e = (i >> 2) / nu / rows;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (e * rows + row) * row_bytes + (long long)u * 64 + q * 16);
+    const long long um = ((e * NB + row / 128) * nu + u) * nm + msub;
+    *reinterpret_cast<uint4*>(dst + um * 8192 + (row % 128) * 64 + q * 16) = v;
+  }
+}
+
+// MXFP4 e8m0 block scales [E+1][rows][K/32] -> one 512-byte chunk per
+// unit-matrix (same indexing as the codes), byte 16 a + 4 b + j = the scale
+// of row 32 b + a of the block for K-block j of the unit: the layout that
+// tcgen05.cp (32x128b, copied to all four lane quarters) turns into tensor-
+// memory column b, lane a, byte j, which is where the block-scaled MMA reads
+// row 32 b + a's scale for its K-step j.
+__global__ void pack_mx_scales_kernel(const uint8_t* src, uint8_t* dst, long long e1, int rows, int ns, int nm,
+                                      int msub) {
+  const int nu = ns / 4, NB = rows / 128;
+  const long long n = e1 * rows * ns;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int k = (int)(i % ns);
+    const long long row = (i / ns) % rows, e = i / ns / rows;
+    const int u = k / 4, j = k % 4, r = (int)(row % 128), a = r % 32, b = r / 32;
+    const long long um = ((e * NB + row / 128) * nu + u) * nm + msub;
+    dst[um * 512 + 16 * a + 4 * b + j] = src[(e * rows + row) * ns + k];
   }
 }
 
@@ -265,6 +277,33 @@ int pack_matrix(mono_ffn_plan_t* p, const void* codes, const void* scales, uint8
                                                      sb, rc, item, sub, vec);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? 0 : cuda_fail(p, e, "pack kernel launch");
+}
+
+// 2-D tensor map of packed MXFP4 unit-matrices: rows of 128 e2m1 codes (64
+// bytes), `rows` of them; one box is a unit-matrix (128 rows).  Data type
+// 16U4_ALIGN16B: in shared memory every 16 codes take a 16-byte slot (8 bytes
+// of codes, then 8 unused), which is how the block-scaled MMA reads e2m1;
+// with the 128-byte swizzle, so that a box is the MMA's swizzled K-major
+// operand.
+int make_f4_map(mono_ffn_plan_t* p, CUtensorMap* map, void* base, unsigned long long rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(p, MONO_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {64};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, base, dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(p, MONO_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return 0;
 }
 
 template <typename T>
@@ -347,6 +386,8 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   need(dt >= MONO_F32 && dt <= MONO_MXFP4, "expert_dtype unknown");
   need(!(cfg.hc_dtype == MONO_BF16 && !cfg.round_bf16), "bf16 residual streams need round_bf16 = 1");
   need(cfg.sinkhorn_iters >= 0, "sinkhorn_iters must be >= 0");
+  need(cfg.dense == 0 || cfg.dense == 1, "dense must be 0 or 1");
+  need(!cfg.dense || cfg.top_k == cfg.n_routed, "a dense layer takes every slot: top_k must equal n_routed");
   if (dt >= MONO_F32 && dt <= MONO_MXFP4 && cfg.hidden > 0 && cfg.inter > 0) {
     const int m = std::max(unit_elems(dt), block_of(dt));
     need(cfg.hidden % m == 0, "hidden must be a multiple of " + std::to_string(m) + " for this expert format");
@@ -379,7 +420,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->tc = dt == MONO_BF16 && cfg.round_bf16 && H % 128 == 0 && I % 128 == 0;
   // FP8 / MXFP4 experts: converted to fp16 on the way into the tensor cores
   p->tq = (dt == MONO_FP8E4M3_B128 || dt == MONO_MXFP4) && cfg.round_bf16 && H % 128 == 0 && I % 128 == 0;
-  const long long tq_mat = dt == MONO_FP8E4M3_B128 ? 16384 : 8192 + 512;   // one 128 x 128 unit of one matrix
+  const long long tq_mat = dt == MONO_FP8E4M3_B128 ? 16384 : 8192;   // one 128 x 128 unit of one matrix in HBM
   // chunking of the packed rows
   const int gu_target = dt == MONO_F32 ? 256 : dt == MONO_BF16 ? 512 : 1024;
   const int dn_target = dt == MONO_F32 ? 512 : dt == MONO_BF16 ? 1024 : 2048;
@@ -400,7 +441,9 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   if (p->tq) {
     p->gu_estride = (long long)(I / 128) * (H / 128) * 2 * tq_mat;
     p->dn_estride = (long long)(H / 128) * (I / 128) * tq_mat;
-    p->slot_bytes = (int)(2 * tq_mat);
+    // FP8: two unit-matrices as they are in HBM; MXFP4: two unit-matrices
+    // with each 16-code group in a 16-byte slot, then their scale chunks
+    p->slot_bytes = dt == MONO_FP8E4M3_B128 ? (int)(2 * tq_mat) : 2 * 16384 + 2 * 512;
   }
 
   // grid and shared memory
@@ -460,10 +503,15 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     if (!rc) rc = dalloc(p, &l.gu, (size_t)(E + 1) * p->gu_estride, &p->packed_bytes);
     if (!rc) rc = dalloc(p, &l.dn, (size_t)(E + 1) * p->dn_estride, &p->packed_bytes);
     if (!rc && p->tq) {
-      // FP8: one block scale per (row, unit); MXFP4: one reference per row
-      const size_t nu_g = dt == MONO_FP8E4M3_B128 ? H / 128 : 1, nu_d = dt == MONO_FP8E4M3_B128 ? I / 128 : 1;
-      rc = dalloc(p, &l.gsc, (size_t)(E + 1) * (I / 128) * nu_g * 256 * 4, &p->packed_bytes);
-      if (!rc) rc = dalloc(p, &l.dsc, (size_t)(E + 1) * (H / 128) * nu_d * 128 * 4, &p->packed_bytes);
+      // FP8: one fp32 block scale per (row, unit); MXFP4: one 512-byte chunk
+      // of e8m0 scales per unit-matrix (4 per row)
+      const size_t units = (size_t)(E + 1) * (I / 128) * (H / 128);
+      rc = dalloc(p, &l.gsc, units * 2 * (dt == MONO_FP8E4M3_B128 ? 128 * 4 : 512), &p->packed_bytes);
+      if (!rc) rc = dalloc(p, &l.dsc, units * (dt == MONO_FP8E4M3_B128 ? 128 * 4 : 512), &p->packed_bytes);
+      if (!rc && dt == MONO_MXFP4) {
+        rc = make_f4_map(p, &l.tm_gu, l.gu, (unsigned long long)units * 2 * 128);
+        if (!rc) rc = make_f4_map(p, &l.tm_dn, l.dn, (unsigned long long)units * 128);
+      }
     }
   }
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
@@ -483,10 +531,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   p->pend.assign(cfg.n_layers, nullptr);
   for (int l = 0; l + 1 < cfg.n_layers && !rc; ++l)
     rc = dalloc(p, &p->pend[l], (size_t)RM * (kS + kS * kS + H) * 4, &p->scratch_bytes);
-  if (cfg.n_layers > 1) {
-    if (!rc) rc = dalloc(p, &p->xbuf[0], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
-    if (!rc) rc = dalloc(p, &p->xbuf[1], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
-  }
+  // residual streams a layer materialises when it opens with a pending
+  // expand: the chain's layers alternate between two, a step opened by the
+  // attention sublayer's expand uses the first
+  if (!rc) rc = dalloc(p, &p->xbuf[0], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
+  if (cfg.n_layers > 1 && !rc) rc = dalloc(p, &p->xbuf[1], (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->sync, sizeof(SyncBlock) * cfg.n_layers, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->err, sizeof(ErrBlock), &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->stage_in, (size_t)RM * kS * H * hc_elem, &p->scratch_bytes);
@@ -521,8 +570,8 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
   std::string why;
   if (!w->mix_w) why += "mix_w is NULL\n";
   if (!w->norm_w) why += "norm_w is NULL\n";
-  if (!w->router_w) why += "router_w is NULL\n";
-  if (!w->router_bias) why += "router_bias is NULL\n";
+  if (!w->router_w && !p->cfg.dense) why += "router_w is NULL\n";
+  if (!w->router_bias && !p->cfg.dense) why += "router_bias is NULL\n";
   if (!w->w_gate || !w->w_up || !w->w_down) why += "expert weights are NULL\n";
   if (!why.empty()) return fail(p, MONO_ERR_INVALID_ARG, why);
   int prev = 0;
@@ -534,8 +583,10 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
   const size_t norm_elem = p->cfg.norm_dtype == MONO_BF16 ? 2 : 4;
   cudaMemcpyAsync(l.mix_w, w->mix_w, (size_t)kS * H * kMixC * 4, cudaMemcpyDeviceToDevice, st);
   cudaMemcpyAsync(l.norm_w, w->norm_w, (size_t)H * norm_elem, cudaMemcpyDeviceToDevice, st);
-  cudaMemcpyAsync(l.bias, w->router_bias, (size_t)E * 4, cudaMemcpyDeviceToDevice, st);
-  transpose_f32_kernel<<<dim3((E + 31) / 32, (H + 31) / 32), dim3(32, 8), 0, st>>>(w->router_w, l.router_t, H, E);
+  if (!p->cfg.dense) {   // a dense layer has no router
+    cudaMemcpyAsync(l.bias, w->router_bias, (size_t)E * 4, cudaMemcpyDeviceToDevice, st);
+    transpose_f32_kernel<<<dim3((E + 31) / 32, (H + 31) / 32), dim3(32, 8), 0, st>>>(w->router_w, l.router_t, H, E);
+  }
   int rc = 0;
   if (p->tc) {
     // 128-row blocks of core matrices: gate and up of a rowgroup side by
@@ -556,8 +607,8 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
     const bool fp8 = p->wt == W_FP8;
     const int th = 256;
     auto grid = [&](long long n) { return (unsigned)std::min<long long>((n + th - 1) / th, 148LL * 64); };
-    const long long mat = fp8 ? 16384 : 8192 + 512;
-    const int code_b = fp8 ? 16384 : 8192, ub = fp8 ? 128 : 64;   // unit-row bytes of codes
+    const long long mat = 16384;   // FP8: one unit-matrix
+    const int ub = 128;            // FP8: unit-row bytes of codes
     const int gu_rb = fp8 ? H : H / 2, dn_rb = fp8 ? I : I / 2;    // code bytes per weight row
     if (!fp8) {
       // e8m0 code 255 is NaN: not a scale the tensor-core path can expand
@@ -585,13 +636,13 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
         return fail(p, MONO_ERR_INVALID_ARG, "pack: MXFP4 scale code 255 (NaN)");
       }
     }
-    pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_gate, l.gu, E + 1, I, gu_rb, ub, 2 * mat, 0, !fp8);
-    pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_up, l.gu, E + 1, I, gu_rb, ub, 2 * mat, (int)mat, !fp8);
-    pack_tq_codes_kernel<<<grid((long long)(E + 1) * H * (dn_rb / 16)), th, 0, st>>>(
-        (const uint8_t*)w->w_down, l.dn, E + 1, H, dn_rb, ub, mat, 0, !fp8);
     if (fp8) {
+      pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
+          (const uint8_t*)w->w_gate, l.gu, E + 1, I, gu_rb, ub, 2 * mat, 0);
+      pack_tq_codes_kernel<<<grid((long long)(E + 1) * I * (gu_rb / 16)), th, 0, st>>>(
+          (const uint8_t*)w->w_up, l.gu, E + 1, I, gu_rb, ub, 2 * mat, (int)mat);
+      pack_tq_codes_kernel<<<grid((long long)(E + 1) * H * (dn_rb / 16)), th, 0, st>>>(
+          (const uint8_t*)w->w_down, l.dn, E + 1, H, dn_rb, ub, mat, 0);
       pack_tq_scales_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
           (const float*)w->s_gate, l.gsc, E + 1, I, H / 128, 2, 0);
       pack_tq_scales_kernel<<<grid((long long)(E + 1) * I * (H / 128)), th, 0, st>>>(
@@ -599,12 +650,22 @@ extern "C" int mono_ffn_pack_weights(mono_ffn_plan_t* p, int layer, const mono_f
       pack_tq_scales_kernel<<<grid((long long)(E + 1) * H * (I / 128)), th, 0, st>>>(
           (const float*)w->s_down, l.dsc, E + 1, H, I / 128, 1, 0);
     } else {
-      pack_tq_rel_kernel<<<grid((long long)(E + 1) * I), th, 0, st>>>((const uint8_t*)w->s_gate, l.gu, l.gsc, E + 1, I,
-                                                                     H / 32, 2 * mat, 0, code_b, 2, 0);
-      pack_tq_rel_kernel<<<grid((long long)(E + 1) * I), th, 0, st>>>((const uint8_t*)w->s_up, l.gu, l.gsc, E + 1, I,
-                                                                     H / 32, 2 * mat, (int)mat, code_b, 2, 1);
-      pack_tq_rel_kernel<<<grid((long long)(E + 1) * H), th, 0, st>>>((const uint8_t*)w->s_down, l.dn, l.dsc, E + 1, H,
-                                                                     I / 32, mat, 0, code_b, 1, 0);
+      // unit-matrices of 128 rows x 64 bytes (gate/up as pairs), and their
+      // 512-byte scale chunks in the order the tensor memory copy takes
+      pack_mx_codes_kernel<<<grid((long long)(E + 1) * I * (H / 128) * 4), th, 0, st>>>(
+          (const uint8_t*)w->w_gate, l.gu, E + 1, I, H / 2, 2, 0);
+      pack_mx_codes_kernel<<<grid((long long)(E + 1) * I * (H / 128) * 4), th, 0, st>>>(
+          (const uint8_t*)w->w_up, l.gu, E + 1, I, H / 2, 2, 1);
+      pack_mx_codes_kernel<<<grid((long long)(E + 1) * H * (I / 128) * 4), th, 0, st>>>(
+          (const uint8_t*)w->w_down, l.dn, E + 1, H, I / 2, 1, 0);
+      uint8_t* gsc = reinterpret_cast<uint8_t*>(l.gsc);
+      uint8_t* dsc = reinterpret_cast<uint8_t*>(l.dsc);
+      pack_mx_scales_kernel<<<grid((long long)(E + 1) * I * (H / 32)), th, 0, st>>>(
+          (const uint8_t*)w->s_gate, gsc, E + 1, I, H / 32, 2, 0);
+      pack_mx_scales_kernel<<<grid((long long)(E + 1) * I * (H / 32)), th, 0, st>>>(
+          (const uint8_t*)w->s_up, gsc, E + 1, I, H / 32, 2, 1);
+      pack_mx_scales_kernel<<<grid((long long)(E + 1) * H * (I / 32)), th, 0, st>>>(
+          (const uint8_t*)w->s_down, dsc, E + 1, H, I / 32, 1, 0);
     }
     cudaError_t e2 = cudaGetLastError();
     cudaSetDevice(prev);
@@ -650,6 +711,28 @@ extern "C" int mono_ffn_set_taps(mono_ffn_plan_t* p, int layer, const mono_ffn_t
   return MONO_OK;
 }
 
+namespace {
+
+// The attention sublayer's pending post / expand that a step may open with
+// (mono_ffn_step_pending); all NULL for a plain step.
+struct Pending {
+  const void* x;
+  const float* post;
+  const float* comb;
+  const void* y;
+};
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const char* x = (const char*)a;
+  const char* y = (const char*)b;
+  return x < y + nb && y < x + na;
+}
+
+int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd, const int* row_slot, void* hc_out,
+              void* stream);
+
+}  // namespace
+
 extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, void* hc_out, void* stream) {
   if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "step: NULL plan");
   if (rows == 0) return MONO_OK;
@@ -658,11 +741,50 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
                                              std::to_string(p->cfg.max_rows) + "]");
   if (!hc_in || !hc_out) return fail(p, MONO_ERR_INVALID_ARG, "step: NULL hc_in or hc_out");
   const size_t hc_bytes = (size_t)rows * kS * p->cfg.hidden * (p->cfg.hc_dtype == MONO_BF16 ? 2 : 4);
-  {
-    const char* a = (const char*)hc_in;
-    const char* b = (const char*)hc_out;
-    if (a < b + hc_bytes && b < a + hc_bytes) return fail(p, MONO_ERR_INVALID_ARG, "step: hc_in and hc_out overlap");
-  }
+  if (overlaps(hc_in, hc_bytes, hc_out, hc_bytes)) return fail(p, MONO_ERR_INVALID_ARG, "step: hc_in and hc_out overlap");
+  return step_impl(p, rows, hc_in, nullptr, nullptr, hc_out, stream);
+}
+
+extern "C" int mono_ffn_step_padded(mono_ffn_plan_t* p, int width, const int* row_slot, const void* hc_in,
+                                    void* hc_out, void* stream) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "step_padded: NULL plan");
+  if (width == 0) return MONO_OK;
+  if (width < 0 || width > p->cfg.max_rows)
+    return fail(p, MONO_ERR_INVALID_ARG, "step_padded: width " + std::to_string(width) + " outside [0, max_rows = " +
+                                             std::to_string(p->cfg.max_rows) + "]");
+  if (!row_slot || !hc_in || !hc_out) return fail(p, MONO_ERR_INVALID_ARG, "step_padded: NULL argument");
+  const size_t hc_bytes = (size_t)width * kS * p->cfg.hidden * (p->cfg.hc_dtype == MONO_BF16 ? 2 : 4);
+  if (overlaps(hc_in, hc_bytes, hc_out, hc_bytes))
+    return fail(p, MONO_ERR_INVALID_ARG, "step_padded: hc_in and hc_out overlap");
+  return step_impl(p, width, hc_in, nullptr, row_slot, hc_out, stream);
+}
+
+extern "C" int mono_ffn_step_pending(mono_ffn_plan_t* p, int rows, const void* x_attn, const float* attn_post,
+                                     const float* attn_comb, const void* y_attn, void* hc_out, void* stream) {
+  if (!p) return fail(nullptr, MONO_ERR_INVALID_ARG, "step_pending: NULL plan");
+  if (rows == 0) return MONO_OK;
+  if (rows < 0 || rows > p->cfg.max_rows)
+    return fail(p, MONO_ERR_INVALID_ARG, "step_pending: rows " + std::to_string(rows) + " outside [0, max_rows = " +
+                                             std::to_string(p->cfg.max_rows) + "]");
+  if (!x_attn || !attn_post || !attn_comb || !y_attn || !hc_out)
+    return fail(p, MONO_ERR_INVALID_ARG, "step_pending: NULL argument");
+  const size_t el = p->cfg.hc_dtype == MONO_BF16 ? 2 : 4;
+  const size_t hc_bytes = (size_t)rows * kS * p->cfg.hidden * el, y_bytes = (size_t)rows * p->cfg.hidden * el;
+  std::string why;
+  if (overlaps(x_attn, hc_bytes, hc_out, hc_bytes)) why += "x_attn and hc_out overlap\n";
+  if (overlaps(y_attn, y_bytes, hc_out, hc_bytes)) why += "y_attn and hc_out overlap\n";
+  if (overlaps(attn_post, (size_t)rows * kS * 4, hc_out, hc_bytes) ||
+      overlaps(attn_comb, (size_t)rows * kS * kS * 4, hc_out, hc_bytes))
+    why += "attn_post or attn_comb overlaps hc_out\n";
+  if (!why.empty()) return fail(p, MONO_ERR_INVALID_ARG, "step_pending: " + why);
+  const Pending pd{x_attn, attn_post, attn_comb, y_attn};
+  return step_impl(p, rows, x_attn, &pd, nullptr, hc_out, stream);
+}
+
+namespace {
+
+int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd, const int* row_slot, void* hc_out,
+              void* stream) {
   for (int l = 0; l < p->cfg.n_layers; ++l)
     if (!p->layers[l].packed)
       return fail(p, MONO_ERR_NOT_PACKED, "step: layer " + std::to_string(l) + " has no packed weights");
@@ -682,7 +804,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.R = rows;
     prm.G = p->G;
     prm.layer = l;
-    prm.first = l == 0;
+    prm.first = l == 0 && !pd;
+    prm.dense = p->cfg.dense;
     prm.last = l == L - 1;
     prm.mix_ctas = p->mix_ctas;
     prm.hc_bf16 = p->cfg.hc_dtype == MONO_BF16;
@@ -694,10 +817,23 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.route_scale = p->cfg.route_scale;
     prm.denom_clamp = p->cfg.denom_clamp;
     prm.sink_iters = p->cfg.sinkhorn_iters;
-    prm.x_prev = l <= 1 ? hc_in : p->xbuf[(l - 1) % 2];
-    prm.xbuf = l == 0 ? nullptr : p->xbuf[l % 2];
+    // layer l reads the residual streams of layer l - 1 (hc_in for layer 0,
+    // or, opened by a pending expand, the attention sublayer's input) and
+    // materialises its own in xbuf[l % 2] when it opens with an expand
+    prm.x_prev = l == 0 ? hc_in : l == 1 ? (pd ? p->xbuf[0] : hc_in) : p->xbuf[(l - 1) % 2];
+    prm.xbuf = prm.first ? nullptr : p->xbuf[l % 2];
     prm.hc_out = hc_out;
-    prm.pend_in = l > 0 ? p->pend[l - 1] : nullptr;
+    if (l > 0) {
+      prm.pend_post = p->pend[l - 1];
+      prm.pend_comb = p->pend[l - 1] + rows * kS;
+      prm.pend_y = p->pend[l - 1] + rows * kS + rows * kS * kS;
+      prm.pend_y_bf16 = 0;
+    } else if (pd) {
+      prm.pend_post = pd->post;
+      prm.pend_comb = pd->comb;
+      prm.pend_y = pd->y;
+      prm.pend_y_bf16 = p->cfg.hc_dtype == MONO_BF16;
+    }
     prm.pend_out = l + 1 < L ? p->pend[l] : nullptr;
     prm.mix_w = ls.mix_w;
     prm.norm_w = ls.norm_w;
@@ -727,6 +863,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.xready = p->xready;
     prm.gsc = ls.gsc;
     prm.dsc = ls.dsc;
+    prm.tm_gu = ls.tm_gu;
+    prm.tm_dn = ls.tm_dn;
     prm.n_xready = p->xready ? rows * p->cfg.top_k + 1 : 0;
     prm.sync = p->sync + l;
     prm.err = p->err;
@@ -736,6 +874,7 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
     prm.regA_bytes = p->regA_bytes;
     prm.ymax = p->ymax;
     prm.timeout_ns = (unsigned long long)p->cfg.wait_timeout_us * 1000ull;
+    prm.row_slot = row_slot;
     prm.fault_cta = p->fault_cta;
     prm.fault_stage = p->fault_cta >= 0 ? p->fault_stage : 0;
     prm.jitter_ns = p->jitter_ns;
@@ -758,6 +897,8 @@ extern "C" int mono_ffn_step(mono_ffn_plan_t* p, int rows, const void* hc_in, vo
   if (e != cudaSuccess) return cuda_fail(p, e, "step launch");
   return MONO_OK;
 }
+
+}  // namespace
 
 extern "C" int mono_ffn_step_host(mono_ffn_plan_t* p, int rows, const void* hc_in_host, void* hc_out_host,
                                   void* stream) {
@@ -825,9 +966,9 @@ extern "C" int mono_ffn_get_info(const mono_ffn_plan_t* p, mono_ffn_info* info) 
   info->expert_bytes = p->gu_estride + p->dn_estride;
   if (p->tq && p->wt == W_FP8)   // the FP8 block scales travel in their own arrays
     info->expert_bytes += (int64_t)(p->cfg.inter / 128) * (H / 128) * 256 * 4 + (int64_t)(H / 128) * (p->cfg.inter / 128) * 128 * 4;
-  if (p->tq && p->wt == W_FP4)   // and the MXFP4 row references
-    info->expert_bytes += (int64_t)(2 * p->cfg.inter + H) * 4;
-  info->dense_bytes = (int64_t)kS * H * kMixC * 4 + (int64_t)E * H * 4 + (int64_t)E * 4 +
+  if (p->tq && p->wt == W_FP4)   // and the MXFP4 e8m0 block scales (one byte per 32 codes)
+    info->expert_bytes += (int64_t)(p->cfg.inter / 128) * (H / 128) * 3 * 512;
+  info->dense_bytes = (int64_t)kS * H * kMixC * 4 + (p->cfg.dense ? 0 : (int64_t)E * H * 4 + (int64_t)E * 4) +
                       (int64_t)H * (p->cfg.norm_dtype == MONO_BF16 ? 2 : 4);
   info->packed_bytes = p->packed_bytes;
   info->scratch_bytes = p->scratch_bytes;

@@ -226,56 +226,6 @@ __device__ __forceinline__ void umma_unit_e4m3(uint32_t d, uint64_t da, uint64_t
   }
 }
 
-// One 128 x 128 e4m3 unit with A in tensor memory (lane = row, 32-bit
-// column c = contraction elements 4c .. 4c + 3, lowest byte first), issued
-// by one elected lane: 4 K-steps of 32 (8 columns each), the first
-// overwriting D; B from the descriptor db advanced db_step units a K-step.
-// pair: a second A (up) 32 columns on, into d + 16.
-__device__ __forceinline__ void umma_unit_e4m3_tmem_a(uint32_t d, uint32_t a, uint64_t db, uint32_t db_step,
-                                                      uint32_t idesc, bool pair) {
-  if (pair) {
-    asm volatile(
-        "{\n .reg .pred e, t, f;\n .reg .b32 rx, a0, a1, d1;\n .reg .b64 b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
-        " mov.b32 a0, %1;\n add.u32 a1, %1, 32;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, f;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, f;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u32 a1, a1, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [d1], [a1], b, %4, t;\n"
-        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n .reg .pred e, t, f;\n .reg .b32 rx, a0;\n .reg .b64 b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
-        " mov.b32 a0, %1;\n mov.b64 b, %2;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, f;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        " add.u32 a0, a0, 8;\n add.u64 b, b, %3;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a0], b, %4, t;\n"
-        "}\n" ::"r"(d), "r"(a), "l"(db), "l"((uint64_t)db_step), "r"(idesc)
-        : "memory");
-  }
-}
-
-// 32 lanes x 8 consecutive 32-bit columns from registers (thread l of the
-// warp writes its quadrant's lane l)
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
-               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
-
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -299,6 +249,100 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
         "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand stored with the
+// 128-byte swizzle (rows of 128 bytes, the 16-byte chunks of row r at chunk
+// index c ^ (r % 8), 8-row atoms of 1024 bytes): sbo = byte distance between
+// 8-row groups; the leading offset is unused for this layout (encoded 1).
+// The atom must sit on a 1024-byte boundary; moving along K inside it adds
+// the byte offset to the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;   // descriptor version of sm_100
+  d |= (uint64_t)2 << 61;   // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scales: e2m1 A, e4m3 B,
+// e8m0 scale factors, fp32 accumulator, both K-major, M = m, N = n; the
+// scale-factor byte selectors (bits 4-5 for B, 29-30 for A) are added per
+// K-step.
+__host__ __device__ constexpr uint32_t umma_idesc_mx_e2m1_e4m3(int m, int n) {
+  return (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(m >> 4) << 24);
+}
+
+// One 128 x 128 unit of e2m1 weights (A, 128-byte-swizzled K-major, in
+// shared memory) against e4m3 B, with the unit's 4 x 128 e8m0 block scales
+// in tensor memory at sfa (4 columns, byte j = K-block j) and B's scales at
+// sfb: tcgen05.cp brings the scale chunk from shared memory (sf_smem) first,
+// then 4 block-scaled MMAs of K = 32, the first overwriting D.  pair: a
+// second A (up) 16384 bytes on, its scales at sfa2 from sf_smem2, into d + 16.
+// One elected lane of a converged warp issues all of it, in order.
+__device__ __forceinline__ void umma_unit_mx(uint32_t d, uint64_t da, uint64_t db, uint32_t db_step, uint32_t idesc,
+                                             uint32_t sfa, uint64_t sfd, uint32_t sfa2, uint64_t sfd2, uint32_t sfb,
+                                             bool pair) {
+  if (pair) {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, d1, i, s0, s1;\n .reg .b64 a0, a1, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n"
+        " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%7], %8;\n"
+        " mov.b64 a0, %1;\n add.u64 a1, %1, 1024;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
+        " mov.b32 i, %4;\n mov.b32 s0, %5;\n mov.b32 s1, %7;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], f;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], f;\n"
+        " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
+        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
+        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
+        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(sfa), "l"(sfd), "r"(sfa2), "l"(sfd2),
+        "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, i, s0;\n .reg .b64 a0, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n"
+        " mov.b64 a0, %1;\n mov.b64 b, %2;\n mov.b32 i, %4;\n mov.b32 s0, %5;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], f;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(sfa), "l"(sfd), "r"(sfb)
+        : "memory");
+  }
+}
+
+// 32 lanes x 4 consecutive 32-bit columns from registers (thread l of the
+// warp writes its quadrant's lane l)
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v0), "r"(v1), "r"(v2),
+               "r"(v3)
+               : "memory");
+}
+
+// 2-D tiled TMA load of the box at coordinates (c0, c1) of the tensor map
+// into this CTA's shared memory, completion counted on bar
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void bar_arrive(int id, int threads) {

@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     c->nu = 0;
     c->n_ready = 0;
     c->epoch = ld_relaxed(&p.sync->epoch);
+    c->live = live_rows(p);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
       // the prologue's later inputs go to L2 ahead of the weight stream:
       // this CTA's router rows, the norm weights and the router bias
       const int e0 = (int)((long long)blockIdx.x * p.E / G), e1 = (int)((long long)(blockIdx.x + 1) * p.E / G);
-      prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
+      if (!p.dense) prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
       prefetch_l2_span(p.norm_w, (size_t)H * (p.norm_bf16 ? 2 : 4));
       prefetch_l2_span(p.bias, (size_t)p.E * 4);
     }

@@ -25,21 +25,22 @@
 // bytes, 2048 bytes between K-neighbours and 128 between row groups.  A ring
 // stage is one gate/up unit (gate, then up) or two down units, 32 KB.
 //
-// MXFP4 takes the same MMAs after one step: warps 4-7 (one thread per weight
-// row, its tensor-memory lane) expand each ring stage's e2m1 codes to e4m3
-// in tensor memory (six A buffers of one stage, 64 columns each), and the
-// MMAs read A from there.  A code times its block scale 2^s is written as
-// the e4m3 value code * 2^(s - s_ref), where s_ref, fixed per weight row at
-// packing, is the row's largest block exponent minus 6: every e2m1 value
-// times 2^d is an e4m3 value for d in [-8, 6] (6 * 2^6 = 384 <= 448; the
-// subnormal step 2^-9 divides 0.5 * 2^-8), so the expansion is exact unless
-// a block's scale lies more than 2^14 below its row's largest, where the
-// values are rounded to e4m3 (an error below 2^-16 of the row's largest
-// scale).  2^s_ref plays the part of the FP8 block scale in the epilogue.
-// Packed MXFP4 units: codes [4 chunks][128 rows][16] (32 e2m1 per chunk, 8
-// a word with the sign bits moved: f4_pack_word), then d = s - s_ref as int8
-// [128 rows][4], 8704 bytes a matrix; the per-row 2^s_ref sit in their own
-// arrays.
+// MXFP4 runs block-scaled MMAs (tcgen05.mma kind::mxf8f6f4.block_scale, e2m1
+// A, e4m3 B, e8m0 scale factors): the weights' own 32-element block scales
+// are applied inside the tensor core, so the codes go from HBM to the tensor
+// core untouched.  A 2-D tensor map of the packed codes (data type
+// 16U4_ALIGN16B) lets the TMA unit place each 16-code group in a 16-byte
+// slot of shared memory (8 bytes of codes, 8 unused) with the 128-byte
+// swizzle, which is the layout the MMA reads e2m1 from; a unit-matrix is 8 KB
+// in HBM and 16 KB in the ring.  Its 4 x 128 scales (512 bytes, packed in the
+// order tcgen05.cp expects) come with the same stage; the issuing lane copies
+// them into tensor memory (tcgen05.cp 32x128b to all four lane quarters)
+// right before the unit's MMAs, which pick the K-block's byte through the
+// scale-factor id.  B's scale factors are all 1 (e8m0 127), written once:
+// the activations keep their power-of-two row scales in the epilogue, as
+// for FP8.
+// Packed MXFP4 unit-matrices: 128 rows x 64 bytes row-major, gate/up units as
+// (gate, up) pairs; scale chunks of 512 bytes in arrays of their own.
 #pragma once
 #include <cuda_fp8.h>
 
@@ -47,21 +48,29 @@
 
 namespace mono {
 
-// one 128 x 128 unit of one matrix in the ring: codes (and MXFP4 d bytes)
+// one 128 x 128 unit of one matrix: bytes in HBM
 template <int WT> struct TqFmt;
 template <> struct TqFmt<W_FP8> {
   static constexpr int MAT_BYTES = 16384;
 };
 template <> struct TqFmt<W_FP4> {
-  static constexpr int MAT_BYTES = 8192 + 512;
+  static constexpr int MAT_BYTES = 8192;
 };
 
 constexpr int kF8TmemCols = 128;   // four accumulators of 32 columns (gate 16 | up 16)
-constexpr int kF4TmemCols = 512;   // the accumulators, then the MXFP4 A buffers
-constexpr int kF4Ab = 6;           // MXFP4 A buffers of one ring stage (64 columns) in tensor memory
-static_assert(kF4Ab <= kMaxAb && kF8TmemCols + 64 * kF4Ab <= kF4TmemCols, "A buffers fit");
+constexpr int kF4TmemCols = 256;   // the accumulators, then the scale factors
+constexpr uint32_t kF4SfaCol = 128;   // A scale factors: 8 columns per accumulator (gate 4 | up 4)
+constexpr uint32_t kF4SfbCol = 160;   // B scale factors: 4 columns of 1.0
+constexpr int kF4SmemMat = 16384;  // one MXFP4 unit-matrix in the ring (16-byte slot per 16 codes)
+constexpr int kF4Sf = 512;         // its scale chunk
+constexpr int kF4SfOff = 2 * kF4SmemMat;   // the scale chunks of a stage, after its two unit-matrices
+// transaction bytes one unit-matrix box of the tensor map counts on its
+// mbarrier: the bytes of codes it writes (the 8-byte gaps of the 16-byte
+// slots are left as they were, and the MMA does not read them)
+constexpr uint32_t kF4BoxTx = kF4SmemMat / 2;
 constexpr uint32_t kF8Acc = 4;
 static_assert(kF8Acc <= (uint32_t)kMaxAcc, "accumulator barriers");
+static_assert(kF4SfaCol + 8 * kF8Acc <= kF4SfbCol && kF4SfbCol + 4 <= (uint32_t)kF4TmemCols, "tensor memory");
 
 // bytes of one expert entry's down B operand: [I/16][16 rows][16] e4m3 codes,
 // then [I/128][8] fp32 inverse scales
@@ -84,83 +93,6 @@ __device__ __forceinline__ void f8_split2(float y0, float y1, uint32_t& hi, uint
       __nv_cvt_float2_to_fp8x2(make_float2(y0 - hf.x, y1 - hf.y), __NV_SATFINITE, __NV_E4M3);
   hi = h;
   lo = l;
-}
-
-// e4m3 of the 8 e2m1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} times 2^d, as
-// bytes 0-3 / 4-7 of a byte-permute table.  For d in [-5, 6] every nonzero
-// entry is a normal e4m3 value and d is added to the exponent field of the
-// d = 0 table (f4_lut_fast); below -5 the values are converted one by one
-// (subnormal, or rounded below -8), out of line since it is rare.
-__device__ __forceinline__ void f4_lut_fast(int d, uint32_t& l0, uint32_t& l1) {
-  const uint32_t de = (uint32_t)(d * 8);
-  l0 = 0x3C383000u + de * 0x01010100u;
-  l1 = 0x4C484440u + de * 0x01010101u;
-}
-__device__ __noinline__ uint2 f4_lut_slow(int d) {
-  const float s = ldexpf(1.0f, max(d, -126));
-  const uint32_t a = __nv_cvt_float2_to_fp8x2(make_float2(0.f, 0.5f * s), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t b = __nv_cvt_float2_to_fp8x2(make_float2(1.0f * s, 1.5f * s), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(2.0f * s, 3.0f * s), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t e = __nv_cvt_float2_to_fp8x2(make_float2(4.0f * s, 6.0f * s), __NV_SATFINITE, __NV_E4M3);
-  return make_uint2(a | (b << 16), c | (e << 16));
-}
-
-// Eight e2m1 codes in the packed word layout of this kernel -> eight e4m3
-// bytes.  The magnitude of code k sits in bits 4k .. 4k + 2 (as in the MXFP4
-// byte stream, two codes a byte, low nibble first); the sign bits are moved at
-// packing (f4_pack_word) to bits 3, 11, 19, 27 for codes 0-3 and 7, 15, 23,
-// 31 for codes 4-7, so that one shift or none puts each on bit 7 of its
-// output byte.  The magnitudes go through the table: one byte permute per
-// four codes.
-__host__ __device__ inline uint32_t f4_pack_word(uint32_t w) {
-  uint32_t o = w & 0x77777777u;
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t sgn = (w >> (4 * k + 3)) & 1u;
-    const int at = k < 4 ? 8 * k + 3 : 8 * (k - 4) + 7;
-    o |= sgn << at;
-  }
-  return o;
-}
-__device__ __forceinline__ void f4x8_to_e4m3(uint32_t w, uint32_t l0, uint32_t l1, uint32_t& o0, uint32_t& o1) {
-  o0 = __byte_perm(l0, l1, w & 0x7777u) | ((w & 0x08080808u) << 4);
-  o1 = __byte_perm(l0, l1, (w >> 16) & 0x7777u) | (w & 0x80808080u);
-}
-
-// One ring stage of MXFP4 (two unit-matrices: gate and up, or two down
-// units; the second is stored only when two), this thread's weight row:
-// codes [4][128 rows][16] and the rows' d [128][4] of each matrix -> e4m3 in
-// the 32 tensor-memory columns from taddr and taddr + 32 (column c = four
-// contraction elements).  Whole warps (tcgen05.st); not inlined.
-__device__ __noinline__ void f4_expand_stage(const uint8_t* src, uint32_t taddr, int row, bool two) {
-  constexpr int MAT = 8192 + 512;
-  uint32_t l0[2][4], l1[2][4];
-  uint4 q[2][4];
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const uint32_t dd = *reinterpret_cast<const uint32_t*>(src + m * MAT + 8192 + row * 4);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      q[m][j] = *reinterpret_cast<const uint4*>(src + m * MAT + j * 2048 + row * 16);
-      const int d = (int)(int8_t)((dd >> (8 * j)) & 0xFFu);
-      f4_lut_fast(d, l0[m][j], l1[m][j]);
-      if (d < -5) {
-        const uint2 t = f4_lut_slow(d);
-        l0[m][j] = t.x;
-        l1[m][j] = t.y;
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t w[4] = {q[m][j].x, q[m][j].y, q[m][j].z, q[m][j].w};
-      uint32_t o[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) f4x8_to_e4m3(w[k], l0[m][j], l1[m][j], o[2 * k], o[2 * k + 1]);
-      if (m == 0 || two) tmem_st8(taddr + 32u * m + 8u * j, o);
-    }
-  }
 }
 
 // n, bf16 in the layout [H/8][8 rows][8], becomes the e4m3 B operand
@@ -276,8 +208,8 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
 
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_constant__ Params p) {
-  constexpr bool F4 = WT == W_FP4;                    // codes expanded by warps 4-7 first
-  constexpr uint32_t MAT = TqFmt<WT>::MAT_BYTES;      // one unit of one matrix in the ring
+  constexpr bool F4 = WT == W_FP4;                    // block-scaled MMAs on e2m1 codes
+  constexpr uint32_t MAT = TqFmt<WT>::MAT_BYTES;      // one unit of one matrix in HBM
   extern __shared__ __align__(1024) uint8_t smem[];
   const SmemLayout L(p.nst, p.slot_bytes, p.regA_bytes, p.ymax);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -297,18 +229,15 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     c->nu = 0;
     c->n_ready = 0;
     c->epoch = ld_relaxed(&p.sync->epoch);
+    c->live = live_rows(p);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], F4 ? 4 : 1);   // the expanding warps, or the MMAs' commit
+      mbar_init(&empty[s], 1);   // the MMAs' commit
     }
     for (uint32_t b = 0; b < kF8Acc; ++b) {
       mbar_init(&c->accfull[b], 1);
       mbar_init(&c->accempty[b], 4);
-    }
-    for (int b = 0; b < kF4Ab; ++b) {
-      mbar_init(&c->abfull[b], 4);
-      mbar_init(&c->abempty[b], 1);
     }
     mbar_init(&c->drain, 1);
     mbar_init(&c->bfull, 1);
@@ -323,6 +252,17 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   tc_fence_after();
   const uint32_t ep1 = c->epoch + 1u;
   const uint32_t tmem = c->tmem_base;
+  if (F4) {
+    // B's scale factors: 1.0 (e8m0 127) in every lane of their 4 columns,
+    // written before any MMA reads them (the barrier below orders them)
+    if (warp < 4) {
+      tmem_st4(tmem + ((uint32_t)(warp * 32) << 16) + kF4SfbCol, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   trace(p, 0, tid == 0);
 
   // a ring stage: one gate/up unit (gate, up) or two down units
@@ -336,16 +276,37 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       if (lane != 0) return;
       const int e = seg_expert(p, c, sg.x);
       const bool gu = sg.list != L_DN;
+      const int per = stage_units(sg);
+      if (F4) {
+        // unit-matrix m of the list's packed array: gate/up pairs (2 u, 2 u + 1)
+        // of unit u, or down unit u; each a box of 128 rows of the tensor map
+        const long long m0 = gu ? ((long long)(e * geo.nbi + sg.blk) * geo.upb_gu) * 2
+                                : (long long)(e * geo.nbh + sg.blk) * geo.upb_dn;
+        const CUtensorMap* map = gu ? &p.tm_gu : &p.tm_dn;
+        const uint8_t* sf = reinterpret_cast<const uint8_t*>(gu ? p.gsc : p.dsc);
+        for (int u = sg.k0; u < sg.k1; u += per) {
+          const uint32_t slot = s % p.nst, q = s / p.nst;
+          const int nm = gu ? 2 : min(per, sg.k1 - u);   // unit-matrices in this stage
+          const long long m = gu ? m0 + 2 * u : m0 + u;
+          if (ok && !dry && q > 0) ok = wait_bar(p, c, &empty[slot], (q - 1) & 1);
+          if (ok && !dry) {
+            uint8_t* dst = ring + (size_t)slot * p.slot_bytes;
+            mbar_arrive_expect_tx(&full[slot], (uint32_t)nm * (kF4BoxTx + kF4Sf));
+            for (int j = 0; j < nm; ++j) tma_load_2d(dst + j * kF4SmemMat, map, 0, (int)((m + j) * 128), &full[slot]);
+            tma_load_1d(dst + kF4SfOff, sf + m * kF4Sf, (uint32_t)nm * kF4Sf, &full[slot]);
+            issued = s + 1;
+          }
+          ++s;
+        }
+        return;
+      }
       const uint8_t* base = gu ? p.gu + (size_t)e * p.gu_estride + (size_t)sg.blk * geo.upb_gu * 2 * MAT
                                : p.dn + (size_t)e * p.dn_estride + (size_t)sg.blk * geo.upb_dn * MAT;
       const uint32_t ub = gu ? 2u * MAT : MAT;
-      // the epilogue's scales: FP8 block scales [unit][gate | up] or [unit]
-      // per block, MXFP4 row references [gate | up] or [rows] per block
+      // the epilogue's FP8 block scales [unit][gate | up] or [unit] per block
       const uint32_t sc_unit = gu ? 256u : 128u;
-      const float* sc_base = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : geo.upb_gu) * 256
-                                : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : geo.upb_dn) * 128;
-      if (F4 && !dry) prefetch_l2(sc_base, sc_unit * 4);
-      const int per = stage_units(sg);
+      const float* sc_base = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * geo.upb_gu * 256
+                                : p.dsc + (size_t)(e * geo.nbh + sg.blk) * geo.upb_dn * 128;
       for (int u = sg.k0; u < sg.k1; u += per) {
         const uint32_t slot = s % p.nst, q = s / p.nst;
         const uint32_t n = (uint32_t)min(per, sg.k1 - u), bytes = n * ub;
@@ -354,14 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           mbar_arrive_expect_tx(&full[slot], bytes);
           tma_load_1d(ring + (size_t)slot * p.slot_bytes, base + (size_t)u * ub, bytes, &full[slot]);
           issued = s + 1;
-          if (!F4) prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
+          prefetch_l2(sc_base + (size_t)u * sc_unit, n * sc_unit * 4);   // read by the epilogue
         }
         ++s;
       }
     };
     if (lane == 0) {
       const int e0 = (int)((long long)blockIdx.x * p.E / G), e1 = (int)((long long)(blockIdx.x + 1) * p.E / G);
-      prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
+      if (!p.dense) prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
       prefetch_l2_span(p.norm_w, (size_t)H * (p.norm_bf16 ? 2 : 4));
       prefetch_l2_span(p.bias, (size_t)p.E * 4);
     }
@@ -405,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     bool ok = true;
     if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
     ok = warp_ok(ok);
-    const uint32_t idesc = umma_idesc_e4m3(128, 16);
+    const uint32_t idesc = F4 ? umma_idesc_mx_e2m1_e4m3(128, 16) : umma_idesc_e4m3(128, 16);
     const uint32_t b_bytes = (uint32_t)I * 16u;
     // B (n, or a down expert's activations): [K/16][16 rows][16], 256 bytes
     // between K-neighbours, rows 8-15 128 bytes on; a unit is 2048 bytes
@@ -440,15 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
       }
       const int per = stage_units(sg);
       for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
-        // the stage's A: the ring slot (FP8) or the A buffer its codes were
-        // expanded into (MXFP4)
-        const uint32_t slot = F4 ? s % kF4Ab : s % p.nst, q = F4 ? s / kF4Ab : s / p.nst;
+        // the stage's A in the ring slot: FP8 unit-matrices of 16 KB in the
+        // no-swizzle core-matrix layout; MXFP4 unit-matrices of 16 KB with the
+        // 128-byte swizzle, their scale chunks behind them
+        const uint32_t slot = s % p.nst, q = s / p.nst;
         const int n = min(per, sg.k1 - u0);
-        if (lane == 0 && ok) ok = wait_bar(p, c, F4 ? &c->abfull[slot] : &full[slot], q & 1);
+        if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
         ok = warp_ok(ok);
         tc_fence_after();
-        const uint8_t* a_st = ring + (size_t)slot * p.slot_bytes;   // FP8
-        const uint32_t a_tm = tmem + (uint32_t)kF8TmemCols + 64u * slot;   // MXFP4
+        const uint8_t* a_st = ring + (size_t)slot * p.slot_bytes;
         if (sg.list == L_RGU && first_rgu) {
           first_rgu = false;
           trace(p, 13, lane == 0);
@@ -463,7 +424,16 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           tc_fence_after();
           if (ok) {
             if (F4) {
-              umma_unit_e4m3_tmem_a(tmem + 32u * buf, a_tm + 32u * j, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
+              // gate/up: gate at the slot start, up 16 KB on, scale chunks
+              // (gate, up) at kF4SfOff; down unit j at 16 KB * j, its chunk
+              // at kF4SfOff + 512 j.  Each accumulator buffer has 8 scale
+              // columns (gate 4 | up 4), free once its epilogue has read it.
+              const uint8_t* a = a_st + (size_t)(gu ? 0 : j) * kF4SmemMat;
+              const uint8_t* sf = a_st + kF4SfOff + (gu ? 0 : j) * kF4Sf;
+              const uint32_t sfa = tmem + kF4SfaCol + 8u * buf;
+              umma_unit_mx(tmem + 32u * buf, umma_desc_sw128(smem_u32(a), 1024u), bdesc + (uint64_t)(u * 128), 32u,
+                           idesc, sfa, umma_desc(smem_u32(sf), 16u, 128u), sfa + 4u,
+                           umma_desc(smem_u32(sf + kF4Sf), 16u, 128u), tmem + kF4SfbCol, gu);
             } else {
               const uint64_t da = umma_desc(smem_u32(a_st + (size_t)j * MAT), 2048u, 128u);
               umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
@@ -472,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           umma_commit_warp(&c->accfull[buf]);
           ++t;
         }
-        umma_commit_warp(F4 ? &c->abempty[slot] : &empty[slot]);
+        umma_commit_warp(&empty[slot]);
         ++s;
       }
     };
@@ -503,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   // ================================================================ prologue
   prologue_mix(p, c, regA, ep1);
   if (warp >= kCtlWarp0) {
-    control_warps(p, c, regA, ep1, false, !F4 && p.R <= 4);
+    control_warps(p, c, regA, ep1, false, p.R <= 4);
     return;
   }
   collapse_norm<true>(p, c, regA, ep1);
@@ -516,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
   trace(p, 3, tid == 0);
   // R <= 4: warps 4-7 take the top-k while warps 0-3 start on the shared
-  // expert's tiles, which need no routing (MXFP4: warps 4-7 expand)
-  const bool split = !F4 && p.R <= 4;
+  // expert's tiles, which need no routing
+  const bool split = p.R <= 4;
   if (!split || warp >= 4) route_rows(p, c, ep1, split);
   // the warps that need it agree on the expert list once
   int nu = 0;
@@ -559,13 +529,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
 #pragma unroll
       for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
       uint32_t v[16], w2[16];
-      // the units' scales (brought to L2 by the producer), two units ahead:
-      // FP8 block scales, or the MXFP4 row reference (the same every unit)
-      const float* sc = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * (F4 ? 1 : upb) * 256
-                           : p.dsc + (size_t)(e * geo.nbh + sg.blk) * (F4 ? 1 : upb) * 128;
-      const int us = F4 ? 0 : gu ? 256 : 128;
-      auto ld_g = [&](int u) { return u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
-      auto ld_u = [&](int u) { return gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
+      // the units' FP8 block scales (brought to L2 by the producer), two units
+      // ahead; MXFP4 block scales are applied inside the MMA (1 here)
+      const float* sc = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * upb * 256
+                           : p.dsc + (size_t)(e * geo.nbh + sg.blk) * upb * 128;
+      const int us = gu ? 256 : 128;
+      auto ld_g = [&](int u) { return F4 ? 1.f : u < sg.k1 ? __ldg(sc + (size_t)u * us + i) : 0.f; };
+      auto ld_u = [&](int u) { return F4 ? 1.f : gu && u < sg.k1 ? __ldg(sc + (size_t)u * us + 128 + i) : 0.f; };
       float sg0 = ld_g(sg.k0), su0 = ld_u(sg.k0), sg1 = ld_g(sg.k0 + 1), su1 = ld_u(sg.k0 + 1);
       if (gu) {
         for (int u = sg.k0; u < sg.k1; ++u) {
@@ -641,41 +611,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     }
     tc_fence_before();
     bar_arrive(kBarEnd, 5 * 32);   // the issuer may free the tensor memory
-  } else if (F4) {
-    // ======================================================= expanders
-    // warps 4-7, thread = weight row: each ring stage's codes into an A buffer
-    const int row = (warp - 4) * 32 + lane;
-    uint32_t s = 0;
-    bool cok = true;
-    auto expand = [&](const Seg& sg) {
-      const bool gu = sg.list != L_DN;
-      const int per = stage_units(sg);
-      for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
-        const uint32_t slot = s % p.nst, q = s / p.nst;
-        const uint32_t ab = s % kF4Ab, qa = s / kF4Ab;
-        const int n = min(per, sg.k1 - u0);
-        if (lane == 0 && cok) cok = wait_bar(p, c, &full[slot], q & 1);
-        if (lane == 0 && cok && qa > 0) cok = wait_bar(p, c, &c->abempty[ab], (qa - 1) & 1);
-        cok = __shfl_sync(0xffffffffu, (int)(cok && !c->dead), 0) != 0;
-        const uint8_t* src = ring + (size_t)slot * p.slot_bytes;
-        const uint32_t dst = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)kF8TmemCols + 64u * ab;
-        tc_fence_after();
-        if (cok) f4_expand_stage(src, dst, row, gu || n == 2);   // gate and up, or one or two down units
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&c->abfull[ab]);
-          mbar_arrive(&empty[slot]);
-        }
-        ++s;
-      }
-    };
-    tc_segments(p, geo, L_SGU, 0, expand);
-    tc_segments(p, geo, L_RGU, nu, expand);
-    tc_segments(p, geo, L_DN, nu, expand);
   }
-  // (FP8: warps 4-7 have no part in the main phase)
+  // warps 4-7 have no part in the main phase
 
   // ==================================================================== tail
   bar_sync(kBarCons, kCW * 32);

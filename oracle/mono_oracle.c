@@ -193,6 +193,7 @@ static int check_cfg(const orc_cfg* c) {
       c->inter <= 0 || c->rows < 0)
     return -1;
   if (c->w_dtype == ORC_FP8 && (c->hidden % 128 || c->inter % 128)) return -1;
+  if (c->dense && c->top_k != c->n_routed) return -1;
   if (c->w_dtype == ORC_MXFP4 && (c->hidden % 32 || c->inter % 32)) return -1;
   return 0;
 }
@@ -366,6 +367,56 @@ static int moe(const orc_cfg* c, const orc_weights* w, row_state* st) {
   return rc;
 }
 
+/* Dense layer: a SwiGLU MLP of width (E + 1) I whose weight rows are the E + 1
+ * slots' rows in slot order (gate / up row i = slot i / I, row i % I; down
+ * row h = the slots' down rows h side by side), evaluated as ONE MLP:
+ * g, u = n W (rounded to bf16 when round_bf16), act = silu(g) u, y = act W_down
+ * summed over the whole width, rounded like the routed + shared sum.  No
+ * router: the vLLM MonoKernel page ("Weights": a dense layer's MLP runs as
+ * six expert-shaped slices) computes this MLP with the same kernel, every
+ * slice taken with weight 1. */
+static int dense_mlp(const orc_cfg* c, const orc_weights* w, row_state* st) {
+  const int H = c->hidden, I = c->inter, E1 = c->n_routed + 1;
+  const int64_t W = (int64_t)E1 * I;
+  double* act;
+  int64_t ch;
+  for (int e = 0; e < E1; ++e)
+    if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) return -(100 + e);
+  act = (double*)malloc(sizeof(double) * (size_t)W);
+#pragma omp parallel for schedule(static)
+  for (ch = 0; ch < W; ++ch) {
+    double* row = (double*)malloc(sizeof(double) * (size_t)H);
+    const int e = (int)(ch / I), i = (int)(ch % I);
+    double g = 0.0, u = 0.0;
+    dec_weight_row(w->w_gate[e], w->s_gate ? w->s_gate[e] : NULL, c->w_dtype, i, H, row);
+    for (int h = 0; h < H; ++h) g += st->n[h] * row[h];
+    dec_weight_row(w->w_up[e], w->s_up ? w->s_up[e] : NULL, c->w_dtype, i, H, row);
+    for (int h = 0; h < H; ++h) u += st->n[h] * row[h];
+    if (c->round_bf16) {
+      g = rbf16(g);
+      u = rbf16(u);
+    }
+    act[ch] = g * sigmoid(g) * u;
+    free(row);
+  }
+#pragma omp parallel for schedule(static)
+  for (ch = 0; ch < H; ++ch) {
+    double* row = (double*)malloc(sizeof(double) * (size_t)W);
+    double acc = 0.0;
+    for (int e = 0; e < E1; ++e)
+      dec_weight_row(w->w_down[e], w->s_down ? w->s_down[e] : NULL, c->w_dtype, ch, I, row + (int64_t)e * I);
+    for (int64_t i = 0; i < W; ++i) acc += act[i] * row[i];
+    st->y[ch] = c->round_bf16 ? rbf16(acc) : acc;
+    free(row);
+  }
+  for (int j = 0; j < c->top_k; ++j) {   /* the slices, each with weight 1 */
+    st->idx[j] = j;
+    st->w[j] = 1.0f;
+  }
+  free(act);
+  return 0;
+}
+
 /* Step 13, the hyper-connection post / expand of the next residual streams:
  * out_i = sum_j comb_ij X_j + post_i y, rounded to the hc element type. */
 static void expand(const orc_cfg* c, const double* X, const double* comb, const double* post, const double* y,
@@ -424,6 +475,7 @@ static void taps_store(const orc_cfg* c, orc_taps* t, int r, const row_state* st
 static int row_steps(const orc_cfg* c, const orc_weights* w, const double* X, row_state* st, int route_only) {
   hc_mix_split(c, w, X, st);
   collapse_norm(c, w, X, st);
+  if (c->dense) return route_only ? 0 : dense_mlp(c, w, st);
   route(c, w, st);
   if (route_only) return 0;
   return moe(c, w, st);
@@ -517,8 +569,12 @@ EXPORT int orc_chain(const orc_cfg* c, int n_layers, const orc_weights* w, const
         }
         orc_sinkhorn(st.mix + 2 * S, S, c->sinkhorn_iters, st.comb);
         collapse_norm(c, w + l, X, &st);
-        route(c, w + l, &st);
-        rc = moe(c, w + l, &st);
+        if (c->dense) {
+          rc = dense_mlp(c, w + l, &st);
+        } else {
+          route(c, w + l, &st);
+          rc = moe(c, w + l, &st);
+        }
       }
       if (!rc) {
         /* the last layer's expand, closed at the tail */
@@ -534,4 +590,101 @@ EXPORT int orc_chain(const orc_cfg* c, int n_layers, const orc_weights* w, const
   free(X);
   free(Xn);
   return rc;
+}
+
+/* ------------------------------------------------- within-layer boundary -- */
+
+/* The attention sublayer's output closed into this FFN's opening pass:
+ * X_i = sum_j attn_comb_ij Xa_j + attn_post_i y_attn, rounded to the hc
+ * element type (the attention sublayer's own post / expand), then this
+ * layer's steps 1-13 on X.  Written in the fused form: the expand and, in the
+ * same pass over (s, h), the square sum and the mix products; the mix is then
+ * scaled by rho as in the unfused mix (SGLang "[DeepSeek-V4] Add
+ * mhc_fused_post_pre kernel", Modifications: the attention's hc_post fused
+ * with the FFN's hc_pre inside one layer).  x_attn [R][S][H] and y_attn [R][H]
+ * in hc_dtype, attn_post [R][S] and attn_comb [R][S][S] fp32.  x_out, when
+ * not NULL, receives the materialised X [R][S][H] in hc_dtype. */
+EXPORT int orc_layer_pending(const orc_cfg* c, const orc_weights* w, const void* x_attn, const float* attn_post,
+                             const float* attn_comb, const void* y_attn, void* hc_out, void* x_out, orc_taps* t) {
+  const int S = c->hc, H = c->hidden, M = 2 * c->hc + c->hc * c->hc;
+  const int64_t SH = (int64_t)S * H;
+  int rc = 0;
+  double* Xa;
+  double* X;
+  double* y;
+  double* out;
+  row_state st;
+  if (check_cfg(c) || S > 8) return -1;
+  Xa = (double*)malloc(sizeof(double) * (size_t)SH);
+  X = (double*)malloc(sizeof(double) * (size_t)SH);
+  out = (double*)malloc(sizeof(double) * (size_t)SH);
+  y = (double*)malloc(sizeof(double) * (size_t)H);
+  state_alloc(c, &st);
+  for (int r = 0; r < c->rows && !rc; ++r) {
+    double pcomb[64], ppost[8], ss = 0.0, acc[64];
+    for (int64_t i = 0; i < SH; ++i) Xa[i] = dec_act(x_attn, (int64_t)r * SH + i, c->hc_dtype);
+    for (int h = 0; h < H; ++h) y[h] = dec_act(y_attn, (int64_t)r * H + h, c->hc_dtype);
+    for (int i = 0; i < S * S; ++i) pcomb[i] = attn_comb[(int64_t)r * S * S + i];
+    for (int i = 0; i < S; ++i) ppost[i] = attn_post[(int64_t)r * S + i];
+    expand(c, Xa, pcomb, ppost, y, X);
+    for (int64_t i = 0; i < SH; ++i) ss += X[i] * X[i];
+    for (int col = 0; col < M; ++col) {
+      acc[col] = 0.0;
+      for (int64_t i = 0; i < SH; ++i) acc[col] += X[i] * (double)w->mix_w[i * M + col];
+    }
+    st.rho = 1.0 / sqrt(ss / (double)SH + c->rms_eps);
+    for (int col = 0; col < M; ++col) st.mix[col] = st.rho * acc[col];
+    for (int i = 0; i < S; ++i) {
+      st.pre[i] = sigmoid(st.mix[i]) + c->pre_eps;
+      st.post[i] = c->post_mult * sigmoid(st.mix[S + i]);
+    }
+    orc_sinkhorn(st.mix + 2 * S, S, c->sinkhorn_iters, st.comb);
+    collapse_norm(c, w, X, &st);
+    if (c->dense) {
+      rc = dense_mlp(c, w, &st);
+    } else {
+      route(c, w, &st);
+      rc = moe(c, w, &st);
+    }
+    taps_store(c, t, r, &st, !rc);
+    if (rc) break;
+    if (x_out)
+      for (int64_t i = 0; i < SH; ++i) enc_act(x_out, (int64_t)r * SH + i, c->hc_dtype, X[i]);
+    expand(c, X, st.comb, st.post, st.y, out);
+    for (int64_t i = 0; i < SH; ++i) enc_act(hc_out, (int64_t)r * SH + i, c->hc_dtype, out[i]);
+  }
+  state_free(&st);
+  free(Xa);
+  free(X);
+  free(out);
+  free(y);
+  return rc;
+}
+
+/* The expand alone, per row: x_out_i = sum_j comb_ij x_in_j + post_i y,
+ * rounded to the hc element type (the op-by-op form of a sublayer's post). */
+EXPORT int orc_expand(const orc_cfg* c, const void* x_in, const float* post, const float* comb, const void* y,
+                      void* x_out) {
+  const int S = c->hc, H = c->hidden;
+  const int64_t SH = (int64_t)S * H;
+  double* Xa;
+  double* X;
+  double* yy;
+  if (check_cfg(c) || S > 8) return -1;
+  Xa = (double*)malloc(sizeof(double) * (size_t)SH);
+  X = (double*)malloc(sizeof(double) * (size_t)SH);
+  yy = (double*)malloc(sizeof(double) * (size_t)H);
+  for (int r = 0; r < c->rows; ++r) {
+    double pc[64], pp[8];
+    for (int64_t i = 0; i < SH; ++i) Xa[i] = dec_act(x_in, (int64_t)r * SH + i, c->hc_dtype);
+    for (int h = 0; h < H; ++h) yy[h] = dec_act(y, (int64_t)r * H + h, c->hc_dtype);
+    for (int i = 0; i < S * S; ++i) pc[i] = comb[(int64_t)r * S * S + i];
+    for (int i = 0; i < S; ++i) pp[i] = post[(int64_t)r * S + i];
+    expand(c, Xa, pc, pp, yy, X);
+    for (int64_t i = 0; i < SH; ++i) enc_act(x_out, (int64_t)r * SH + i, c->hc_dtype, X[i]);
+  }
+  free(Xa);
+  free(X);
+  free(yy);
+  return 0;
 }

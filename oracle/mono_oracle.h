@@ -56,6 +56,7 @@ typedef struct {
   int round_bf16; /* 1: round to bf16 after collapse, after norm, gate/up, routed+shared sum */
   int sinkhorn_iters;
   double rms_eps, pre_eps, post_mult, route_scale, denom_clamp;
+  int dense;      /* 1: no router; a dense SwiGLU MLP of width (E + 1) I over all slots (top_k = E) */
 } orc_cfg;
 
 /* Logical layouts (row-major):
@@ -113,6 +114,17 @@ int orc_route(const orc_cfg* cfg, const orc_weights* w, const void* hc_in, orc_t
  * expand is closed at the tail. */
 int orc_chain(const orc_cfg* cfg, int n_layers, const orc_weights* w, const void* hc_in, void* hc_out,
               int deferred);
+
+/* Within-layer boundary: the attention sublayer's pending post / expand
+ * (x_attn [R][S][H] and y_attn [R][H] in hc_dtype, attn_post [R][S] and
+ * attn_comb [R][S][S] fp32) closed in this layer's opening pass, then the
+ * layer.  x_out (may be NULL): the materialised residual streams. */
+int orc_layer_pending(const orc_cfg* cfg, const orc_weights* w, const void* x_attn, const float* attn_post,
+                      const float* attn_comb, const void* y_attn, void* hc_out, void* x_out, orc_taps* taps);
+
+/* The expand alone (op by op): x_out_i = sum_j comb_ij x_in_j + post_i y. */
+int orc_expand(const orc_cfg* cfg, const void* x_in, const float* post, const float* comb, const void* y,
+               void* x_out);
 
 /* Building blocks, exported for the oracle's own pins. */
 void orc_sinkhorn(const double* logits, int s, int iters, double* comb);

@@ -41,7 +41,8 @@ def build():
 class Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "hc", "n_routed", "top_k", "inter", "rows", "hc_dtype",
                                             "norm_dtype", "w_dtype", "round_bf16", "sinkhorn_iters")] + \
-               [(n, ctypes.c_double) for n in ("rms_eps", "pre_eps", "post_mult", "route_scale", "denom_clamp")]
+               [(n, ctypes.c_double) for n in ("rms_eps", "pre_eps", "post_mult", "route_scale", "denom_clamp")] + \
+               [("dense", ctypes.c_int)]
 
 
 class Weights(ctypes.Structure):
@@ -68,6 +69,9 @@ def lib():
         L.orc_layer.argtypes = [ctypes.POINTER(Cfg), ctypes.POINTER(Weights), vp, vp, ctypes.POINTER(Taps)]
         L.orc_route.argtypes = [ctypes.POINTER(Cfg), ctypes.POINTER(Weights), vp, ctypes.POINTER(Taps)]
         L.orc_chain.argtypes = [ctypes.POINTER(Cfg), ctypes.c_int, ctypes.POINTER(Weights), vp, vp, ctypes.c_int]
+        L.orc_layer_pending.argtypes = [ctypes.POINTER(Cfg), ctypes.POINTER(Weights), vp, vp, vp, vp, vp, vp,
+                                        ctypes.POINTER(Taps)]
+        L.orc_expand.argtypes = [ctypes.POINTER(Cfg), vp, vp, vp, vp, vp]
         L.orc_sinkhorn.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
         L.orc_topk.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp]
         L.orc_dec_bf16.argtypes = [ctypes.c_uint16]
@@ -95,7 +99,7 @@ def make_cfg(wl, rows=None):
                rows=wl.rows if rows is None else rows, hc_dtype=_DT[wl.hc_dtype], norm_dtype=_DT[wl.norm_dtype],
                w_dtype=_DT[wl.w_dtype], round_bf16=int(wl.round_bf16), sinkhorn_iters=wl.sinkhorn_iters,
                rms_eps=wl.rms_eps, pre_eps=wl.pre_eps, post_mult=wl.post_mult, route_scale=wl.route_scale,
-               denom_clamp=wl.denom_clamp)
+               denom_clamp=wl.denom_clamp, dense=int(wl.dense))
 
 
 class LayerWeights:
@@ -184,6 +188,37 @@ def layer(wl, lw: LayerWeights, hc_in):
     if rc != 0:
         raise RuntimeError(f"orc_layer failed: {rc}")
     return out, taps
+
+
+def layer_pending(wl, lw: LayerWeights, x_attn, attn_post, attn_comb, y_attn):
+    """One layer opened by the attention sublayer's pending expand: returns
+    (hc_out raw array, materialised X raw array, taps)."""
+    rows = x_attn.shape[0]
+    cfg = make_cfg(wl, rows)
+    taps = TapSet(wl, rows)
+    x_attn = np.ascontiguousarray(x_attn)
+    y_attn = np.ascontiguousarray(y_attn)
+    post = np.ascontiguousarray(attn_post, np.float32)
+    comb = np.ascontiguousarray(attn_comb, np.float32)
+    out = _hc_buf(wl, rows)
+    x = _hc_buf(wl, rows)
+    rc = lib().orc_layer_pending(ctypes.byref(cfg), ctypes.byref(lw.struct), _p(x_attn), _p(post), _p(comb),
+                                 _p(y_attn), _p(out), _p(x), ctypes.byref(taps.struct))
+    if rc != 0:
+        raise RuntimeError(f"orc_layer_pending failed: {rc}")
+    return out, x, taps
+
+
+def expand(wl, x_in, post, comb, y):
+    """x_out_i = sum_j comb_ij x_in_j + post_i y per row, in the hc element type."""
+    rows = x_in.shape[0]
+    cfg = make_cfg(wl, rows)
+    out = _hc_buf(wl, rows)
+    rc = lib().orc_expand(ctypes.byref(cfg), _p(np.ascontiguousarray(x_in)), _p(np.ascontiguousarray(post, np.float32)),
+                          _p(np.ascontiguousarray(comb, np.float32)), _p(np.ascontiguousarray(y)), _p(out))
+    if rc != 0:
+        raise RuntimeError(f"orc_expand failed: {rc}")
+    return out
 
 
 def chain(wl, lws, hc_in, deferred):

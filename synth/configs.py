@@ -40,6 +40,7 @@ class Workload:
     denom_clamp: float = 1e-20
     sinkhorn_iters: int = 20
     mx_spread: int = 0   # MXFP4: block magnitudes within a row span up to 2^mx_spread
+    dense: bool = False  # a dense MLP of width (n_routed + 1) * inter over every slot, no router
 
     def with_(self, **kw):
         return replace(self, **kw)
@@ -66,6 +67,11 @@ FLASH_MXFP4_CHAIN4_R8 = _flash("v41flash-mxfp4-chain4-r8", 8, 4, "mxfp4", n_laye
 
 FULL = [TINY_FP32, FLASH_BF16_R1, FLASH_BF16_R6, FLASH_BF16_R8, FLASH_FP8_R4, FLASH_MXFP4_CHAIN4_R8]
 
+# a dense layer of the same model family: SwiGLU width 6 x 2048 = 12288 run as
+# six expert-shaped slices (five routed slots and the shared slot), weight 1
+DENSE6_BF16_R1 = Workload("v41flash-dense6-bf16-r1", hidden=5120, n_routed=5, top_k=5, inter=2048, rows=1, seed=7,
+                          hc_dtype="bf16", norm_dtype="bf16", w_dtype="bf16", round_bf16=True, dense=True)
+
 
 def scaled(w: Workload, hidden=1024, n_routed=32, top_k=4, inter=512, **kw) -> Workload:
     """A smaller copy of a workload that the oracle finishes in seconds while
@@ -74,4 +80,4 @@ def scaled(w: Workload, hidden=1024, n_routed=32, top_k=4, inter=512, **kw) -> W
                    inter=inter, **kw)
 
 
-BY_NAME = {w.name: w for w in FULL}
+BY_NAME = {w.name: w for w in FULL + [DENSE6_BF16_R1]}

@@ -22,6 +22,7 @@ CPU_SO = os.path.join(HERE, "libsynth_cpu.so")
 GPU_SO = os.path.join(HERE, "libsynth_gpu.so")
 
 HC_IN, MIX_W, NORM_W, ROUTER_W, ROUTER_BIAS, GATE, UP, DOWN = range(1, 9)
+ATTN_X, ATTN_POST, ATTN_COMB, ATTN_Y = range(9, 13)
 _OUT = {"f32": 0, "bf16": 1, "f64": 2}
 
 
@@ -134,6 +135,26 @@ def cpu_hc_in(w: Workload):
     return cpu_fill(w.seed, 0, HC_IN, 0, (w.rows, w.hc, w.hidden), 0, 0.0, 1.0, w.hc_dtype)
 
 
+def attn_specs(w: Workload):
+    """(kind, shape, dist, p0, p1, element type) of the attention sublayer's
+    pending state that opens a layer at the within-layer boundary: the
+    residual streams before attention N(0, 1), its post U(0, 2), its comb
+    U(0, 0.5) (any matrix: the boundary does not assume a doubly stochastic
+    one), its output N(0, 1)."""
+    R, S, H = w.rows, w.hc, w.hidden
+    return {
+        "x": (ATTN_X, (R, S, H), 0, 0.0, 1.0, w.hc_dtype),
+        "post": (ATTN_POST, (R, S), 1, 0.0, 2.0, "f32"),
+        "comb": (ATTN_COMB, (R, S, S), 1, 0.0, 0.5, "f32"),
+        "y": (ATTN_Y, (R, H), 0, 0.0, 1.0, w.hc_dtype),
+    }
+
+
+def cpu_attn_pending(w: Workload):
+    return {k: cpu_fill(w.seed, 0, kind, 0, shape, dist, p0, p1, t)
+            for k, (kind, shape, dist, p0, p1, t) in attn_specs(w).items()}
+
+
 def cpu_dense(w: Workload, layer: int):
     out = {}
     for name, (kind, shape, dist, p0, p1, t) in tensor_specs(w, layer).items():
@@ -220,6 +241,15 @@ def gpu_hc_in(w: Workload, device="cuda"):
     import torch
     t = torch.empty((w.rows, w.hc, w.hidden), dtype=_torch_dtype(w.hc_dtype), device=device)
     return gpu_fill_(t, w.seed, 0, HC_IN, 0, 0, 0.0, 1.0, w.hc_dtype)
+
+
+def gpu_attn_pending(w: Workload, device="cuda"):
+    import torch
+    out = {}
+    for k, (kind, shape, dist, p0, p1, t) in attn_specs(w).items():
+        x = torch.empty(shape, dtype=_torch_dtype(t), device=device)
+        out[k] = gpu_fill_(x, w.seed, 0, kind, 0, dist, p0, p1, t)
+    return out
 
 
 def gpu_dense(w: Workload, layer: int, device="cuda"):

@@ -48,7 +48,11 @@ enum {
   SYNTH_ROUTER_BIAS = 5,
   SYNTH_GATE = 6,
   SYNTH_UP = 7,
-  SYNTH_DOWN = 8
+  SYNTH_DOWN = 8,
+  SYNTH_ATTN_X = 9,     /* the attention sublayer's pending state (within-layer boundary) */
+  SYNTH_ATTN_POST = 10,
+  SYNTH_ATTN_COMB = 11,
+  SYNTH_ATTN_Y = 12
 };
 
 SYNTH_FN uint64_t synth_mix64(uint64_t z) {

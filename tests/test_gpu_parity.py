@@ -163,16 +163,17 @@ def test_cuda_core_mxfp4_hidden_not_multiple_of_128():
     CUDA-core kernel."""
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=411, hidden=1056, inter=544, rows=3)
     run = LayerRun(wl)
-    assert run.plan.info()["ring_slot_bytes"] != 2 * (8192 + 512)
+    assert run.plan.info()["ring_slot_bytes"] != 2 * 16384 + 2 * 512   # not the tensor-core layout
     run.step()
     _check_layer(wl, run, list(range(wl.rows)))
     run.close()
 
 
 def test_scaled_mxfp4_wide_block_spread():
-    """MXFP4 rows whose block scales span up to 2^20: the tensor-core path's
-    e4m3 expansion relative to each row's largest scale takes its table, its
-    one-by-one (subnormal) and its rounded branches."""
+    """MXFP4 rows whose block scales span up to 2^20: the tensor-core path
+    applies each 32-element block's e8m0 scale inside the block-scaled MMA,
+    so every block keeps its own exponent, however far from its row's
+    largest."""
     wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=431, mx_spread=20)
     run = LayerRun(wl)
     run.step()

@@ -428,3 +428,82 @@ def test_deferred_post_chain_is_bit_identical(wdt):
     for lw in lws:
         x, _ = O.layer(wl, lw, x)
     assert np.array_equal(a, x)
+
+
+# ------------------------------------------------- within-layer boundary --
+
+def _pending_case(wdt, hc="bf16"):
+    wl = C.scaled(C.FLASH_BF16_R8, hidden=128, n_routed=8, top_k=2, inter=64, rows=3, w_dtype=wdt, seed=77)
+    if hc == "f32":
+        wl = wl.with_(hc_dtype="f32", norm_dtype="f32", round_bf16=False)
+    lw = O.LayerWeights(wl, S.cpu_dense(wl, 0), all_experts(wl, 0))
+    return wl, lw, S.cpu_attn_pending(wl)
+
+
+@pytest.mark.parametrize("wdt, hc", [("bf16", "bf16"), ("mxfp4", "bf16"), ("f32", "f32")])
+def test_pending_boundary_equals_expand_then_layer(wdt, hc):
+    """The attention sublayer's expand closed in the FFN's opening pass (mix
+    products and square sum taken in the same pass) equals closing it first
+    and running the layer on the result, bit for bit."""
+    wl, lw, a = _pending_case(wdt, hc)
+    out, x, t = O.layer_pending(wl, lw, a["x"], a["post"], a["comb"], a["y"])
+    x_ref = O.expand(wl, a["x"], a["post"], a["comb"], a["y"])
+    assert np.array_equal(x, x_ref)
+    out_ref, t_ref = O.layer(wl, lw, x_ref)
+    assert np.array_equal(out, out_ref)
+    assert np.array_equal(t.mix, t_ref.mix) and np.array_equal(t.idx, t_ref.idx) and np.array_equal(t.y, t_ref.y)
+
+
+def test_pending_boundary_special_cases():
+    """comb = identity and post = 0 leave the streams as they are (the layer
+    then sees x_attn itself); comb = 0 and post = 1 give every stream the
+    attention output y (rounded to the stream type)."""
+    wl, lw, a = _pending_case("bf16")
+    R, S_ = wl.rows, wl.hc
+    eye = np.broadcast_to(np.eye(S_, dtype=np.float32), (R, S_, S_)).copy()
+    out, x, _ = O.layer_pending(wl, lw, a["x"], np.zeros((R, S_), np.float32), eye, a["y"])
+    assert np.array_equal(x, a["x"])
+    assert np.array_equal(out, O.layer(wl, lw, a["x"])[0])
+    x2 = O.expand(wl, a["x"], np.ones((R, S_), np.float32), np.zeros((R, S_, S_), np.float32), a["y"])
+    assert np.array_equal(x2, np.broadcast_to(a["y"][:, None, :], x2.shape))
+
+
+# ------------------------------------------------------------- dense layer --
+
+def test_dense_layer_is_one_swiglu_mlp_over_every_slot():
+    """A dense layer (no router): y = down(silu(gate n) * up n) with the
+    E + 1 slots' gate / up rows stacked and their down rows side by side,
+    one MLP of width (E + 1) I, against torch.nn.functional in float64; the
+    taps show every slice with weight 1."""
+    wl = tiny(n_routed=5, top_k=5, rows=2, dense=True)
+    hc, dense, ex = layer_inputs(wl, experts="all")
+    out, t = O.layer(wl, O.LayerWeights(wl, dense, ex), hc)
+    n = torch.from_numpy(t.n)
+    slots = range(wl.n_routed + 1)
+    g = torch.cat([torch.from_numpy(ex[e]["gate"][0].astype(np.float64)) for e in slots], 0)
+    u = torch.cat([torch.from_numpy(ex[e]["up"][0].astype(np.float64)) for e in slots], 0)
+    d = torch.cat([torch.from_numpy(ex[e]["down"][0].astype(np.float64)) for e in slots], 1)
+    y = F.linear(F.silu(F.linear(n, g)) * F.linear(n, u), d)
+    assert torch.allclose(torch.from_numpy(t.y), y, rtol=1e-12, atol=1e-14)
+    assert t.idx.tolist() == [list(range(5))] * 2 and np.all(t.w == 1.0)
+
+
+def test_dense_layer_with_bf16_rounding_equals_routed_slices_of_weight_one():
+    """With the bf16 roundings, the dense MLP equals the same slots taken as
+    experts with weight 1 (the routed + shared sum of the MoE step written
+    out by hand): bf16 round of g and u is per element, so splitting the
+    width changes only the order of the double-precision sum."""
+    wl = tiny(n_routed=5, top_k=5, rows=2, dense=True, hc_dtype="bf16", norm_dtype="bf16", w_dtype="bf16",
+              round_bf16=True)
+    hc, dense, ex = layer_inputs(wl, experts="all")
+    _, t = O.layer(wl, O.LayerWeights(wl, dense, ex), hc)
+    n = t.n
+    y = np.zeros_like(t.y)
+    for e in range(wl.n_routed + 1):
+        m = f32_of(wl, ex[e])
+        rb = lambda v: torch.from_numpy(v).to(torch.float32).to(torch.bfloat16).double().numpy()
+        gg, uu = rb(n @ m["gate"].T), rb(n @ m["up"].T)
+        y += (gg / (1 + np.exp(-gg)) * uu) @ m["down"].T
+    yb = torch.from_numpy(y).to(torch.float32).to(torch.bfloat16).double().numpy()
+    assert np.mean(yb == t.y) > 0.99
+    assert np.allclose(yb, t.y, rtol=2 ** -7, atol=1e-6)
