@@ -393,6 +393,10 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     need(cfg.hidden % m == 0, "hidden must be a multiple of " + std::to_string(m) + " for this expert format");
     need(cfg.inter % m == 0, "inter must be a multiple of " + std::to_string(m) + " for this expert format");
     need(cfg.hidden % 8 == 0 && cfg.inter % 8 == 0, "hidden and inter must be multiples of 8");
+    // MXFP4 on the tensor cores keeps one B-scale column per 128 of inter
+    need(!(dt == MONO_MXFP4 && cfg.round_bf16 && cfg.hidden % 128 == 0 && cfg.inter % 128 == 0) ||
+             cfg.inter <= kF4MaxI,
+         "MXFP4 on the tensor cores takes inter <= " + std::to_string(kF4MaxI));
   }
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) why += "no CUDA device\n";
@@ -469,7 +473,9 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   const int smem_max = prop.sharedMemPerBlockOptin;
   SmemLayout L0(0, p->slot_bytes, p->regA_bytes, p->ymax);
   long long room = (long long)smem_max - (long long)L0.ring - 2 * 8 * 16 - kRingGuard;
-  p->nst = (int)std::min<long long>(16, room / p->slot_bytes);
+  // MXFP4 on the tensor cores: each ring slot has its own A scale columns in
+  // tensor memory, and there are columns for kF4MaxSlots of them
+  p->nst = (int)std::min<long long>(p->tq && dt == MONO_MXFP4 ? kF4MaxSlots : 16, room / p->slot_bytes);
   if (p->nst < 2) {
     std::string m = "shared memory: " + std::to_string(smem_max) + " bytes leave room for " + std::to_string(p->nst) +
                     " ring stages of " + std::to_string(p->slot_bytes) + " bytes (need 2)";

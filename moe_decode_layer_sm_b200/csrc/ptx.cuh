@@ -275,56 +275,80 @@ __host__ __device__ constexpr uint32_t umma_idesc_mx_e2m1_e4m3(int m, int n) {
 }
 
 // One 128 x 128 unit of e2m1 weights (A, 128-byte-swizzled K-major, in
-// shared memory) against e4m3 B, with the unit's 4 x 128 e8m0 block scales
-// in tensor memory at sfa (4 columns, byte j = K-block j) and B's scales at
-// sfb: tcgen05.cp brings the scale chunk from shared memory (sf_smem) first,
-// then 4 block-scaled MMAs of K = 32, the first overwriting D.  pair: a
-// second A (up) 16384 bytes on, its scales at sfa2 from sf_smem2, into d + 16.
-// One elected lane of a converged warp issues all of it, in order.
+// shared memory) against e4m3 B, block-scaled: 4 MMAs of K = 32.  The unit's
+// 4 x 128 e8m0 A scales are first copied from shared memory (sfd, a chunk of
+// 512 bytes) to tensor memory at sfa by tcgen05.cp (32x128b, all four lane
+// quarters); K-step j then reads byte j there.  B's scales are at sfb: with
+// bstep set, K-step j reads byte j (a scale per K-block), else every K-step
+// reads byte bsel (one scale for the unit).  acc: the first K-step adds to D
+// (else it overwrites D).  pair: a second A (up) 16384 bytes on, its scales
+// from sfd2 to sfa2, into d + 16.  One elected lane of a converged warp issues
+// all of it, in order.
 __device__ __forceinline__ void umma_unit_mx(uint32_t d, uint64_t da, uint64_t db, uint32_t db_step, uint32_t idesc,
                                              uint32_t sfa, uint64_t sfd, uint32_t sfa2, uint64_t sfd2, uint32_t sfb,
-                                             bool pair) {
+                                             bool bstep, uint32_t bsel, bool acc, bool pair) {
+  // per K-step: A scale byte +1 (idesc bits 29-30, address bits 30-31); B
+  // scale byte +1 when bstep (idesc bits 4-5, address bits 30-31)
+  const uint32_t istep = 0x20000000u | (bstep ? 0x10u : 0u);
+  const uint32_t bastep = bstep ? 0x40000000u : 0u;
+  const uint32_t i0 = idesc | ((bstep ? 0u : bsel) << 4);
+  const uint32_t b0 = sfb | ((bstep ? 0u : bsel) << 30);
   if (pair) {
     asm volatile(
-        "{\n .reg .pred e, t, f;\n .reg .b32 rx, d1, i, s0, s1;\n .reg .b64 a0, a1, b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, d1, i, s0, s1, sb;\n .reg .b64 a0, a1, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, %11, 0;\n"
         " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n"
         " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%7], %8;\n"
         " mov.b64 a0, %1;\n add.u64 a1, %1, 1024;\n add.u32 d1, %0, 16;\n mov.b64 b, %2;\n"
-        " mov.b32 i, %4;\n mov.b32 s0, %5;\n mov.b32 s1, %7;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], f;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], f;\n"
+        " mov.b32 i, %4;\n mov.b32 s0, %5;\n mov.b32 s1, %7;\n mov.b32 sb, %9;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], f;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [sb], f;\n"
         " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
-        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
+        " add.u32 i, i, %10;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n add.u32 sb, sb, %12;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [sb], t;\n"
         " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
-        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
+        " add.u32 i, i, %10;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n add.u32 sb, sb, %12;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [sb], t;\n"
         " add.u64 a0, a0, 2;\n add.u64 a1, a1, 2;\n add.u64 b, b, %3;\n"
-        " add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%9], t;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [%9], t;\n"
-        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(sfa), "l"(sfd), "r"(sfa2), "l"(sfd2),
-        "r"(sfb)
+        " add.u32 i, i, %10;\n add.u32 s0, s0, 0x40000000;\n add.u32 s1, s1, 0x40000000;\n add.u32 sb, sb, %12;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [d1], a1, b, i, [s1], [sb], t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(i0), "r"(sfa), "l"(sfd), "r"(sfa2), "l"(sfd2),
+        "r"(b0), "r"(istep), "r"((uint32_t)acc), "r"(bastep)
         : "memory");
   } else {
     asm volatile(
-        "{\n .reg .pred e, t, f;\n .reg .b32 rx, i, s0;\n .reg .b64 a0, b;\n"
-        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, 0, 0;\n"
+        "{\n .reg .pred e, t, f;\n .reg .b32 rx, i, s0, sb;\n .reg .b64 a0, b;\n"
+        " elect.sync rx|e, 0xffffffff;\n setp.eq.b32 t, 0, 0;\n setp.ne.b32 f, %9, 0;\n"
         " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n"
-        " mov.b64 a0, %1;\n mov.b64 b, %2;\n mov.b32 i, %4;\n mov.b32 s0, %5;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], f;\n"
-        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
-        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
-        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, 0x20000000;\n add.u32 s0, s0, 0x40000000;\n"
-        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [%7], t;\n"
-        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(idesc), "r"(sfa), "l"(sfd), "r"(sfb)
+        " mov.b64 a0, %1;\n mov.b64 b, %2;\n mov.b32 i, %4;\n mov.b32 s0, %5;\n mov.b32 sb, %7;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], f;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, %8;\n add.u32 s0, s0, 0x40000000;\n"
+        " add.u32 sb, sb, %10;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, %8;\n add.u32 s0, s0, 0x40000000;\n"
+        " add.u32 sb, sb, %10;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        " add.u64 a0, a0, 2;\n add.u64 b, b, %3;\n add.u32 i, i, %8;\n add.u32 s0, s0, 0x40000000;\n"
+        " add.u32 sb, sb, %10;\n"
+        " @e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], a0, b, i, [s0], [sb], t;\n"
+        "}\n" ::"r"(d), "l"(da), "l"(db), "l"((uint64_t)db_step), "r"(i0), "r"(sfa), "l"(sfd), "r"(b0),
+        "r"(istep), "r"((uint32_t)acc), "r"(bastep)
         : "memory");
   }
+}
+
+// tcgen05.cp of one 512-byte scale chunk (32 rows x 16 bytes in shared memory)
+// to 4 tensor-memory columns at taddr in every lane quarter, by one elected
+// lane of a converged warp
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sfd) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
+      " @e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n}\n" ::"r"(taddr),
+      "l"(sfd)
+      : "memory");
 }
 
 // 32 lanes x 4 consecutive 32-bit columns from registers (thread l of the
@@ -344,6 +368,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int c0, 
       "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+
+// tcgen05.ld of 32 lanes x 16 columns without the wait (pair it with
+// tmem_ld_wait before the registers are used)
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void bar_arrive(int id, int threads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");

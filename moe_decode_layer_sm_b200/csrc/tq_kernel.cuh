@@ -59,10 +59,13 @@ template <> struct TqFmt<W_FP4> {
 
 constexpr int kF8TmemCols = 128;   // four accumulators of 32 columns (gate 16 | up 16)
 constexpr int kF4TmemCols = 256;   // the accumulators, then the scale factors
-constexpr uint32_t kF4SfaCol = 128;   // A scale factors: 8 columns per accumulator (gate 4 | up 4)
-constexpr uint32_t kF4SfbCol = 160;   // B scale factors: 4 columns of 1.0
+constexpr uint32_t kF4SfaCol = 128;   // A scale factors: 8 columns per ring slot (gate 4 | up 4, or 2 down units)
+constexpr uint32_t kF4SfbNCol = 160;  // B scale factors of n (gate/up): 4 columns
+constexpr uint32_t kF4SfbDnCol = 192; // B scale factors of a down expert's activations: I / 128 columns
+constexpr int kF4MaxSlots = 4;        // ring slots whose A scales fit in tensor memory
+constexpr int kF4MaxI = (kF4TmemCols - (int)kF4SfbDnCol) * 128;   // one down-scale column per 128 of I
+constexpr int kF4Sf = 512;         // one scale chunk (tcgen05.cp 32x128b source)
 constexpr int kF4SmemMat = 16384;  // one MXFP4 unit-matrix in the ring (16-byte slot per 16 codes)
-constexpr int kF4Sf = 512;         // its scale chunk
 constexpr int kF4SfOff = 2 * kF4SmemMat;   // the scale chunks of a stage, after its two unit-matrices
 // transaction bytes one unit-matrix box of the tensor map counts on its
 // mbarrier: the bytes of codes it writes (the 8-byte gaps of the 16-byte
@@ -70,11 +73,15 @@ constexpr int kF4SfOff = 2 * kF4SmemMat;   // the scale chunks of a stage, after
 constexpr uint32_t kF4BoxTx = kF4SmemMat / 2;
 constexpr uint32_t kF8Acc = 4;
 static_assert(kF8Acc <= (uint32_t)kMaxAcc, "accumulator barriers");
-static_assert(kF4SfaCol + 8 * kF8Acc <= kF4SfbCol && kF4SfbCol + 4 <= (uint32_t)kF4TmemCols, "tensor memory");
+static_assert(kF4SfaCol + 8 * kF4MaxSlots <= kF4SfbNCol && kF4SfbNCol + 4 <= kF4SfbDnCol, "tensor memory");
 
 // bytes of one expert entry's down B operand: [I/16][16 rows][16] e4m3 codes,
-// then [I/128][8] fp32 inverse scales
-__host__ __device__ inline size_t f8_act_stride(int I) { return (size_t)I * 16 + (size_t)(I / 128) * 32; }
+// then [I/128][8] fp32 inverse scales; with MXFP4 (block-scaled MMAs) also
+// the same scales as e8m0 B scale factors, one 512-byte chunk per 4 blocks:
+// lane n (B row, < 16) byte j of chunk g = the scale of block 4 g + j
+__host__ __device__ inline size_t f8_act_stride(int I, bool mx) {
+  return (size_t)I * 16 + (size_t)(I / 128) * 32 + (mx ? (size_t)(I / 512) * kF4Sf : 0);
+}
 
 // e with m 2^e in [128, 256) for m > 0 (0 for m = 0), within [-126, 126] so
 // that 2^e and 2^-e are normal floats
@@ -153,7 +160,7 @@ __device__ void f8_convert_n(const Params& p, Ctl* c, uint8_t* regA) {
 // zero for rows that do not use the expert.  Then the block counts for its
 // expert.  Every epilogue thread, live or not.
 __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg& sg, bool live, int i,
-                                             const float (&a)[8], const float (&b)[8]) {
+                                             const float (&a)[8], const float (&b)[8], bool mx) {
   const int R = p.R, K = p.K, I = p.I, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int x = sg.x;
   float act[8];
@@ -173,7 +180,7 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
     if (lane == 0) c->amax[warp][r] = __uint_as_float(mb);
   }
   bar_sync(kBarEpi, 4 * 32);
-  uint8_t* base = p.actb + (size_t)x * f8_act_stride(I);
+  uint8_t* base = p.actb + (size_t)x * f8_act_stride(I, mx);
   const int ch = sg.blk * 128 + i;
   uint8_t* dst = base + (size_t)(ch >> 4) * 256 + (ch & 15);
 #pragma unroll
@@ -194,6 +201,15 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
       float* inv = reinterpret_cast<float*>(base + (size_t)I * 16) + sg.blk * 8;
       if (i == r) inv[r] = pow2i(-e[0]);
       if (i == r + 1) inv[r + 1] = pow2i(-e[1]);
+      if (mx && (i == r || i == r + 1)) {
+        // the block's scale as the e8m0 B scale factor of rows rr (hi) and
+        // 8 + rr (lo): byte (blk % 4) of lane n in chunk blk / 4
+        const int rr = i;
+        const uint8_t code = (uint8_t)(127 - e[rr - r]);
+        uint8_t* sfb = base + (size_t)I * 16 + (size_t)(I / 128) * 32 + (size_t)(sg.blk / 4) * kF4Sf + (sg.blk % 4);
+        sfb[16 * rr] = code;
+        sfb[16 * (8 + rr)] = code;
+      }
     }
   }
   // the block's activations are out: count it for its expert (the codes are
@@ -252,17 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   tc_fence_after();
   const uint32_t ep1 = c->epoch + 1u;
   const uint32_t tmem = c->tmem_base;
-  if (F4) {
-    // B's scale factors: 1.0 (e8m0 127) in every lane of their 4 columns,
-    // written before any MMA reads them (the barrier below orders them)
-    if (warp < 4) {
-      tmem_st4(tmem + ((uint32_t)(warp * 32) << 16) + kF4SfbCol, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
   trace(p, 0, tid == 0);
 
   // a ring stage: one gate/up unit (gate, up) or two down units
@@ -367,7 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
     ok = warp_ok(ok);
     const uint32_t idesc = F4 ? umma_idesc_mx_e2m1_e4m3(128, 16) : umma_idesc_e4m3(128, 16);
-    const uint32_t b_bytes = (uint32_t)I * 16u;
+    // the down B operand: codes, and for MXFP4 also its e8m0 scale chunks
+    // (the fp32 inverse scales between them are read by the epilogue only)
+    const uint32_t b_bytes = F4 ? (uint32_t)f8_act_stride(I, true) : (uint32_t)I * 16u;
     // B (n, or a down expert's activations): [K/16][16 rows][16], 256 bytes
     // between K-neighbours, rows 8-15 128 bytes on; a unit is 2048 bytes
     const uint64_t bdesc = umma_desc(smem_u32(regA), 256u, 128u);
@@ -389,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         if (ok) {   // (a copy whose wait failed is waited for again at exit)
           if (lane == 0) {
             mbar_arrive_expect_tx(&c->bfull, b_bytes);
-            tma_load_1d(regA, p.actb + (size_t)sg.x * f8_act_stride(I), b_bytes, &c->bfull);
+            tma_load_1d(regA, p.actb + (size_t)sg.x * f8_act_stride(I, F4), b_bytes, &c->bfull);
             ok = wait_bar(p, c, &c->bfull, nb & 1u);
           }
           ok = warp_ok(ok);
@@ -397,13 +404,62 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           ++nb;
         }
         tc_fence_after();
+        if (F4 && ok) {
+          // the expert's activation scales: chunk g (blocks 4 g .. 4 g + 3)
+          // to the 4 B-scale columns from kF4SfbDnCol + 4 g
+          const uint8_t* sfb = regA + (size_t)I * 16 + (size_t)(I / 128) * 32;
+          for (int g = 0; g < I / 512; ++g)
+            tmem_cp_sf(tmem + kF4SfbDnCol + 4u * g, umma_desc(smem_u32(sfb + (size_t)g * kF4Sf), 16u, 128u));
+        }
         trace(p, 15, nb == 1 && lane == 0);
       }
       const int per = stage_units(sg);
+      if (F4) {
+        // MXFP4: the weights' block scales and the activations' scales are
+        // applied inside the MMAs, so the whole segment accumulates in one
+        // buffer.  Stage s's A scale chunks go to the 8 columns of its ring
+        // slot (gate 4 | up 4, or unit 0 | unit 1), free again once the
+        // slot's MMAs are complete (which the producer waits for).
+        const uint32_t buf = t % kF8Acc;
+        if (t >= kF8Acc) {
+          if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / kF8Acc) - 1) & 1u);
+          ok = warp_ok(ok);
+        }
+        tc_fence_after();
+        for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
+          const uint32_t slot = s % p.nst, q = s / p.nst;
+          const int n = min(per, sg.k1 - u0);
+          if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
+          ok = warp_ok(ok);
+          tc_fence_after();
+          if (sg.list == L_RGU && first_rgu) {
+            first_rgu = false;
+            trace(p, 13, lane == 0);
+          }
+          const uint8_t* a_st = ring + (size_t)slot * p.slot_bytes;
+          const uint32_t sfa = tmem + kF4SfaCol + 8u * slot;
+          for (int j = 0; j < n && ok; ++j) {
+            const int u = u0 + j;
+            const uint8_t* a = a_st + (size_t)j * kF4SmemMat;   // gate/up: gate here, up 16 KB on
+            const uint8_t* sf = a_st + kF4SfOff + j * kF4Sf;
+            // gate/up: n's scale per row (any byte); down: unit u's scale,
+            // byte u % 4 of the columns of its chunk
+            const uint32_t sfb = gu ? tmem + kF4SfbNCol : tmem + kF4SfbDnCol + 4u * (uint32_t)(u / 4);
+            umma_unit_mx(tmem + 32u * buf, umma_desc_sw128(smem_u32(a), 1024u), bdesc + (uint64_t)(u * 128), 32u,
+                         idesc, sfa + 4u * j, umma_desc(smem_u32(sf), 16u, 128u), sfa + 4u,
+                         umma_desc(smem_u32(sf + kF4Sf), 16u, 128u), sfb, gu, gu ? 0u : (uint32_t)(u % 4),
+                         u > sg.k0, gu);
+          }
+          umma_commit_warp(&empty[slot]);
+          ++s;
+        }
+        umma_commit_warp(&c->accfull[buf]);
+        ++t;
+        return;
+      }
       for (int u0 = sg.k0; u0 < sg.k1; u0 += per) {
         // the stage's A in the ring slot: FP8 unit-matrices of 16 KB in the
-        // no-swizzle core-matrix layout; MXFP4 unit-matrices of 16 KB with the
-        // 128-byte swizzle, their scale chunks behind them
+        // no-swizzle core-matrix layout
         const uint32_t slot = s % p.nst, q = s / p.nst;
         const int n = min(per, sg.k1 - u0);
         if (lane == 0 && ok) ok = wait_bar(p, c, &full[slot], q & 1);
@@ -423,21 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           }
           tc_fence_after();
           if (ok) {
-            if (F4) {
-              // gate/up: gate at the slot start, up 16 KB on, scale chunks
-              // (gate, up) at kF4SfOff; down unit j at 16 KB * j, its chunk
-              // at kF4SfOff + 512 j.  Each accumulator buffer has 8 scale
-              // columns (gate 4 | up 4), free once its epilogue has read it.
-              const uint8_t* a = a_st + (size_t)(gu ? 0 : j) * kF4SmemMat;
-              const uint8_t* sf = a_st + kF4SfOff + (gu ? 0 : j) * kF4Sf;
-              const uint32_t sfa = tmem + kF4SfaCol + 8u * buf;
-              umma_unit_mx(tmem + 32u * buf, umma_desc_sw128(smem_u32(a), 1024u), bdesc + (uint64_t)(u * 128), 32u,
-                           idesc, sfa, umma_desc(smem_u32(sf), 16u, 128u), sfa + 4u,
-                           umma_desc(smem_u32(sf + kF4Sf), 16u, 128u), tmem + kF4SfbCol, gu);
-            } else {
-              const uint64_t da = umma_desc(smem_u32(a_st + (size_t)j * MAT), 2048u, 128u);
-              umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
-            }
+            const uint64_t da = umma_desc(smem_u32(a_st + (size_t)j * MAT), 2048u, 128u);
+            umma_unit_e4m3(tmem + 32u * buf, da, bdesc + (uint64_t)(u * 128), 32u, idesc, gu);
           }
           umma_commit_warp(&c->accfull[buf]);
           ++t;
@@ -482,6 +525,17 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   router_logits<true>(p, c, regA, false);
   f8_convert_n(p, c, regA);
   fence_proxy_async_smem();   // n is read by the tensor cores (async proxy)
+  bar_sync(kBarCons, kCW * 32);
+  if (F4 && warp < 4) {
+    // n's row scales as the B scale factors of the gate/up MMAs: lane n of
+    // every lane quarter holds B row n's e8m0 code (rows 8-15, the lo terms,
+    // share their token row's scale) in every byte of its first column
+    const uint32_t code = lane < 16 ? (__float_as_uint(c->nsc[lane & 7]) >> 23) & 0xFFu : 127u;
+    tmem_st4(tmem + ((uint32_t)(warp * 32) << 16) + kF4SfbNCol, code * 0x01010101u, 0x7F7F7F7Fu, 0x7F7F7F7Fu,
+             0x7F7F7F7Fu);
+    tmem_st_wait();
+    tc_fence_before();
+  }
   bar_sync(kBarCons, kCW * 32);
   if (tid == 0) *(volatile int*)&c->n_ready = 1;
   trace(p, 3, tid == 0);
@@ -529,6 +583,22 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
 #pragma unroll
       for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
       uint32_t v[16], w2[16];
+      if (F4) {
+        // the segment's sums, every scale already applied in the MMAs: the
+        // hi (rows 0-7) and lo (rows 8-15) columns of each token row added
+        take(v, w2, gu);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          a[r] = __uint_as_float(v[r]) + __uint_as_float(v[8 + r]);
+          b[r] = gu ? __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]) : 0.f;
+        }
+        trace(p, 20, t == 1 && tid == 0);
+        const bool live = ok && !c->dead;
+        if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
+        if (gu) f8_store_act(p, c, sg, live, i, a, b, true);
+        else epi_store(p, c, geo, sg, false, live, i, a, b);
+        return;
+      }
       // the units' FP8 block scales (brought to L2 by the producer), two units
       // ahead; MXFP4 block scales are applied inside the MMA (1 here)
       const float* sc = gu ? p.gsc + (size_t)(e * geo.nbi + sg.blk) * upb * 256
@@ -562,35 +632,64 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         if (tid == 0 && ok) ok = wait_count(p, c, &p.xready[sg.x], (uint32_t)geo.nbi, 4u);
         bar_sync(kBarEpi, 4 * 32);
         const float4* asc =
-            reinterpret_cast<const float4*>(p.actb + (size_t)sg.x * f8_act_stride(I) + (size_t)I * 16);
+            reinterpret_cast<const float4*>(p.actb + (size_t)sg.x * f8_act_stride(I, false) + (size_t)I * 16);
         auto ld_a = [&](int u, float4& lo4, float4& hi4) {
           const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
           lo4 = u < sg.k1 ? __ldcg(asc + 2 * u) : z;
           hi4 = u < sg.k1 ? __ldcg(asc + 2 * u + 1) : z;
         };
-        float4 a0l, a0h, a1l, a1h;
-        ld_a(sg.k0, a0l, a0h);
-        ld_a(sg.k0 + 1, a1l, a1h);
-        for (int u = sg.k0; u < sg.k1; ++u) {
-          const float sg2 = ld_g(u + 2);
-          float4 a2l, a2h;
-          ld_a(u + 2, a2l, a2h);
-          take(v, w2, false);
-          const float k8[8] = {a0l.x, a0l.y, a0l.z, a0l.w, a0h.x, a0h.y, a0h.z, a0h.w};
+        // two units per round: one wait and one tensor-memory load latency
+        // for the pair (a down stage holds two units); the sums stay in unit
+        // order.  The scales of the next pair are loaded before this pair's
+        // tiles are waited for.
+        float4 al[2], ah[2], nl[2], nh[2];
+        float ws[2], nws[2];
+        ld_a(sg.k0, al[0], ah[0]);
+        ld_a(sg.k0 + 1, al[1], ah[1]);
+        ws[0] = ld_g(sg.k0);
+        ws[1] = ld_g(sg.k0 + 1);
+        for (int u = sg.k0; u < sg.k1; u += 2) {
+          const bool two = u + 1 < sg.k1;
+          ld_a(u + 2, nl[0], nh[0]);
+          ld_a(u + 3, nl[1], nh[1]);
+          nws[0] = ld_g(u + 2);
+          nws[1] = ld_g(u + 3);
+          const uint32_t b0 = t % kF8Acc, b1 = (t + 1) % kF8Acc;
+          if (ok) ok = wait_bar(p, c, &c->accfull[b0], (t / kF8Acc) & 1u);
+          if (ok && two) ok = wait_bar(p, c, &c->accfull[b1], ((t + 1) / kF8Acc) & 1u);
+          tc_fence_after();
+          const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
+          tmem_ld16_nowait(ta + 32u * b0, v);
+          if (two) tmem_ld16_nowait(ta + 32u * b1, w2);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&c->accempty[b0]);
+            if (two) mbar_arrive(&c->accempty[b1]);
+          }
+          t += two ? 2u : 1u;
+          const float k0[8] = {al[0].x, al[0].y, al[0].z, al[0].w, ah[0].x, ah[0].y, ah[0].z, ah[0].w};
 #pragma unroll
-          for (int r = 0; r < 8; ++r) a[r] = fmaf(sg0 * k8[r], __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
-          sg0 = sg1;
-          sg1 = sg2;
-          a0l = a1l;
-          a0h = a1h;
-          a1l = a2l;
-          a1h = a2h;
+          for (int r = 0; r < 8; ++r) a[r] = fmaf(ws[0] * k0[r], __uint_as_float(v[r]) + __uint_as_float(v[8 + r]), a[r]);
+          if (two) {
+            const float k1[8] = {al[1].x, al[1].y, al[1].z, al[1].w, ah[1].x, ah[1].y, ah[1].z, ah[1].w};
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              a[r] = fmaf(ws[1] * k1[r], __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]), a[r]);
+          }
+          al[0] = nl[0];
+          ah[0] = nh[0];
+          al[1] = nl[1];
+          ah[1] = nh[1];
+          ws[0] = nws[0];
+          ws[1] = nws[1];
         }
       }
       trace(p, 20, t == 1 && tid == 0);
       const bool live = ok && !c->dead;
       if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
-      if (gu) f8_store_act(p, c, sg, live, i, a, b);
+      if (gu) f8_store_act(p, c, sg, live, i, a, b, false);
       else epi_store(p, c, geo, sg, false, live, i, a, b);
     };
     tc_segments(p, geo, L_SGU, 0, seg);
