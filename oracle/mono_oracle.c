@@ -113,6 +113,39 @@ EXPORT void orc_quant_fp8(const float* w, int64_t rows, int64_t cols, uint8_t* q
   }
 }
 
+/* MXFP8 (e4m3) quantiser of an activation vector, OCP MX v1.0 shared-exponent
+ * rule: per block of 32 consecutive values, X = floor(log2 amax) - 8 (8 = the
+ * largest e4m3 exponent), clamped to the e8m0 range [-127, 127]; each element
+ * becomes the e4m3 value nearest to x / 2^X (ties to the even code),
+ * saturating at 448, and decodes to that value times 2^X.  An all-zero block
+ * keeps scale byte 0 and zero codes.  codes / scales (may be NULL) receive the
+ * e4m3 codes and the e8m0 bytes. */
+EXPORT void orc_quant_mx8(const double* x, int64_t n, double* out, uint8_t* codes, uint8_t* scales) {
+  double mag[127];
+  for (int c = 0; c < 127; ++c) mag[c] = orc_dec_e4m3((uint8_t)c);
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const double* src = x + b * 32;
+    double amax = 0.0;
+    int X = -127;
+    for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(src[i]));
+    if (amax > 0.0) {
+      int ex;
+      frexp(amax, &ex);
+      X = (ex - 1) - 8;
+      if (X < -127) X = -127;
+      if (X > 127) X = 127;
+    }
+    if (scales) scales[b] = amax > 0.0 ? (uint8_t)(X + 127) : 0;
+    for (int i = 0; i < 32; ++i) {
+      const double v = ldexp(src[i], -X);
+      const int code = amax > 0.0 ? nearest_even(mag, 127, fabs(v)) : 0;
+      const int neg = signbit(v) && code != 0;
+      out[b * 32 + i] = (neg ? -1.0 : 1.0) * ldexp(mag[code], X);
+      if (codes) codes[b * 32 + i] = (uint8_t)(code | (neg ? 0x80 : 0));
+    }
+  }
+}
+
 /* MXFP4 quantiser (OCP MX v1.0 shared-exponent rule): per 32-block,
  * X = floor(log2 amax) - 2 (the largest e2m1 exponent), scale byte X + 127
  * clamped to [0, 254] (0 when amax = 0); element = e2m1(w / 2^X), the scaled
@@ -187,6 +220,9 @@ static void dec_weight_row(const void* codes, const void* scales, int dt, int64_
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 static double softplus(double x) { return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x))); }
+
+/* the MXFP8-activation numerics apply to MXFP4 experts only */
+static int mx8_on(const orc_cfg* c) { return c->act_mx8 && c->w_dtype == ORC_MXFP4; }
 
 static int check_cfg(const orc_cfg* c) {
   if (c->hidden <= 0 || c->hc <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->top_k > c->n_routed ||
@@ -319,6 +355,16 @@ static int expert(const orc_cfg* c, const orc_weights* w, int e, const double* n
   if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) return -(100 + e);
   act = (double*)malloc(sizeof(double) * (size_t)I);
   d = (double*)malloc(sizeof(double) * (size_t)H);
+  /* MXFP8 activations (vLLM MonoKernel page, Numerics: the kernel quantises
+   * the activations to MXFP8 for the MXFP4 experts): n before gate / up,
+   * and the SwiGLU output before down, each in blocks of 32 along the
+   * contraction */
+  double* nq = NULL;
+  if (mx8_on(c)) {
+    nq = (double*)malloc(sizeof(double) * (size_t)H);
+    orc_quant_mx8(n, H, nq, NULL, NULL);
+    n = nq;
+  }
 #pragma omp parallel for schedule(static)
   for (ch = 0; ch < I; ++ch) {
     double* row = (double*)malloc(sizeof(double) * (size_t)H);
@@ -334,6 +380,7 @@ static int expert(const orc_cfg* c, const orc_weights* w, int e, const double* n
     act[ch] = g * sigmoid(g) * u;
     free(row);
   }
+  if (mx8_on(c)) orc_quant_mx8(act, I, act, NULL, NULL);
 #pragma omp parallel for schedule(static)
   for (ch = 0; ch < H; ++ch) {
     double* row = (double*)malloc(sizeof(double) * (size_t)I);
@@ -346,6 +393,7 @@ static int expert(const orc_cfg* c, const orc_weights* w, int e, const double* n
   for (int h = 0; h < H; ++h) dst[h] += wt * d[h];
   free(act);
   free(d);
+  free(nq);
   return 0;
 }
 
@@ -383,15 +431,18 @@ static int dense_mlp(const orc_cfg* c, const orc_weights* w, row_state* st) {
   for (int e = 0; e < E1; ++e)
     if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) return -(100 + e);
   act = (double*)malloc(sizeof(double) * (size_t)W);
+  double* nq = (double*)malloc(sizeof(double) * (size_t)H);
+  memcpy(nq, st->n, sizeof(double) * (size_t)H);
+  if (mx8_on(c)) orc_quant_mx8(st->n, H, nq, NULL, NULL);
 #pragma omp parallel for schedule(static)
   for (ch = 0; ch < W; ++ch) {
     double* row = (double*)malloc(sizeof(double) * (size_t)H);
     const int e = (int)(ch / I), i = (int)(ch % I);
     double g = 0.0, u = 0.0;
     dec_weight_row(w->w_gate[e], w->s_gate ? w->s_gate[e] : NULL, c->w_dtype, i, H, row);
-    for (int h = 0; h < H; ++h) g += st->n[h] * row[h];
+    for (int h = 0; h < H; ++h) g += nq[h] * row[h];
     dec_weight_row(w->w_up[e], w->s_up ? w->s_up[e] : NULL, c->w_dtype, i, H, row);
-    for (int h = 0; h < H; ++h) u += st->n[h] * row[h];
+    for (int h = 0; h < H; ++h) u += nq[h] * row[h];
     if (c->round_bf16) {
       g = rbf16(g);
       u = rbf16(u);
@@ -399,6 +450,7 @@ static int dense_mlp(const orc_cfg* c, const orc_weights* w, row_state* st) {
     act[ch] = g * sigmoid(g) * u;
     free(row);
   }
+  if (mx8_on(c)) orc_quant_mx8(act, W, act, NULL, NULL);
 #pragma omp parallel for schedule(static)
   for (ch = 0; ch < H; ++ch) {
     double* row = (double*)malloc(sizeof(double) * (size_t)W);
@@ -414,6 +466,7 @@ static int dense_mlp(const orc_cfg* c, const orc_weights* w, row_state* st) {
     st->w[j] = 1.0f;
   }
   free(act);
+  free(nq);
   return 0;
 }
 

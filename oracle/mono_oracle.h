@@ -57,6 +57,7 @@ typedef struct {
   int sinkhorn_iters;
   double rms_eps, pre_eps, post_mult, route_scale, denom_clamp;
   int dense;      /* 1: no router; a dense SwiGLU MLP of width (E + 1) I over all slots (top_k = E) */
+  int act_mx8;    /* 1 (MXFP4 experts only): activations quantised to MXFP8 before each expert matvec */
 } orc_cfg;
 
 /* Logical layouts (row-major):
@@ -136,6 +137,7 @@ double orc_dec_e8m0(uint8_t b);
 uint16_t orc_round_bf16(double x);
 void orc_quant_fp8(const float* w, int64_t rows, int64_t cols, uint8_t* q, float* s);
 void orc_quant_mxfp4(const float* w, int64_t rows, int64_t cols, uint8_t* q, uint8_t* e);
+void orc_quant_mx8(const double* x, int64_t n, double* out, uint8_t* codes, uint8_t* scales);
 
 #ifdef __cplusplus
 }

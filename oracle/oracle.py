@@ -42,7 +42,7 @@ class Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "hc", "n_routed", "top_k", "inter", "rows", "hc_dtype",
                                             "norm_dtype", "w_dtype", "round_bf16", "sinkhorn_iters")] + \
                [(n, ctypes.c_double) for n in ("rms_eps", "pre_eps", "post_mult", "route_scale", "denom_clamp")] + \
-               [("dense", ctypes.c_int)]
+               [("dense", ctypes.c_int), ("act_mx8", ctypes.c_int)]
 
 
 class Weights(ctypes.Structure):
@@ -86,6 +86,7 @@ def lib():
         L.orc_round_bf16.restype = ctypes.c_uint16
         L.orc_quant_fp8.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp]
         L.orc_quant_mxfp4.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp]
+        L.orc_quant_mx8.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -99,7 +100,7 @@ def make_cfg(wl, rows=None):
                rows=wl.rows if rows is None else rows, hc_dtype=_DT[wl.hc_dtype], norm_dtype=_DT[wl.norm_dtype],
                w_dtype=_DT[wl.w_dtype], round_bf16=int(wl.round_bf16), sinkhorn_iters=wl.sinkhorn_iters,
                rms_eps=wl.rms_eps, pre_eps=wl.pre_eps, post_mult=wl.post_mult, route_scale=wl.route_scale,
-               denom_clamp=wl.denom_clamp, dense=int(wl.dense))
+               denom_clamp=wl.denom_clamp, dense=int(wl.dense), act_mx8=int(wl.act_mx8))
 
 
 class LayerWeights:
@@ -262,6 +263,16 @@ def quant_mxfp4(x):
     e = np.empty((x.shape[0], x.shape[1] // 32), np.uint8)
     lib().orc_quant_mxfp4(_p(x), x.shape[0], x.shape[1], _p(q), _p(e))
     return q, e
+
+
+def quant_mx8(x):
+    """MXFP8 (e4m3, e8m0 per 32) of a float64 vector: (values, codes, scales)."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.empty_like(x)
+    q = np.empty(x.shape, np.uint8)
+    e = np.empty(x.size // 32, np.uint8)
+    lib().orc_quant_mx8(_p(x), x.size, _p(out), _p(q), _p(e))
+    return out, q, e
 
 
 def decode_hc(wl, raw):

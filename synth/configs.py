@@ -41,6 +41,7 @@ class Workload:
     sinkhorn_iters: int = 20
     mx_spread: int = 0   # MXFP4: block magnitudes within a row span up to 2^mx_spread
     dense: bool = False  # a dense MLP of width (n_routed + 1) * inter over every slot, no router
+    act_mx8: bool = False  # MXFP4 experts: activations quantised to MXFP8 before each expert matvec
 
     def with_(self, **kw):
         return replace(self, **kw)

@@ -507,3 +507,72 @@ def test_dense_layer_with_bf16_rounding_equals_routed_slices_of_weight_one():
     yb = torch.from_numpy(y).to(torch.float32).to(torch.bfloat16).double().numpy()
     assert np.mean(yb == t.y) > 0.99
     assert np.allclose(yb, t.y, rtol=2 ** -7, atol=1e-6)
+
+
+# ------------------------------------------------------ MXFP8 activations --
+
+def _e4m3_table():
+    return np.array([O.lib().orc_dec_e4m3(c) for c in range(127)], np.float64)   # code 127 is NaN
+
+
+def test_mx8_quantiser_vs_brute_force():
+    """OCP MX rule for e4m3 blocks: scale 2^(floor(log2 amax) - 8); each value
+    the nearest of the 127 e4m3 magnitudes times the scale (ties to the even
+    code), saturating at 448; brute force over every code, on blocks spanning
+    normal, subnormal, saturating and zero values."""
+    mag = _e4m3_table()
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(32 * 40) * 10.0 ** rng.integers(-6, 6, 32 * 40),
+                        np.zeros(32), np.full(32, 448.0 * 2 ** -3), rng.standard_normal(32) * 1e-30])
+    got, codes, scales = O.quant_mx8(x)
+    for b in range(x.size // 32):
+        blk = x[b * 32:(b + 1) * 32]
+        amax = np.abs(blk).max()
+        if amax == 0:
+            assert scales[b] == 0 and np.all(got[b * 32:(b + 1) * 32] == 0)
+            continue
+        X = max(-127, min(127, int(np.floor(np.log2(amax))) - 8))
+        assert scales[b] == X + 127
+        for i, v in enumerate(blk):
+            a = abs(v) / 2.0 ** X
+            d = np.abs(mag - a)
+            best = np.flatnonzero(d == d.min())
+            code = best[0] if len(best) == 1 else (best[0] if best[0] % 2 == 0 else best[1])
+            want = np.copysign(mag[code] * 2.0 ** X, v) if code else 0.0
+            assert got[b * 32 + i] == want, (b, i, v, got[b * 32 + i], want)
+
+
+def test_mx8_quantiser_matches_torch_float8_in_range():
+    """Within the e4m3 range the element codes equal torch's float8_e4m3fn
+    rounding of x / 2^X (RNE)."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(32 * 64) * 3.0
+    _, codes, scales = O.quant_mx8(x)
+    X = scales.astype(np.int64) - 127
+    v = torch.from_numpy(x / np.repeat(2.0 ** X, 32))
+    t = v.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    keep = np.abs(v.numpy()) <= 448.0
+    assert np.array_equal(t[keep], codes[keep])
+
+
+def test_mx8_single_expert_reduces_to_swiglu_mlp_on_quantised_activations():
+    """E = k = 1, zero shared expert, MXFP4 weights, act_mx8: y = 2.5 down(q(
+    silu(gate q(n)) up q(n))) with q the MXFP8 quantiser, evaluated with
+    torch.nn.functional in float64 on the dequantised weights."""
+    wl = tiny(n_routed=1, top_k=1, rows=2, hidden=64, inter=32, w_dtype="mxfp4", act_mx8=True)
+    hc, dense, ex = layer_inputs(wl, experts="all")
+    zq, zs = (np.zeros_like(a) for a in ex[0]["gate"])
+    ex[1] = {"gate": (zq, zs), "up": (zq.copy(), zs.copy()),
+             "down": (np.zeros_like(ex[0]["down"][0]), np.zeros_like(ex[0]["down"][1]))}
+    _, t = O.layer(wl, O.LayerWeights(wl, dense, ex), hc)
+    m = f32_of(wl, ex[0])
+    for r in range(wl.rows):
+        nq = torch.from_numpy(O.quant_mx8(t.n[r])[0])
+        g = F.linear(nq, torch.from_numpy(m["gate"]))
+        u = F.linear(nq, torch.from_numpy(m["up"]))
+        act = torch.from_numpy(O.quant_mx8((F.silu(g) * u).numpy())[0])
+        y = 2.5 * F.linear(act, torch.from_numpy(m["down"]))
+        assert torch.allclose(torch.from_numpy(t.y[r]), y, rtol=1e-12, atol=1e-14)
+    # and the quantisation is really applied: without it the result differs
+    _, t2 = O.layer(wl.with_(act_mx8=False), O.LayerWeights(wl, dense, ex), hc)
+    assert not np.allclose(t.y, t2.y, rtol=1e-9)
