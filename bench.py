@@ -66,6 +66,7 @@ def wl_config(wl, extra=None):
     cfg = {"workload": wl.name, "rows": wl.rows, "hidden": wl.hidden, "hc_streams": wl.hc,
            "routed_experts": wl.n_routed, "top_k": wl.top_k, "shared_experts": 1, "inter": wl.inter,
            "layers_per_step": wl.n_layers, "expert_format": wl.w_dtype, "hc_format": wl.hc_dtype,
+           "activations": "mxfp8 (e4m3, e8m0 per 32)" if getattr(wl, "act_mx8", False) else "as the layer defines",
            "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so that the "
                  "written lines are back in HBM and L2 holds only clean lines of an unrelated buffer)"
                  if L2_MODE[0] == "flush" else
@@ -77,7 +78,8 @@ def wl_config(wl, extra=None):
 
 
 def dtype_of(wl):
-    return {"f32": "f32", "bf16": "bf16", "fp8": "fp8e4m3", "mxfp4": "mxfp4"}[wl.w_dtype]
+    d = {"f32": "f32", "bf16": "bf16", "fp8": "fp8e4m3", "mxfp4": "mxfp4"}[wl.w_dtype]
+    return d + "+mxfp8act" if getattr(wl, "act_mx8", False) else d
 
 
 # ------------------------------------------------------------------ clocks --
@@ -223,10 +225,10 @@ def run_reference(args):
 TRACE_NAMES = ["start", "mix published", "mix totals seen", "n ready", "logits published", "lists ready",
                "shared gate/up done", "routed gate/up done", "1st down expert ready", "down done", "end",
                "producer saw lists", "producer issued all", "issuer: 1st routed stage", "issuer: routed issued",
-               "issuer: 1st down operand", "issuer: all issued", "(unused)", "producer: 1st routed",
+               "issuer: 1st down operand", "issuer: all issued", "mix: partials computed", "producer: 1st routed",
                "producer: 1st down", "epilogue: 1st shared", "ctl: logits complete", "ctl: top-k done",
                "pre/post ready", "collapse: all slices", "router: dots done", "top-k: loads done",
-               "collapse: slice out", "mix: inputs in smem"]
+               "collapse: slice out", "mix: inputs in smem", "collapse: slices in smem", "norm: n done"]
 TRACE_POINTS = 32
 
 
@@ -277,7 +279,7 @@ def job_value(tot_ms, steps, layers, world):
 
 
 PER_CONFIG = ["v41flash-bf16-r1", "v41flash-bf16-r6", "v41flash-bf16-r8", "v41flash-fp8b128-r4",
-              "v41flash-mxfp4-chain4-r8"]
+              "v41flash-mxfp4-chain4-r8", "v41flash-mxfp4-mx8act-chain4-r8"]
 
 
 def traffic_of(wl):

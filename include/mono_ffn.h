@@ -13,8 +13,9 @@
  *      pre-norm GEMM partials + RMS square-sum partials, finalised together;
  *      ds4 "v41: fuse the single-box decode glue", HC fusion commit.)
  *   2. collapse a = sum_s pre_s X_s -> bf16; weighted RMSNorm
- *      n = a / sqrt(mean a^2 + eps) * norm_w -> bf16.  (ds4 page, HC fusion:
- *      "pre-weighted collapse + BF16 + weighted RMSNorm + BF16".)
+ *      n = a / sqrt(mean a^2 + eps) * norm_w -> bf16.  (ds4 page, HC fusion
+ *      commit: the collapse weighted by pre and the weighted RMSNorm, each
+ *      rounded to bf16.)
  *   3. router select: fp32 logits n @ router_w; score = sqrt(softplus);
  *      sel = score + bias (selection only); canonical top-k by (sel desc,
  *      index asc); weight = score / max(sum, clamp) * route_scale.  (ds4
@@ -24,8 +25,8 @@
  *      MoE fusion; vLLM "[ROCm][Perf][GLM-5] Fused sparse-layer decode via
  *      AITER MonoKernel", Weights: shared expert in the last slot.)
  *   5. y = bf16(sum_j w_j d_j + d_shared); out_i = bf16(sum_j comb_ij X_j +
- *      post_i y).  (ds4 page: "block = bf16(routed + shared)" folded into the
- *      tail's expand.)
+ *      post_i y).  (ds4 page: the routed + shared sum rounded to bf16 and
+ *      folded into the tail's expand.)
  * The bf16 roundings apply when round_bf16 is set; an fp32 configuration
  * keeps every value in fp32.
  *
@@ -100,6 +101,11 @@ typedef struct {
                        the n_routed + 1 slots in slot order, run as expert-shaped slices each taken
                        with weight 1 (vLLM MonoKernel page, Weights); top_k must equal n_routed, and
                        router_w / router_bias may be NULL at packing */
+  int act_mx8;      /* 1: MXFP8 activations for MXFP4 experts (vLLM MonoKernel page, Numerics): n and the
+                       SwiGLU output are quantised to e4m3 with one e8m0 scale per 32 values (OCP MX rule)
+                       before each expert matvec, which then runs as one block-scaled e2m1 x e4m3 MMA
+                       term; MXFP4 experts on the tensor-core path only (round_bf16, hidden and inter
+                       multiples of 128, hidden and inter <= 5120).  0: weight-only dequantisation */
 } mono_ffn_config;
 
 /* One layer's weights, device pointers in logical (caller) layouts, read only
@@ -185,7 +191,7 @@ int mono_ffn_plan(const mono_ffn_config* cfg, mono_ffn_plan_t** out);
 
 /* Repack one layer's weights (logical layouts above) into the plan's kernel
  * layout, router transposed to [E][H].  A one-time conversion (vLLM
- * MonoKernel page, Weights: "packed once").  Expert layouts:
+ * MonoKernel page, Weights: the weights are packed one time).  Expert layouts:
  *   - bf16 on the tensor cores (hidden, inter multiples of 128): blocks of 128
  *     rows of K-major core matrices, gate and up interleaved per row group;
  *   - FP8 / MXFP4 on the tensor cores (bf16-rounded layers, multiples of 128):
@@ -223,7 +229,8 @@ int mono_ffn_step_padded(mono_ffn_plan_t* plan, int width, const int* row_slot, 
 
 /* One step opened by the attention sublayer's pending post / expand (the
  * within-layer boundary: SGLang "[DeepSeek-V4] Add mhc_fused_post_pre
- * kernel", Modifications, "attention hc_post + FFN hc_pre" inside one layer):
+ * kernel", Modifications: the attention sublayer's hc_post fused with the
+ * FFN's hc_pre inside one layer):
  * for each row r the FFN's residual streams are
  *   X_i = round(sum_j attn_comb[r][i][j] x_attn[r][j] + attn_post[r][i] y_attn[r])
  * (round = to hc_dtype), materialised in the opening pass together with the
@@ -266,11 +273,13 @@ int mono_ffn_get_info(const mono_ffn_plan_t* plan, mono_ffn_info* info);
  * 10 end, 11 producer saw the lists, 12 producer issued every copy;
  * tensor-core kernel also: 13 first routed gate/up stage arrived, 14 routed
  * gate/up MMAs issued, 15 first down operand ready, 16 every MMA issued,
- * 17 (unused), 18 first routed copy issued, 19 first down
+ * 18 first routed copy issued, 19 first down
  * copy issued, 20 first shared gate/up tile read; both: 21 logits counter
  * complete, 22 top-k done, 23 pre/post ready, 24 every CTA's collapsed
  * slice seen, 25 router dot products done, 26 top-k inputs loaded, 27 this
- * CTA's collapsed slice published, 28 mix inputs in shared memory.
+ * CTA's collapsed slice published, 28 mix inputs in shared memory; all
+ * kernels: 17 mix partials computed, 29 every slice of the collapse in
+ * shared memory, 30 n normalised.
  * The tensor-core kernel stores its SM id (not a time) at point 31.
  * Points a kernel does not reach stay as they were.
  * NULL turns it off (the default). */

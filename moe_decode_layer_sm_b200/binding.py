@@ -31,7 +31,7 @@ class Config(ctypes.Structure):
                                             "hc_dtype", "norm_dtype", "expert_dtype", "round_bf16")] + \
                [(n, ctypes.c_float) for n in ("rms_eps", "pre_eps", "post_mult", "route_scale", "denom_clamp")] + \
                [("sinkhorn_iters", ctypes.c_int), ("wait_timeout_us", ctypes.c_uint), ("device", ctypes.c_int),
-                ("grid", ctypes.c_int), ("dense", ctypes.c_int)]
+                ("grid", ctypes.c_int), ("dense", ctypes.c_int), ("act_mx8", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -110,14 +110,15 @@ class Plan:
 
     def __init__(self, hidden, n_routed, top_k, inter, max_rows, n_layers=1, hc_dtype="bf16", norm_dtype="bf16",
                  expert_dtype="bf16", round_bf16=True, rms_eps=1e-6, pre_eps=1e-6, post_mult=2.0, route_scale=2.5,
-                 denom_clamp=1e-20, sinkhorn_iters=20, wait_timeout_us=0, device=0, grid=0, dense=False):
+                 denom_clamp=1e-20, sinkhorn_iters=20, wait_timeout_us=0, device=0, grid=0, dense=False,
+                 act_mx8=False):
         self._lib = lib()
         self.cfg = Config(hidden=hidden, hc=4, n_routed=n_routed, top_k=top_k, inter=inter, max_rows=max_rows,
                           n_layers=n_layers, hc_dtype=DTYPE[hc_dtype], norm_dtype=DTYPE[norm_dtype],
                           expert_dtype=DTYPE[expert_dtype], round_bf16=int(round_bf16), rms_eps=rms_eps,
                           pre_eps=pre_eps, post_mult=post_mult, route_scale=route_scale, denom_clamp=denom_clamp,
                           sinkhorn_iters=sinkhorn_iters, wait_timeout_us=wait_timeout_us, device=device, grid=grid,
-                          dense=int(dense))
+                          dense=int(dense), act_mx8=int(act_mx8))
         h = ctypes.c_void_p()
         rc = self._lib.mono_ffn_plan(ctypes.byref(self.cfg), ctypes.byref(h))
         if rc != 0:
@@ -131,7 +132,7 @@ class Plan:
                    hc_dtype=wl.hc_dtype, norm_dtype=wl.norm_dtype, expert_dtype=wl.w_dtype,
                    round_bf16=wl.round_bf16, rms_eps=wl.rms_eps, pre_eps=wl.pre_eps, post_mult=wl.post_mult,
                    route_scale=wl.route_scale, denom_clamp=wl.denom_clamp, sinkhorn_iters=wl.sinkhorn_iters,
-                   dense=getattr(wl, "dense", False), **kw)
+                   dense=getattr(wl, "dense", False), act_mx8=getattr(wl, "act_mx8", False), **kw)
 
     def _check(self, rc):
         if rc != 0:

@@ -49,7 +49,7 @@ constexpr int kRingGuard = 4096;   // bytes after the ring that a tensor-core ti
 enum WType { W_F32 = 0, W_BF16 = 1, W_FP8 = 2, W_FP4 = 3 };
 
 struct SyncBlock {   // one per layer slot, 64 bytes
-  uint32_t epoch, cnt_mix, cnt_logit, cnt_act, cnt_done, cnt_y, cnt_a, pad[9];
+  uint32_t epoch, cnt_mix, cnt_logit, cnt_act, cnt_done, cnt_y, cnt_a, cnt_mix2, pad[8];
 };
 struct ErrBlock {
   uint32_t abort, code, stage, cta, layer, pad[11];
@@ -65,6 +65,7 @@ struct Params {
   int H, I, E, K, R, G;
   int layer, first, last;
   int dense;            // no router: every slot is a slice of one dense MLP, weight 1
+  int mx8;              // MXFP4 experts with MXFP8 activations (one e4m3 term per row, N = 8)
   int mix_ctas;
   int hc_bf16, norm_bf16, round_bf16;
   float rms_eps, pre_eps, post_mult, route_scale, denom_clamp;
@@ -96,6 +97,7 @@ struct Params {
   long long gu_estride, dn_estride;
   // scratch
   float* mix_part;   // [R*25][G] output-major partials of the mix
+  float* mix_tot;    // [R*25] the mix totals (each summed by one CTA)
   float* logits;     // [R][E]
   float* act;        // [R][K+1][I]
   void* abuf;        // [R][H] collapsed rows a (bf16 when rounded, else fp32), one h-slice per CTA
@@ -633,6 +635,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       c->red[op] = acc;
     }
     bar_sync(kBarPre, kPreThreads);
+    trace(p, 17, ptid == 0);
     // partials stored output-major: mix_part[o][G]
     for (int o = ptid; o < nout; o += kPreThreads) {
       float acc = 0.f;
@@ -650,10 +653,10 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
   if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix, ep1 * (uint32_t)G, 1u);
   bar_sync(kBarPre, kPreThreads);
   trace(p, 2, ptid == 0);
-  {
-    // every CTA's partials into shared memory at once (behind the slices,
-    // which the collapse still needs), then lane-strided sums and a butterfly
-    // across the warp: the same order in every CTA
+  if (R <= 3) {
+    // few outputs: every CTA's partials into shared memory at once (behind
+    // the slices, which the collapse still needs), then lane-strided sums
+    // and a butterfly across the warp, in the same order in every CTA
     float* parts = reinterpret_cast<float*>(regA + L.parts);
     const int cap = (int)(((size_t)p.regA_bytes - L.parts) / sizeof(float) / G);   // outputs per pass
     for (int o0 = 0; o0 < nout; o0 += cap) {
@@ -673,6 +676,31 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       }
       bar_sync(kBarPre, kPreThreads);
     }
+  } else {
+    // more outputs: the totals in two levels.  CTA c sums its share of the
+    // outputs over every CTA's partial (the same lane-strided sums and
+    // butterfly, so the same totals), publishes them, and after one more
+    // grid stage every CTA reads all of them (a few hundred bytes instead of
+    // every partial)
+    const int o0 = (int)((long long)blockIdx.x * nout / G), o1 = (int)((long long)(blockIdx.x + 1) * nout / G);
+    for (int o = o0 + pwarp; o < o1; o += kPreThreads / 32) {
+      float acc = 0.f;
+      if (!c->dead)
+        for (int m = lane; m < G; m += 32) acc += __ldcg(p.mix_part + (size_t)o * G + m);
+      acc = warp_sum(acc);
+      if (lane == 0) p.mix_tot[o] = acc;
+    }
+    bar_sync(kBarPre, kPreThreads);
+    if (ptid == 0 && may_publish(p, c->epoch, 0, 10)) {
+      __threadfence();
+      red_release_add(&p.sync->cnt_mix2, 1u);
+    }
+    if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix2, ep1 * (uint32_t)G, 1u);
+    bar_sync(kBarPre, kPreThreads);
+    for (int o = ptid; o < nout; o += kPreThreads) c->smix[o / kMixP][o % kMixP] = c->dead ? 0.f : __ldcg(p.mix_tot + o);
+    bar_sync(kBarPre, kPreThreads);
+  }
+  {
     if (ptid < R) {
       const int r = ptid;
       const float rho = 1.0f / sqrtf(c->smix[r][kMixC] / (float)(kS * H) + p.rms_eps);
@@ -894,6 +922,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
   }
   cp_async_wait_all();
   bar_sync(kBarCons, kCW * 32);
+  trace(p, 29, ctid == 0);
   // n = a * inv * norm_w, in place: one norm_w load per 8 columns, all rows
   {
     const int H8 = H / 8;
@@ -931,6 +960,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
     }
   }
   bar_sync(kBarCons, kCW * 32);
+  trace(p, 30, ctid == 0);
 }
 
 // Router logits of this CTA's experts (two rows of router_t at a time; each

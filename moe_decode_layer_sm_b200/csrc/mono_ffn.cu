@@ -48,6 +48,7 @@ struct mono_ffn_plan_s {
   long long gu_estride = 0, dn_estride = 0;
   std::vector<LayerSlot> layers;
   float* mix_part = nullptr;
+  float* mix_tot = nullptr;
   void* abuf = nullptr;
   float* sq_part = nullptr;
   float* logits = nullptr;
@@ -343,6 +344,7 @@ extern "C" void mono_ffn_destroy(mono_ffn_plan_t* p) {
   }
   for (float* q : p->pend) cudaFree(q);
   cudaFree(p->mix_part);
+  cudaFree(p->mix_tot);
   cudaFree(p->abuf);
   cudaFree(p->sq_part);
   cudaFree(p->logits);
@@ -388,6 +390,11 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
   need(cfg.sinkhorn_iters >= 0, "sinkhorn_iters must be >= 0");
   need(cfg.dense == 0 || cfg.dense == 1, "dense must be 0 or 1");
   need(!cfg.dense || cfg.top_k == cfg.n_routed, "a dense layer takes every slot: top_k must equal n_routed");
+  need(cfg.act_mx8 == 0 || cfg.act_mx8 == 1, "act_mx8 must be 0 or 1");
+  need(!cfg.act_mx8 || (dt == MONO_MXFP4 && cfg.round_bf16 && cfg.hidden % 128 == 0 && cfg.inter % 128 == 0 &&
+                        cfg.hidden <= kMx8MaxK && cfg.inter <= kMx8MaxK),
+       "act_mx8 needs MXFP4 experts on the tensor cores (round_bf16, hidden and inter multiples of 128, at most " +
+           std::to_string(kMx8MaxK) + ")");
   if (dt >= MONO_F32 && dt <= MONO_MXFP4 && cfg.hidden > 0 && cfg.inter > 0) {
     const int m = std::max(unit_elems(dt), block_of(dt));
     need(cfg.hidden % m == 0, "hidden must be a multiple of " + std::to_string(m) + " for this expert format");
@@ -521,6 +528,7 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
     }
   }
   if (!rc) rc = dalloc(p, &p->mix_part, (size_t)p->G * RM * kMixP * 4, &p->scratch_bytes);
+  if (!rc) rc = dalloc(p, &p->mix_tot, (size_t)RM * kMixP * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->abuf, (size_t)RM * H * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->sq_part, (size_t)RM * p->G * 4, &p->scratch_bytes);
   if (!rc) rc = dalloc(p, &p->logits, (size_t)RM * E * 4, &p->scratch_bytes);
@@ -812,6 +820,7 @@ int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd
     prm.layer = l;
     prm.first = l == 0 && !pd;
     prm.dense = p->cfg.dense;
+    prm.mx8 = p->cfg.act_mx8;
     prm.last = l == L - 1;
     prm.mix_ctas = p->mix_ctas;
     prm.hc_bf16 = p->cfg.hc_dtype == MONO_BF16;
@@ -856,6 +865,7 @@ int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd
     prm.gu_estride = p->gu_estride;
     prm.dn_estride = p->dn_estride;
     prm.mix_part = p->mix_part;
+    prm.mix_tot = p->mix_tot;
     prm.abuf = p->abuf;
     prm.sq_part = p->sq_part;
     prm.logits = p->logits;

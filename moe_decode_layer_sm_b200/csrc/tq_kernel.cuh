@@ -75,6 +75,28 @@ constexpr uint32_t kF8Acc = 4;
 static_assert(kF8Acc <= (uint32_t)kMaxAcc, "accumulator barriers");
 static_assert(kF4SfaCol + 8 * kF4MaxSlots <= kF4SfbNCol && kF4SfbNCol + 4 <= kF4SfbDnCol, "tensor memory");
 
+// MXFP8 activations (act_mx8): one e4m3 term per token row (B has N = 8 rows)
+// with an e8m0 scale per 32 values; tensor memory: 2 accumulators [0, 64), A
+// scales 8 columns per ring slot [64, 96), B scales one 4-column group per
+// 128 of the contraction from 96 (n's in the gate/up phase, a down expert's
+// activations in the down phase).
+constexpr uint32_t kMx8Acc = 2;
+constexpr uint32_t kMx8SfaCol = 64;
+constexpr uint32_t kMx8SfbCol = 96;
+constexpr int kMx8MaxK = (kF4TmemCols - (int)kMx8SfbCol) / 4 * 128;   // 40 groups: 5120
+static_assert(kMx8SfaCol + 8 * kF4MaxSlots <= kMx8SfbCol, "tensor memory");
+// a down expert's operand: codes [I/16][8 rows][16], then one 512-byte scale
+// chunk per 128 of I (lane n = row, byte j = 32-block j)
+__host__ __device__ inline size_t mx8_act_stride(int I) { return (size_t)I * 8 + (size_t)(I / 128) * kF4Sf; }
+
+// The e8m0 exponent X of a block of MXFP8 values (OCP MX rule: floor(log2
+// amax) - 8, at least -127), from amax as fp32 bits; 0 codes for amax = 0.
+__device__ __forceinline__ int mx8_exp(uint32_t amax_bits) {
+  const int e = (int)((amax_bits >> 23) & 0xFFu);
+  if (e == 0) return -127;              // zero or subnormal amax: the smallest scale
+  return max(-127, e - 127 - 8);
+}
+
 // bytes of one expert entry's down B operand: [I/16][16 rows][16] e4m3 codes,
 // then [I/128][8] fp32 inverse scales; with MXFP4 (block-scaled MMAs) also
 // the same scales as e8m0 B scale factors, one 512-byte chunk per 4 blocks:
@@ -154,6 +176,58 @@ __device__ void f8_convert_n(const Params& p, Ctl* c, uint8_t* regA) {
   }
 }
 
+// n, bf16 in the layout [H/8][8 rows][8], becomes MXFP8: e4m3 codes
+// [H/16][8 rows][16] in place (the B operand of N = 8), and one e8m0 scale
+// per (row, 32 columns) into sf[unit][row] (4 bytes: the unit's 32-blocks)
+// for the tensor-memory copy.  Lane (r, q) of a warp takes columns 32q ..
+// 32q + 31 of row r of a 128-column block: exactly one 32-block, so its
+// scale needs no exchange.  Blocks go in waves of one per warp; a wave
+// reads all its inputs before any output is written, and a block's output
+// (1 KB at kb KB) only overlaps the input of block kb / 2, which an earlier
+// wave (or this one, before its barrier) has read.  Compute warps.
+__device__ void mx8_convert_n(const Params& p, uint8_t* regA, uint32_t* sf) {
+  const int H = p.H, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane & 7, q = lane >> 3, nb = H / 128;
+  for (int kb0 = 0; kb0 < nb; kb0 += kCW) {
+    const int kb = kb0 + warp;
+    uint4 v[4];
+    if (kb < nb) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) v[cc] = *reinterpret_cast<const uint4*>(regA + (size_t)(kb * 16 + 4 * q + cc) * 128 + r * 16);
+    }
+    bar_sync(kBarCons, kCW * 32);
+    if (kb < nb) {
+      float x[32];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        x[8 * cc + 0] = bf16lo(v[cc].x); x[8 * cc + 1] = bf16hi(v[cc].x);
+        x[8 * cc + 2] = bf16lo(v[cc].y); x[8 * cc + 3] = bf16hi(v[cc].y);
+        x[8 * cc + 4] = bf16lo(v[cc].z); x[8 * cc + 5] = bf16hi(v[cc].z);
+        x[8 * cc + 6] = bf16lo(v[cc].w); x[8 * cc + 7] = bf16hi(v[cc].w);
+      }
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(x[k]));
+      const int X = mx8_exp(__float_as_uint(m));
+      const float inv = pow2i(-X);   // X <= 120 for finite bf16 values, so 2^-X is a normal float
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * k] * inv, x[4 * k + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(x[4 * k + 2] * inv, x[4 * k + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        w[k] = lo | (hi << 16);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<uint4*>(regA + (size_t)(kb * 8 + 2 * q + h) * 128 + r * 16) =
+            make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+      reinterpret_cast<uint8_t*>(sf)[((size_t)kb * 8 + r) * 4 + q] = m > 0.f ? (uint8_t)(X + 127) : (uint8_t)0;
+    }
+    bar_sync(kBarCons, kCW * 32);
+  }
+}
+
 // A complete gate/up block: SwiGLU, then each token row's 128 activations of
 // the block as e4m3 hi/lo under the block's power-of-two scale, into the
 // down B operand of expert entry x, with the inverse scale behind the codes;
@@ -214,6 +288,50 @@ __device__ __forceinline__ void f8_store_act(const Params& p, Ctl* c, const Seg&
   }
   // the block's activations are out: count it for its expert (the codes are
   // read by a bulk copy, the async proxy; the scales by the epilogues)
+  __threadfence();
+  bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
+  if (tid == 0 && live && may_publish(p, c->epoch, 0, 8) && !(p.fault_stage == 4 && x == 0 && sg.blk == 0)) {
+    fence_proxy_async_global();
+    red_release_add(&p.xready[x], 1u);
+  }
+}
+
+// MXFP8 activations: a complete gate/up block's SwiGLU as e4m3 codes of the
+// down B operand [I/16][8 rows][16] of expert entry x, each token row's 32
+// channels of a warp under their own e8m0 scale (OCP MX rule), the scale
+// byte at lane r, byte = warp, of the block's 512-byte chunk; zero for rows
+// that do not use the expert.  Then the block counts for its expert.  Every
+// epilogue thread, live or not.
+__device__ __forceinline__ void mx8_store_act(const Params& p, Ctl* c, const Seg& sg, bool live, int i,
+                                              const float (&a)[8], const float (&b)[8]) {
+  const int R = p.R, K = p.K, I = p.I, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int x = sg.x;
+  uint8_t* base = p.actb + (size_t)x * mx8_act_stride(I);
+  const int ch = sg.blk * 128 + i;
+  uint8_t* dst = base + (size_t)(ch >> 4) * 128 + (ch & 15);
+  uint8_t* sfc = base + (size_t)I * 8 + (size_t)sg.blk * kF4Sf;
+#pragma unroll
+  for (int r = 0; r < kMaxR; ++r) {
+    const int sl = x == 0 ? K : c->uslot[x - 1][r];
+    float act = 0.f;
+    if (live && r < R && sl >= 0) {
+      float gg = a[r], uu = b[r];
+      if (p.round_bf16) {
+        gg = round_bf16(gg);
+        uu = round_bf16(uu);
+      }
+      act = gg / (1.0f + expf(-gg)) * uu;
+    }
+    const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(act)));
+    const int X = mx8_exp(mb);
+    const uint32_t code = __nv_cvt_float2_to_fp8x2(make_float2(act * pow2i(-X), 0.f), __NV_SATFINITE, __NV_E4M3);
+    if (live) {
+      dst[r * 16] = (uint8_t)(code & 0xFFu);
+      if (lane == 0) sfc[16 * r + warp] = mb ? (uint8_t)(X + 127) : (uint8_t)0;
+    }
+  }
+  // the block's activations are out: count it for its expert (read by a
+  // bulk copy, the async proxy)
   __threadfence();
   bar_sync(kBarEpi, 4 * 32);   // reached by every epilogue thread, live or not
   if (tid == 0 && live && may_publish(p, c->epoch, 0, 8) && !(p.fault_stage == 4 && x == 0 && sg.blk == 0)) {
@@ -371,13 +489,19 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     bool ok = true;
     if (lane == 0) ok = wait_flag(p, c, &c->n_ready);
     ok = warp_ok(ok);
-    const uint32_t idesc = F4 ? umma_idesc_mx_e2m1_e4m3(128, 16) : umma_idesc_e4m3(128, 16);
+    const bool mx8 = F4 && p.mx8;
+    const uint32_t nacc = mx8 ? kMx8Acc : kF8Acc;
+    const uint32_t idesc =
+        F4 ? umma_idesc_mx_e2m1_e4m3(128, mx8 ? 8 : 16) : umma_idesc_e4m3(128, 16);
     // the down B operand: codes, and for MXFP4 also its e8m0 scale chunks
     // (the fp32 inverse scales between them are read by the epilogue only)
-    const uint32_t b_bytes = F4 ? (uint32_t)f8_act_stride(I, true) : (uint32_t)I * 16u;
+    const uint32_t b_bytes = mx8 ? (uint32_t)mx8_act_stride(I) : F4 ? (uint32_t)f8_act_stride(I, true) : (uint32_t)I * 16u;
     // B (n, or a down expert's activations): [K/16][16 rows][16], 256 bytes
-    // between K-neighbours, rows 8-15 128 bytes on; a unit is 2048 bytes
-    const uint64_t bdesc = umma_desc(smem_u32(regA), 256u, 128u);
+    // between K-neighbours, rows 8-15 128 bytes on, a unit 2048 bytes; with
+    // MXFP8 activations [K/16][8 rows][16]: 128 bytes between K-neighbours, a
+    // unit 1024 bytes
+    const uint64_t bdesc = mx8 ? umma_desc(smem_u32(regA), 128u, 128u) : umma_desc(smem_u32(regA), 256u, 128u);
+    const uint32_t bunit = mx8 ? 64u : 128u, bkstep = mx8 ? 16u : 32u;   // descriptor units per unit / K-step
     auto seg = [&](const Seg& sg) {
       const bool gu = sg.list != L_DN;
       if (!gu && sg.x != prev_x) {
@@ -396,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         if (ok) {   // (a copy whose wait failed is waited for again at exit)
           if (lane == 0) {
             mbar_arrive_expect_tx(&c->bfull, b_bytes);
-            tma_load_1d(regA, p.actb + (size_t)sg.x * f8_act_stride(I, F4), b_bytes, &c->bfull);
+            tma_load_1d(regA, p.actb + (size_t)sg.x * (mx8 ? mx8_act_stride(I) : f8_act_stride(I, F4)), b_bytes,
+                        &c->bfull);
             ok = wait_bar(p, c, &c->bfull, nb & 1u);
           }
           ok = warp_ok(ok);
@@ -404,7 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
           ++nb;
         }
         tc_fence_after();
-        if (F4 && ok) {
+        if (mx8 && ok) {
+          // the expert's activation scales: unit u's chunk to the 4-column
+          // group from kMx8SfbCol + 4u (n's scales there are no longer read:
+          // the drain above completed every gate/up MMA)
+          const uint8_t* sfb = regA + (size_t)I * 8;
+          for (int u = 0; u < I / 128; ++u)
+            tmem_cp_sf(tmem + kMx8SfbCol + 4u * u, umma_desc(smem_u32(sfb + (size_t)u * kF4Sf), 16u, 128u));
+        } else if (F4 && ok) {
           // the expert's activation scales: chunk g (blocks 4 g .. 4 g + 3)
           // to the 4 B-scale columns from kF4SfbDnCol + 4 g
           const uint8_t* sfb = regA + (size_t)I * 16 + (size_t)(I / 128) * 32;
@@ -420,9 +552,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         // buffer.  Stage s's A scale chunks go to the 8 columns of its ring
         // slot (gate 4 | up 4, or unit 0 | unit 1), free again once the
         // slot's MMAs are complete (which the producer waits for).
-        const uint32_t buf = t % kF8Acc;
-        if (t >= kF8Acc) {
-          if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / kF8Acc) - 1) & 1u);
+        const uint32_t buf = t % nacc;
+        if (t >= nacc) {
+          if (lane == 0 && ok) ok = wait_bar(p, c, &c->accempty[buf], ((t / nacc) - 1) & 1u);
           ok = warp_ok(ok);
         }
         tc_fence_after();
@@ -437,17 +569,20 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
             trace(p, 13, lane == 0);
           }
           const uint8_t* a_st = ring + (size_t)slot * p.slot_bytes;
-          const uint32_t sfa = tmem + kF4SfaCol + 8u * slot;
+          const uint32_t sfa = tmem + (mx8 ? kMx8SfaCol : kF4SfaCol) + 8u * slot;
           for (int j = 0; j < n && ok; ++j) {
             const int u = u0 + j;
             const uint8_t* a = a_st + (size_t)j * kF4SmemMat;   // gate/up: gate here, up 16 KB on
             const uint8_t* sf = a_st + kF4SfOff + j * kF4Sf;
-            // gate/up: n's scale per row (any byte); down: unit u's scale,
-            // byte u % 4 of the columns of its chunk
-            const uint32_t sfb = gu ? tmem + kF4SfbNCol : tmem + kF4SfbDnCol + 4u * (uint32_t)(u / 4);
-            umma_unit_mx(tmem + 32u * buf, umma_desc_sw128(smem_u32(a), 1024u), bdesc + (uint64_t)(u * 128), 32u,
+            // B scales.  MXFP8 activations: unit u's group, byte = K-block.
+            // Otherwise gate/up: n's scale per row (any byte); down: unit u's
+            // scale, byte u % 4 of the columns of its chunk
+            const uint32_t sfb = mx8 ? tmem + kMx8SfbCol + 4u * (uint32_t)u
+                                     : gu ? tmem + kF4SfbNCol : tmem + kF4SfbDnCol + 4u * (uint32_t)(u / 4);
+            const bool bstep = mx8 || gu;
+            umma_unit_mx(tmem + 32u * buf, umma_desc_sw128(smem_u32(a), 1024u), bdesc + (uint64_t)(u * bunit), bkstep,
                          idesc, sfa + 4u * j, umma_desc(smem_u32(sf), 16u, 128u), sfa + 4u,
-                         umma_desc(smem_u32(sf + kF4Sf), 16u, 128u), sfb, gu, gu ? 0u : (uint32_t)(u % 4),
+                         umma_desc(smem_u32(sf + kF4Sf), 16u, 128u), sfb, bstep, bstep ? 0u : (uint32_t)(u % 4),
                          u > sg.k0, gu);
           }
           umma_commit_warp(&empty[slot]);
@@ -523,10 +658,23 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   // the router reads n as bf16 (the layer's values); the MMAs then take it
   // as e4m3 hi/lo
   router_logits<true>(p, c, regA, false);
-  f8_convert_n(p, c, regA);
+  const bool mx8 = F4 && p.mx8;
+  uint32_t* mx8_sf = reinterpret_cast<uint32_t*>(c->red);   // [H/128][8] scale words of n (the prologue is done with red)
+  if (mx8) mx8_convert_n(p, regA, mx8_sf);
+  else f8_convert_n(p, c, regA);
   fence_proxy_async_smem();   // n is read by the tensor cores (async proxy)
   bar_sync(kBarCons, kCW * 32);
-  if (F4 && warp < 4) {
+  if (mx8 && warp < 4) {
+    // n's scales as the B scale factors of the gate/up MMAs: 128-unit u in
+    // the 4-column group from kMx8SfbCol + 4u, lane n = row, byte j = its
+    // 32-block j, in every lane quarter
+    const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16) + kMx8SfbCol;
+    for (int u = 0; u < H / 128; ++u)
+      tmem_st4(tq + 4u * u, lane < 8 ? mx8_sf[u * 8 + lane] : 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+    tmem_st_wait();
+    tc_fence_before();
+  }
+  if (F4 && !mx8 && warp < 4) {
     // n's row scales as the B scale factors of the gate/up MMAs: lane n of
     // every lane quarter holds B row n's e8m0 code (rows 8-15, the lo terms,
     // share their token row's scale) in every byte of its first column
@@ -563,9 +711,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     const int i = tid;
     uint32_t t = 0;
     bool ok = true;
-    auto take = [&](uint32_t* v, uint32_t* w2, bool gu) {   // the next unit's tile
-      const uint32_t buf = t % kF8Acc;
-      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / kF8Acc) & 1u);
+    const uint32_t nacc = mx8 ? kMx8Acc : kF8Acc;
+    auto take = [&](uint32_t* v, uint32_t* w2, bool gu) {   // the next unit's (or MXFP4 segment's) tile
+      const uint32_t buf = t % nacc;
+      if (ok) ok = wait_bar(p, c, &c->accfull[buf], (t / nacc) & 1u);
       tc_fence_after();
       const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + 32u * buf;
       tmem_ld16(ta, v);
@@ -588,14 +737,15 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
         // hi (rows 0-7) and lo (rows 8-15) columns of each token row added
         take(v, w2, gu);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          a[r] = __uint_as_float(v[r]) + __uint_as_float(v[8 + r]);
-          b[r] = gu ? __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]) : 0.f;
+        for (int r = 0; r < 8; ++r) {   // MXFP8 activations: one term (N = 8)
+          a[r] = mx8 ? __uint_as_float(v[r]) : __uint_as_float(v[r]) + __uint_as_float(v[8 + r]);
+          b[r] = !gu ? 0.f : mx8 ? __uint_as_float(w2[r]) : __uint_as_float(w2[r]) + __uint_as_float(w2[8 + r]);
         }
         trace(p, 20, t == 1 && tid == 0);
         const bool live = ok && !c->dead;
         if (!epi_combine(p, c, geo, sg, upb, gu, live, i, a, b)) return;
-        if (gu) f8_store_act(p, c, sg, live, i, a, b, true);
+        if (gu && mx8) mx8_store_act(p, c, sg, live, i, a, b);
+        else if (gu) f8_store_act(p, c, sg, live, i, a, b, true);
         else epi_store(p, c, geo, sg, false, live, i, a, b);
         return;
       }

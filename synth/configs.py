@@ -81,4 +81,8 @@ def scaled(w: Workload, hidden=1024, n_routed=32, top_k=4, inter=512, **kw) -> W
                    inter=inter, **kw)
 
 
-BY_NAME = {w.name: w for w in FULL + [DENSE6_BF16_R1]}
+# the MXFP4 chain with the MXFP8-activation numerics (vLLM MonoKernel page,
+# Numerics): not one of the five configurations; a parity and bench case
+FLASH_MXFP4_MX8_CHAIN4_R8 = FLASH_MXFP4_CHAIN4_R8.with_(name="v41flash-mxfp4-mx8act-chain4-r8", act_mx8=True)
+
+BY_NAME = {w.name: w for w in FULL + [DENSE6_BF16_R1, FLASH_MXFP4_MX8_CHAIN4_R8]}

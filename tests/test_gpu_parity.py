@@ -208,6 +208,29 @@ def test_scaled_mxfp4_single_layer():
     run.close()
 
 
+@pytest.mark.parametrize("rows", [8, 3])
+def test_scaled_mxfp4_mxfp8_activations(rows):
+    """MXFP4 experts with MXFP8 activations (one e4m3 term per row under an
+    e8m0 scale per 32 values, block-scaled MMAs with N = 8) against the
+    oracle's act_mx8 numerics."""
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, n_layers=1, seed=461 + rows, rows=rows, act_mx8=True)
+    run = LayerRun(wl)
+    run.step()
+    _check_layer(wl, run, list(range(wl.rows)))
+    run.close()
+
+
+def test_scaled_mxfp4_mxfp8_activations_chain():
+    wl = C.scaled(C.FLASH_MXFP4_CHAIN4_R8, seed=471, act_mx8=True)
+    run = LayerRun(wl)
+    got = run.step()
+    lws = [O.LayerWeights(wl, S.cpu_dense(wl, l), all_experts(wl, l)) for l in range(wl.n_layers)]
+    for l, lw in enumerate(lws):
+        nxt = run.tap(l + 1, "x") if l + 1 < wl.n_layers else got
+        check_chain_layer(wl, run, l, lw, nxt)
+    run.close()
+
+
 @pytest.mark.parametrize("wdt, rows", [("bf16", 8), ("mxfp4", 8), ("bf16", 2), ("mxfp4", 1)])
 def test_scaled_chain_four_layers(wdt, rows):
     """Every layer of the chain, every row, checked on the residual streams
