@@ -339,7 +339,9 @@ int mono_ffn_debug_jitter(mono_ffn_plan_t* plan, unsigned max_ns);
  * in time on one device (other streams, other threads) share the scratch and
  * race: order them.  The first call on each device looks the scratch address
  * up (cudaGetSymbolAddress, which may load the module); make that first call
- * outside stream capture. */
+ * outside stream capture.  The address is kept for the life of the process:
+ * after cudaDeviceReset on a device, do not call this entry point on that
+ * device again. */
 int mono_ffn_route_noalloc(int rows, int hidden, int n_routed, int top_k, const void* n, int n_bf16,
                            const float* router_w, const float* router_bias, float route_scale, float denom_clamp,
                            int* idx, float* w, void* stream);

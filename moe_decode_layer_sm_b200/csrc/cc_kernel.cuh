@@ -185,6 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
   const int R = p.R, H = p.H, I = p.I, E = p.E, K = p.K, G = p.G;
   const bool nbf = p.round_bf16 != 0;   // n is stored as bf16 exactly when it is rounded to bf16
 
+  // launched behind another grid of the stream (programmatic dependent
+  // launch), this grid may be resident before that one has finished: nothing
+  // it wrote is read before this point
+  grid_dep_wait();
   if (tid == 0) {
     c->dead = 0;
     c->lists_ready = 0;
@@ -199,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dep_launch();   // the next layer's grid may take each SM as this grid leaves it
   if (c->dead) return;
   const uint32_t ep1 = c->epoch + 1u;
   trace(p, 0, tid == 0);

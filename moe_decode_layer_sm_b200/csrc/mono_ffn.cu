@@ -68,6 +68,7 @@ struct mono_ffn_plan_s {
   void* stage_in = nullptr;
   void* stage_out = nullptr;
   int64_t packed_bytes = 0, scratch_bytes = 0;
+  bool pdl_ok = true;   // a chain's later layers launch as programmatic dependents
   int fault_cta = -1;
   int fault_stage = 0;
   unsigned jitter_ns = 0;
@@ -901,13 +902,26 @@ int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd
     lc.blockDim = dim3(kThreads);
     lc.dynamicSmemBytes = p->smem;
     lc.stream = (cudaStream_t)stream;
-    cudaLaunchAttribute attr[1];
+    // cooperative: every CTA resident at once (the grid-wide stages wait on
+    // one another); a chain's later layers also as programmatic dependent
+    // launches, so that each starts launching while the layer before it ends
+    // (the kernel waits for that layer before it reads anything)
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
-    lc.numAttrs = 1;
+    lc.numAttrs = (l > 0 && p->pdl_ok) ? 2 : 1;
     void* args[] = {&prm};
     e = cudaLaunchKernelExC(&lc, kfn, args);
+    if (e != cudaSuccess && lc.numAttrs == 2) {
+      // the driver refused the combination: launch as before from now on
+      cudaGetLastError();
+      p->pdl_ok = false;
+      lc.numAttrs = 1;
+      e = cudaLaunchKernelExC(&lc, kfn, args);
+    }
   }
   if (prev != p->cfg.device) cudaSetDevice(prev);
   if (e != cudaSuccess) return cuda_fail(p, e, "step launch");

@@ -293,6 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   const int R = p.R, H = p.H, I = p.I, K = p.K, G = p.G;
   const TcGeo geo(p);
 
+  // launched behind another grid of the stream (programmatic dependent
+  // launch), this grid may be resident before that one has finished: nothing
+  // it wrote is read before this point
+  grid_dep_wait();
   if (tid == 0) {
     c->dead = 0;
     c->lists_ready = 0;
@@ -314,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dep_launch();   // the next layer's grid may take each SM as this grid leaves it
   if (c->dead) return;
   if (warp == kMmaWarp) tmem_alloc(&c->tmem_base, kTmemCols);
   tc_fence_before();

@@ -357,6 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
   const int H = p.H, I = p.I, K = p.K, G = p.G;
   const TcGeo geo(p);
 
+  // launched behind another grid of the stream (programmatic dependent
+  // launch), this grid may be resident before that one has finished: nothing
+  // it wrote is read before this point
+  grid_dep_wait();
   if (tid == 0) {
     c->dead = 0;
     c->lists_ready = 0;
@@ -378,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dep_launch();   // the next layer's grid may take each SM as this grid leaves it
   if (c->dead) return;
   constexpr int kCols = F4 ? kF4TmemCols : kF8TmemCols;
   if (warp == kMmaWarp) tmem_alloc(&c->tmem_base, kCols);
