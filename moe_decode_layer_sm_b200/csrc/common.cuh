@@ -223,21 +223,25 @@ __device__ __forceinline__ void record_error(const Params& p, Ctl* c, uint32_t c
 __device__ bool wait_count(const Params& p, Ctl* c, const uint32_t* cnt, uint32_t target, uint32_t stage) {
   volatile int* dead = &c->dead;
   uint64_t t0 = globaltimer();
-  uint32_t ns = 32;
+  uint32_t ns = 32, it = 0;
   while (true) {
     if (*dead) return false;
     uint32_t v = ld_acquire(cnt);
     if ((int32_t)(v - target) >= 0) return true;
-    if (ld_relaxed(&p.err->abort)) {
-      c->dead = 1;
-      return false;
-    }
-    if (globaltimer() - t0 > p.timeout_ns) {
-      record_error(p, c, 7u, stage);   // MONO_ERR_DEVICE_TIMEOUT (negated on the host)
-      return false;
+    // the abort word and the clock every eighth poll, so that a poll is one
+    // round trip (an acquire load orders the loads after it)
+    if ((++it & 7u) == 0u) {
+      if (ld_relaxed(&p.err->abort)) {
+        c->dead = 1;
+        return false;
+      }
+      if (globaltimer() - t0 > p.timeout_ns) {
+        record_error(p, c, 7u, stage);   // MONO_ERR_DEVICE_TIMEOUT (negated on the host)
+        return false;
+      }
     }
     __nanosleep(ns);
-    if (ns < 256) ns <<= 1;
+    if (ns < 128) ns <<= 1;
   }
 }
 
