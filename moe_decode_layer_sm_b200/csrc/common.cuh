@@ -414,27 +414,20 @@ __device__ __forceinline__ void load8(const uint8_t* base, size_t i, bool bf, fl
   }
 }
 
-// Router select of one row by one warp: score = sqrt(softplus(logit)) in
-// fp32, sel = score + bias, canonical top-k by (sel desc, index asc) through
-// warp max / min reductions, then weight = score / max(sum, clamp) * scale
-// with each op rounded to fp32.  Lane l holds experts l + 32 q, q < NQ.
-// dry: run the same code without storing anything (it is then warm in the
-// SM's instruction cache when the real call comes); not inlined, so that the
-// dry and the real call share one copy of the code.
-template <int NQ>
-__device__ __noinline__ void topk_row(const Params& p, Ctl* c, int r, bool dry) {
+// The router select of one row by one warp, from each expert's logit and
+// bias (lane l holds experts l + 32 q, q < NQ; experts >= E are ignored):
+// score = sqrt(softplus(logit)) in fp32, sel = score + bias, the canonical
+// top-k by (sel desc, index asc) through warp max / min reductions, then
+// weight = score / max(sum, clamp) * scale with each op rounded to fp32.
+// put_idx(j, e) runs on lane 0 for selection j; after a warp sync,
+// put_w(j, w) runs on lane j < K.  Shared by the fused kernels' top-k and
+// the allocation-free router select, so the two cannot drift apart.
+template <int NQ, class FI, class FW>
+__device__ __forceinline__ void select_row(const float (&lg)[NQ], const float (&bs)[NQ], int E, int K, float denom_clamp,
+                                           float route_scale, FI put_idx, FW put_w) {
   const int lane = threadIdx.x & 31;
-  const int E = p.E, K = p.K;
   float score[NQ];
   uint32_t key[NQ];
-  // every load first (a store in between would order them one by one)
-  float lg[NQ], bs[NQ];
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    const int e = lane + 32 * q;
-    lg[q] = (e < E && !c->dead) ? __ldcg(p.logits + (size_t)r * E + e) : 0.f;
-    bs[q] = e < E ? __ldg(p.bias + e) : 0.f;
-  }
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
     const int e = lane + 32 * q;
@@ -446,46 +439,72 @@ __device__ __noinline__ void topk_row(const Params& p, Ctl* c, int r, bool dry) 
       key[q] = ord_key(score[q] + bs[q]);
     }
   }
-  if (blockIdx.x == 0 && p.taps.logits && !dry) {
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-      if (lane + 32 * q < E) p.taps.logits[(size_t)r * E + lane + 32 * q] = lg[q];
-  }
-  trace(p, 26, r == 0 && lane == 0 && !dry);
   uint32_t taken = 0u;
   float ssum = 0.f, wsel = 0.f;
   for (int j = 0; j < K; ++j) {
     uint32_t bk = 0u;
     int be = 0x7FFFFFFF;
-    float bs = 0.f;
+    float bsc = 0.f;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       if (!((taken >> q) & 1u) && key[q] > bk) {
         bk = key[q];
         be = lane + 32 * q;
-        bs = score[q];
+        bsc = score[q];
       }
     }
     const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
     const int we = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(bk == wk ? be : 0x7FFFFFFF));
     const int wl = we & 31;
     if (we < E && wl == lane) taken |= 1u << (we >> 5);
-    const float ws = __shfl_sync(0xffffffffu, bs, wl);
+    const float ws = __shfl_sync(0xffffffffu, bsc, wl);
     if (lane == j) wsel = ws;   // lane j keeps the j-th raw score
-    if (lane == 0 && !dry) c->idx[r][j] = we < E ? we : 0;
+    if (lane == 0) put_idx(j, we < E ? we : 0);
     ssum += ws;   // selection order, fp32
   }
   __syncwarp();
-  if (lane < K && !dry) {
-    const float den = fmaxf(ssum, p.denom_clamp);
-    const float w = __fmul_rn(__fdiv_rn(wsel, den), p.route_scale);
-    c->wt[r][lane] = w;
-    if (blockIdx.x == 0) {
-      if (p.taps.idx) p.taps.idx[r * K + lane] = c->idx[r][lane];
-      if (p.taps.w) p.taps.w[r * K + lane] = w;
-    }
+  if (lane < K) {
+    const float den = fmaxf(ssum, denom_clamp);
+    put_w(lane, __fmul_rn(__fdiv_rn(wsel, den), route_scale));
   }
   __syncwarp();
+}
+
+// The fused kernels' top-k of row r: every CTA's logits and the bias, then
+// select_row into the control block.  dry: run the same code without storing
+// anything (it is then warm in the SM's instruction cache when the real call
+// comes); not inlined, so that the dry and the real call share one copy.
+template <int NQ>
+__device__ __noinline__ void topk_row(const Params& p, Ctl* c, int r, bool dry) {
+  const int lane = threadIdx.x & 31;
+  const int E = p.E;
+  // every load first (a store in between would order them one by one)
+  float lg[NQ], bs[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = lane + 32 * q;
+    lg[q] = (e < E && !c->dead) ? __ldcg(p.logits + (size_t)r * E + e) : 0.f;
+    bs[q] = e < E ? __ldg(p.bias + e) : 0.f;
+  }
+  if (blockIdx.x == 0 && p.taps.logits && !dry) {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      if (lane + 32 * q < E) p.taps.logits[(size_t)r * E + lane + 32 * q] = lg[q];
+  }
+  trace(p, 26, r == 0 && lane == 0 && !dry);
+  select_row<NQ>(
+      lg, bs, E, p.K, p.denom_clamp, p.route_scale,
+      [&](int j, int e) {
+        if (!dry) c->idx[r][j] = e;
+      },
+      [&](int j, float w) {
+        if (dry) return;
+        c->wt[r][j] = w;
+        if (blockIdx.x == 0) {
+          if (p.taps.idx) p.taps.idx[r * p.K + j] = c->idx[r][j];
+          if (p.taps.w) p.taps.w[r * p.K + j] = w;
+        }
+      });
 }
 
 // A dense layer's "routing" of row r (one warp): every routed slot, in slot

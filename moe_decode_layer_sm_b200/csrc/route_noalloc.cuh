@@ -90,48 +90,20 @@ __global__ void __launch_bounds__(kRtThreads) route_noalloc_kernel(int R, int H,
   // the last block: logits = sum of the splits in order, then one warp per
   // row: scores, canonical (selection desc, index asc) top-k, weights
   for (int r = warp; r < R; r += kRtThreads / 32) {
-    uint32_t key[kRtMaxE / 32];
-    float score[kRtMaxE / 32];
+    float lg[kRtMaxE / 32], bs[kRtMaxE / 32];
 #pragma unroll
     for (int q = 0; q < kRtMaxE / 32; ++q) {
       const int ee = lane + 32 * q;
-      key[q] = 0u;
-      score[q] = 0.f;
+      lg[q] = 0.f;
+      bs[q] = 0.f;
       if (ee < E) {
-        float lg = 0.f;
-        for (int ss = 0; ss < kRtSplit; ++ss) lg += __ldcg(&sc->part[ss][r][ee]);
-        const float sp = fmaxf(lg, 0.f) + log1pf(expf(-fabsf(lg)));
-        score[q] = sqrtf(sp);
-        key[q] = ord_key(score[q] + __ldg(bias + ee));
+        for (int ss = 0; ss < kRtSplit; ++ss) lg[q] += __ldcg(&sc->part[ss][r][ee]);
+        bs[q] = __ldg(bias + ee);
       }
     }
-    uint32_t taken = 0u;
-    float ssum = 0.f, wsel = 0.f;
-    for (int j = 0; j < K; ++j) {
-      uint32_t bk = 0u;
-      int be = 0x7FFFFFFF;
-      float bs = 0.f;
-#pragma unroll
-      for (int q = 0; q < kRtMaxE / 32; ++q) {
-        if (!((taken >> q) & 1u) && key[q] > bk) {
-          bk = key[q];
-          be = lane + 32 * q;
-          bs = score[q];
-        }
-      }
-      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-      const int we = (int)__reduce_min_sync(0xffffffffu, (uint32_t)(bk == wk ? be : 0x7FFFFFFF));
-      const int wl = we & 31;
-      if (we < E && wl == lane) taken |= 1u << (we >> 5);
-      const float ws = __shfl_sync(0xffffffffu, bs, wl);
-      if (lane == j) wsel = ws;
-      if (lane == 0) idx[r * K + j] = we < E ? we : 0;
-      ssum += ws;   // selection order, fp32
-    }
-    if (lane < K) {
-      const float den = fmaxf(ssum, denom_clamp);
-      wout[r * K + lane] = __fmul_rn(__fdiv_rn(wsel, den), route_scale);
-    }
+    select_row<kRtMaxE / 32>(
+        lg, bs, E, K, denom_clamp, route_scale, [&](int j, int e) { idx[r * K + j] = e; },
+        [&](int j, float wv) { wout[r * K + j] = wv; });
   }
   __syncthreads();
   if (threadIdx.x == 0) atomicExch(&sc->arrivals, 0u);   // ready for the next call

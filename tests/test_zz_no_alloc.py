@@ -1,7 +1,7 @@
 """mono_ffn_route_noalloc (router select with no plan and no allocation)
 against the fused step's own routing: same normed rows n, same router
-weights and bias, two calls in a row; and at its size limits against a
-float64 restatement of the select.  The file name puts it last in
+weights and bias, two calls in a row; at its size limits against a
+float64 restatement of the select; and captured in a CUDA graph.  The file name puts it last in
 collection, so that a run stopping at the first failure has run every other
 test first; it passes alone in a fresh process and after the others."""
 
@@ -119,3 +119,36 @@ def test_route_noalloc_binding_checks_its_arguments():
         binding.route_noalloc(n, rw, rb, 4, 2.5, 1e-20, torch.zeros(2, 4), torch.zeros(2, 4))
     with pytest.raises(ValueError, match=r"\[rows\]\[top_k\]"):
         binding.route_noalloc(n, rw, rb, 4, 2.5, 1e-20, torch.zeros(2, 3, dtype=torch.int32), torch.zeros(2, 3))
+
+
+@pytest.mark.gpu
+def test_route_noalloc_inside_a_captured_graph():
+    """The call between captured graph segments, the case it exists for: after
+    one eager call (which looks up the scratch), one call is captured into a
+    CUDA graph; replaying the graph gives the eager call's bytes, and the
+    replays allocate no device memory."""
+    import torch
+    g = torch.Generator().manual_seed(1001)
+    R, H, E, K = 4, 1024, 256, 8
+    n = torch.randn(R, H, generator=g).to(torch.bfloat16).cuda()
+    rw = (torch.randn(H, E, generator=g) / H ** 0.5).float().cuda()
+    rb = (torch.rand(E, generator=g) * 0.2 - 0.1).float().cuda()
+    idx0 = torch.full((R, K), -1, dtype=torch.int32, device="cuda")
+    w0 = torch.zeros((R, K), dtype=torch.float32, device="cuda")
+    binding.route_noalloc(n, rw, rb, K, 2.5, 1e-20, idx0, w0)
+    torch.cuda.synchronize()
+    idx = torch.full((R, K), -1, dtype=torch.int32, device="cuda")
+    w = torch.zeros((R, K), dtype=torch.float32, device="cuda")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        binding.route_noalloc(n, rw, rb, K, 2.5, 1e-20, idx, w)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        idx.fill_(-1)
+        w.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(idx, idx0) and torch.equal(w, w0)
+    assert torch.cuda.mem_get_info()[0] == free0
+    del graph
