@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
     c->dead = 0;
     c->lists_ready = 0;
     c->nu = 0;
-    c->epoch = ld_relaxed(&p.sync->epoch);
+    c->epoch = ld_relaxed(&p.sync->cnt_done);   // every grid counter's value at this launch's start
     c->live = live_rows(p);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
   __syncthreads();
   grid_dep_launch();   // the next layer's grid may take each SM as this grid leaves it
   if (c->dead) return;
-  const uint32_t ep1 = c->epoch + 1u;
+  const uint32_t ep1 = c->epoch + (uint32_t)G;   // every grid counter's target in this launch
   trace(p, 0, tid == 0);
 
   // ================================================================ producer
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
       __threadfence();
       red_release_add(&p.sync->cnt_act, 1u);
     }
-    wait_count(p, c, &p.sync->cnt_act, ep1 * (uint32_t)G, 4u);
+    wait_count(p, c, &p.sync->cnt_act, ep1, 4u);
   }
   int h0, h1;
   Walk::dn_range(p, h0, h1);

@@ -111,6 +111,7 @@ struct Params {
   CUtensorMap tm_gu; // MXFP4 tensor-core kernel: 2-D maps of the packed gate/up and down codes,
   CUtensorMap tm_dn; // rows of 128 e2m1 codes, unpacked into 16-byte slots, 128-byte swizzle
   int n_xready;
+  int n_xready_all;   // the plan's entries (max rows x top_k + 1): all cleared each launch
   uint8_t* actb;     // tensor-core kernel: [R*K+1][I/8][16][8] bf16 down-projection B operands
   float* gpart;      // tensor-core kernel: [G][4][128][16] partial gate|up tiles of split blocks
   float* dpart;      // tensor-core kernel: [G][2][128][16] partial down tiles
@@ -542,8 +543,8 @@ enum Phase { PH_SGU = 0, PH_RGU = 1, PH_DN = 2 };
 struct Walk {
   // shared expert gate/up: channels [c0, c1)
   __device__ static void sgu_range(const Params& p, int& c0, int& c1) {
-    c0 = (int)((long long)blockIdx.x * p.I / p.G);
-    c1 = (int)((long long)(blockIdx.x + 1) * p.I / p.G);
+    c0 = (int)(blockIdx.x * (uint32_t)p.I / (uint32_t)p.G);
+    c1 = (int)((blockIdx.x + 1) * (uint32_t)p.I / (uint32_t)p.G);
   }
   // routed gate/up over the unique-expert list: global channels [g0, g1)
   __device__ static void rgu_range(const Params& p, int nu, long long& g0, long long& g1) {
@@ -553,8 +554,8 @@ struct Walk {
   }
   // down: output channels [h0, h1) of every expert
   __device__ static void dn_range(const Params& p, int& h0, int& h1) {
-    h0 = (int)((long long)blockIdx.x * p.H / p.G);
-    h1 = (int)((long long)(blockIdx.x + 1) * p.H / p.G);
+    h0 = (int)(blockIdx.x * (uint32_t)p.H / (uint32_t)p.G);
+    h1 = (int)((blockIdx.x + 1) * (uint32_t)p.H / (uint32_t)p.G);
   }
 };
 
@@ -665,6 +666,8 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       for (int part = 0; part < P; ++part) acc += c->red[o * P + part];
       p.mix_part[(size_t)o * G + blockIdx.x] = acc;
     }
+    if (blockIdx.x == 0)
+      for (int i = ptid; i < p.n_xready_all; i += kPreThreads) p.xready[i] = 0u;
     bar_sync(kBarPre, kPreThreads);
     if (ptid == 0 && may_publish(p, c->epoch, 1, 0)) {
       __threadfence();
@@ -673,13 +676,17 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
     trace(p, 1, ptid == 0);
   }
 
-  if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix, ep1 * (uint32_t)G, 1u);
+  if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix, ep1, 1u);
   bar_sync(kBarPre, kPreThreads);
   trace(p, 2, ptid == 0);
   if (R <= 3) {
     // few outputs: every CTA's partials into shared memory at once (behind
     // the slices, which the collapse still needs), then lane-strided sums
-    // and a butterfly across the warp, in the same order in every CTA
+    // and a butterfly across the warp, in the same order in every CTA.
+    // The second-level counter still takes this CTA's arrival (nobody waits
+    // for it in this step): its wait target counts every step, so a later
+    // step with more rows finds it in step with the others.
+    if (ptid == 0) red_release_add(&p.sync->cnt_mix2, 1u);
     float* parts = reinterpret_cast<float*>(regA + L.parts);
     const int cap = (int)(((size_t)p.regA_bytes - L.parts) / sizeof(float) / G);   // outputs per pass
     for (int o0 = 0; o0 < nout; o0 += cap) {
@@ -705,7 +712,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
     // butterfly, so the same totals), publishes them, and after one more
     // grid stage every CTA reads all of them (a few hundred bytes instead of
     // every partial)
-    const int o0 = (int)((long long)blockIdx.x * nout / G), o1 = (int)((long long)(blockIdx.x + 1) * nout / G);
+    const int o0 = (int)(blockIdx.x * (uint32_t)nout / G), o1 = (int)((blockIdx.x + 1) * (uint32_t)nout / G);
     for (int o = o0 + pwarp; o < o1; o += kPreThreads / 32) {
       float acc = 0.f;
       if (!c->dead)
@@ -718,7 +725,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       __threadfence();
       red_release_add(&p.sync->cnt_mix2, 1u);
     }
-    if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix2, ep1 * (uint32_t)G, 1u);
+    if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix2, ep1, 1u);
     bar_sync(kBarPre, kPreThreads);
     for (int o = ptid; o < nout; o += kPreThreads) c->smix[o / kMixP][o % kMixP] = c->dead ? 0.f : __ldcg(p.mix_tot + o);
     bar_sync(kBarPre, kPreThreads);
@@ -786,7 +793,7 @@ __device__ void control_warps(const Params& p, Ctl* c, const uint8_t* regA, uint
   }
   if (ctl_topk) {
     // the top-k rows here, two warps over the rows
-    if (ct == 0 && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)G, 2u);
+    if (ct == 0 && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1, 2u);
     trace(p, 21, ct == 0);
     bar_sync(kBarCtl, kCtlWarps * 32);
     for (int r = cw; r < R; r += kCtlWarps) {
@@ -918,7 +925,7 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
       *reinterpret_cast<uint4*>(regA + n_off<true>(r, h, H, true)) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  if (ctid == 0) wait_count(p, c, &p.sync->cnt_a, ep1 * (uint32_t)G, 7u);
+  if (ctid == 0) wait_count(p, c, &p.sync->cnt_a, ep1, 7u);
   bar_sync(kBarCons, kCW * 32);
   trace(p, 24, ctid == 0);
   // every slice of a into the n area, 16 bytes at a time
@@ -996,7 +1003,7 @@ __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_
   if (p.dense) return;   // no router (and no logits stage) in a dense layer
   const int R = p.R, H = p.H, E = p.E, G = p.G, ctid = threadIdx.x, warp = ctid >> 5, lane = ctid & 31;
   const bool nbf = CANON || p.round_bf16;
-  const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
+  const int e0 = (int)(blockIdx.x * (uint32_t)E / G), e1 = (int)((blockIdx.x + 1) * (uint32_t)E / G);
   constexpr int kRq = 5;                  // float4 per thread and row per pass
   constexpr int kSpan = kRq * kCW * 32 * 4;   // columns per pass (5120)
   for (int e = e0; e < e1; e += 2) {
@@ -1062,7 +1069,7 @@ __device__ void route_rows(const Params& p, Ctl* c, uint32_t ep1, bool split) {
   const int R = p.R, warp = threadIdx.x >> 5;
   const int w0 = split ? 4 : 0, nw = kCW - w0;
   const bool lead = (int)threadIdx.x == w0 * 32;
-  if (lead && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1 * (uint32_t)p.G, 2u);
+  if (lead && !p.dense) wait_count(p, c, &p.sync->cnt_logit, ep1, 2u);
   if (split) bar_sync(kBarTop, 4 * 32);
   else bar_sync(kBarCons, kCW * 32);
   trace(p, 21, lead);
@@ -1110,19 +1117,15 @@ __device__ void tail(const Params& p, Ctl* c, YF yfun) {
   }
 }
 
-// The CTA's arrival at the end counter; the last CTA of the step advances the
-// layer's epoch.  Compute thread 0.
+// The CTA's arrival at the end counter, with no round trip: the next launch
+// on this layer slot reads the counter as the value every grid counter holds
+// at its start (each takes one arrival per CTA per launch), and its CTA 0
+// clears the per-expert readiness counts in its prologue.  Compute thread 0.
 __device__ __forceinline__ void finish_step(const Params& p, Ctl* c, uint32_t ep1) {
+  (void)ep1;
   if (threadIdx.x == 0 && !c->dead) {
     may_publish(p, c->epoch, 0, 3);
-    __threadfence();
-    const uint32_t old = atomicAdd(&p.sync->cnt_done, 1u);
-    if (old == ep1 * (uint32_t)p.G - 1u) {
-      // every CTA is past its last read of the per-expert counters
-      for (int i = 0; i < p.n_xready; ++i) p.xready[i] = 0u;
-      __threadfence();
-      atomicAdd(&p.sync->epoch, 1u);
-    }
+    red_release_add(&p.sync->cnt_done, 1u);
   }
 }
 

@@ -406,6 +406,10 @@ extern "C" int mono_ffn_plan(const mono_ffn_config* cfg_in, mono_ffn_plan_t** ou
              cfg.inter <= kF4MaxI,
          "MXFP4 on the tensor cores takes inter <= " + std::to_string(kF4MaxI));
   }
+  // the kernels partition every work list in 32-bit arithmetic: units x grid < 2^31
+  need((long long)(cfg.max_rows * cfg.top_k + 1) * ((cfg.inter + 127) / 128) * ((cfg.hidden + 127) / 128) * 1024 <
+           (1ll << 31),
+       "hidden x inter too large for the work partition");
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) why += "no CUDA device\n";
   else if (cfg.device < 0 || cfg.device >= ndev) why += "device ordinal out of range\n";
@@ -883,6 +887,7 @@ int step_impl(mono_ffn_plan_t* p, int rows, const void* hc_in, const Pending* pd
     prm.tm_gu = ls.tm_gu;
     prm.tm_dn = ls.tm_dn;
     prm.n_xready = p->xready ? rows * p->cfg.top_k + 1 : 0;
+    prm.n_xready_all = p->xready ? p->cfg.max_rows * p->cfg.top_k + 1 : 0;
     prm.sync = p->sync + l;
     prm.err = p->err;
     prm.taps = ls.taps;

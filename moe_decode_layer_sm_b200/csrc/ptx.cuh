@@ -73,6 +73,11 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// one cache line to L2 through the load path
+__device__ __forceinline__ void prefetch_l2_line(const void* src) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(src) : "memory");
+}
+
 // L2 prefetch of the 16-byte granules inside [src, src + bytes)
 __device__ __forceinline__ void prefetch_l2_span(const void* src, size_t bytes) {
   const uintptr_t a = ((uintptr_t)src + 15) & ~(uintptr_t)15;

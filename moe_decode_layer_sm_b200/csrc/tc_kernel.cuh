@@ -47,11 +47,16 @@ struct Seg {
   long long gblk, N;
 };
 
-__device__ __forceinline__ long long part_start(long long N, int G, int c) { return (long long)c * N / G; }
+// 32-bit arithmetic: the plan keeps every list's units times the grid below
+// 2^31 (64-bit division is a long software sequence, on the critical path of
+// every segment's combine)
+__device__ __forceinline__ long long part_start(long long N, int G, int c) {
+  return (long long)((uint32_t)c * (uint32_t)N / (uint32_t)G);
+}
 
 // the CTA whose range holds unit u
 __device__ __forceinline__ int part_owner(long long N, int G, long long u) {
-  int c = (int)((u * G) / N);
+  int c = (int)((uint32_t)u * (uint32_t)G / (uint32_t)N);
   while (c + 1 < G && part_start(N, G, c + 1) <= u) ++c;
   while (c > 0 && part_start(N, G, c) > u) --c;
   return c;
@@ -109,13 +114,13 @@ __device__ __forceinline__ void tc_segments(const Params& p, const TcGeo& g, int
   const long long N = nexp * nb * upb;
   long long a = part_start(N, p.G, blockIdx.x), b = part_start(N, p.G, blockIdx.x + 1);
   while (a < b) {
-    const long long gb = a / upb;
-    const int k0 = (int)(a % upb);
+    const long long gb = (uint32_t)a / (uint32_t)upb;
+    const int k0 = (int)((uint32_t)a % (uint32_t)upb);
     const int k1 = (int)min((long long)upb, k0 + (b - a));
     Seg s;
     s.list = list;
-    s.x = list == L_SGU ? 0 : list == L_RGU ? (int)(gb / nb) + 1 : (int)(gb / nb);
-    s.blk = (int)(gb % nb);
+    s.x = list == L_SGU ? 0 : list == L_RGU ? (int)((uint32_t)gb / (uint32_t)nb) + 1 : (int)((uint32_t)gb / (uint32_t)nb);
+    s.blk = (int)((uint32_t)gb % (uint32_t)nb);
     s.k0 = k0;
     s.k1 = k1;
     s.gblk = gb;
@@ -297,12 +302,28 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   // launch), this grid may be resident before that one has finished: nothing
   // it wrote is read before this point
   grid_dep_wait();
+  if (threadIdx.x >= 32 && threadIdx.x < 64) {
+    // this CTA's slice of the mix weights and of the residual streams to L2
+    // while thread 0 sets up (the prologue's first loads then hit L2)
+    const int lane = threadIdx.x & 31;
+    int h0, h1;
+    Walk::dn_range(p, h0, h1);
+    const int nh = h1 - h0;
+    for (int sg = lane; sg < kS; sg += 32)
+      prefetch_l2_span(p.mix_w + ((size_t)sg * p.H + h0) * kMixC, (size_t)nh * kMixC * 4);
+    const int eb = p.hc_bf16 ? 2 : 4;
+    for (int q = lane; q < p.R * kS; q += 32) {
+      const uint8_t* row = reinterpret_cast<const uint8_t*>(p.x_prev) + ((size_t)q * p.H + h0) * eb;
+      for (int o = 0; o < nh * eb; o += 128) prefetch_l2_line(row + o);
+      prefetch_l2_line(row + nh * eb - 1);
+    }
+  }
   if (tid == 0) {
     c->dead = 0;
     c->lists_ready = 0;
     c->nu = 0;
     c->n_ready = 0;
-    c->epoch = ld_relaxed(&p.sync->epoch);
+    c->epoch = ld_relaxed(&p.sync->cnt_done);   // every grid counter's value at this launch's start
     c->live = live_rows(p);
     if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
@@ -324,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t ep1 = c->epoch + 1u;
+  const uint32_t ep1 = c->epoch + (uint32_t)G;   // every grid counter's target in this launch
   const uint32_t tmem = c->tmem_base;
   trace(p, 0, tid == 0);
   if (p.trace && tid == 0) {   // which SM this CTA runs on
@@ -366,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     if (lane == 0) {
       // the prologue's later inputs go to L2 ahead of the weight stream:
       // this CTA's router rows, the norm weights and the router bias
-      const int e0 = (int)((long long)blockIdx.x * p.E / G), e1 = (int)((long long)(blockIdx.x + 1) * p.E / G);
+      const int e0 = (int)(blockIdx.x * (uint32_t)p.E / G), e1 = (int)((blockIdx.x + 1) * (uint32_t)p.E / G);
       if (!p.dense) prefetch_l2_span(p.router_t + (size_t)e0 * H, (size_t)(e1 - e0) * H * 4);
       prefetch_l2_span(p.norm_w, (size_t)H * (p.norm_bf16 ? 2 : 4));
       prefetch_l2_span(p.bias, (size_t)p.E * 4);
@@ -610,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
 
   // ==================================================================== tail
   bar_sync(kBarCons, kCW * 32);
-  if (tid == 0) wait_count(p, c, &p.sync->cnt_y, ep1 * (uint32_t)G, 6u);
+  if (tid == 0) wait_count(p, c, &p.sync->cnt_y, ep1, 6u);
   bar_sync(kBarCons, kCW * 32);
   tail(p, c, [&](int r, int h) {
     const float* src = p.yp + (size_t)r * (K + 1) * H + h;

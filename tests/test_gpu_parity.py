@@ -127,6 +127,22 @@ def test_scaled_bf16(rows):
     run.close()
 
 
+@pytest.mark.parametrize("case", ["tiny-fp32", "scaled-bf16", "scaled-fp8"])
+def test_rows_vary_across_steps_on_one_plan(case):
+    """One plan stepped with row counts on both sides of the mix reduction's
+    one-level / two-level switch (3 | 4 rows): every grid counter must stay in
+    step with the others whatever path a step took, so no wait times out and
+    every step matches the oracle on its rows."""
+    wl, seq = {"tiny-fp32": (C.TINY_FP32.with_(rows=8, seed=120), [2, 8, 3, 5, 1]),
+               "scaled-bf16": (C.scaled(C.FLASH_BF16_R8, seed=121), [2, 8, 3, 5, 1]),
+               "scaled-fp8": (C.scaled(C.FLASH_FP8_R4, seed=122), [2, 4, 3, 4, 1])}[case]
+    run = LayerRun(wl)
+    for n in seq:
+        run.step(n)   # asserts that the device reported no error
+        _check_layer(wl, run, list(range(n)))
+    run.close()
+
+
 def test_scaled_fp8_rows4():
     wl = C.scaled(C.FLASH_FP8_R4, seed=301)
     run = LayerRun(wl)
