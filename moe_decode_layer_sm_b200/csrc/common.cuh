@@ -10,9 +10,11 @@
 //   warp  9      tensor-core issuer (tcgen05.mma) in the tensor-core kernel
 //   warps 10-11  control: Sinkhorn, the canonical top-k, the expert lists
 //
-// Grid-wide dependencies are epoch-tagged counters in global memory (no reset
-// between steps): a CTA publishes with a release-add and waits with acquire
-// loads until the counter reaches (epoch + 1) * contributors.  Every wait is
+// Grid-wide dependencies are counters in global memory that are never reset
+// between launches: each counter a kernel waits on takes one arrival (a
+// release-add) from every CTA in every launch, so at a launch's start it
+// holds the completion counter's value b, and a CTA waits with acquire loads
+// until it reaches b + grid (modulo 2^32, so wrap-safe).  Every wait is
 // bounded by the plan's timeout; on expiry the CTA records an error word,
 // raises the abort flag and runs the rest of its control flow without waiting
 // (so every named barrier is still reached), then returns.
