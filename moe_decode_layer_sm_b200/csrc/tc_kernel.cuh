@@ -319,13 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     }
   }
   if (tid == 0) {
+    // both grid words in flight at once, used after the barrier set-up
+    const uint32_t ep0 = ld_relaxed(&p.sync->cnt_done);
+    const uint32_t abort0 = ld_relaxed(&p.err->abort);
     c->dead = 0;
     c->lists_ready = 0;
     c->nu = 0;
     c->n_ready = 0;
-    c->epoch = ld_relaxed(&p.sync->cnt_done);   // every grid counter's value at this launch's start
-    c->live = live_rows(p);
-    if (ld_relaxed(&p.err->abort)) c->dead = 1;   // fail-stop after an unreported error
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -336,6 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     }
     mbar_init(&c->drain, 1);
     mbar_init(&c->bfull, 1);
+    c->epoch = ep0;
+    c->live = live_rows(p);
+    if (abort0) c->dead = 1;   // fail-stop after an unreported error
     fence_barrier_init();
   }
   __syncthreads();
