@@ -690,7 +690,7 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
     // step with more rows finds it in step with the others.
     if (ptid == 0) red_release_add(&p.sync->cnt_mix2, 1u);
     float* parts = reinterpret_cast<float*>(regA + L.parts);
-    const int cap = (int)(((size_t)p.regA_bytes - L.parts) / sizeof(float) / G);   // outputs per pass
+    const int cap = (int)((uint32_t)(p.regA_bytes - (int)L.parts) / 4u / (uint32_t)G);   // outputs per pass
     for (int o0 = 0; o0 < nout; o0 += cap) {
       const int no = min(cap, nout - o0);
       const int n4 = no * G / 4;   // G * 4 bytes is a multiple of 16 (the plan keeps G % 4 == 0)

@@ -174,6 +174,66 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
   const bool q1 = R > 4;
   const int slot = slot_of((int)blockIdx.x, sl0);
   float4* mine = reinterpret_cast<float4*>((gu ? p.gpart : p.dpart) + (((size_t)blockIdx.x * nsl + slot) * 128 + i) * 16);
+  if (!by_block) {
+    // A list cut in contiguous ranges: the block runs past c_lo's range, so
+    // c_lo's part is its last segment of the list, computed after every
+    // other holder's (each one's first segment, or its whole range).  c_lo
+    // adds the parts; the others publish theirs and go on.
+    uint32_t* cnt = (gu ? p.gcnt : p.dcnt) + (size_t)sg.x * (gu ? geo.nbi : geo.nbh) + sg.blk;
+    if ((int)blockIdx.x != c_lo) {
+      if (live) {
+        __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
+        if (q1) __stcg(mine + 1, make_float4(a[4], a[5], a[6], a[7]));
+        if (gu) __stcg(mine + 2, make_float4(b[0], b[1], b[2], b[3]));
+        if (gu && q1) __stcg(mine + 3, make_float4(b[4], b[5], b[6], b[7]));
+      }
+      __threadfence();
+      bar_sync(kBarEpi, 4 * 32);
+      if (tid == 0 && live && may_publish(p, c->epoch, 0, 5 + (uint32_t)sg.list)) red_release_add(cnt, 1u);
+      return false;
+    }
+    if (tid == 0 && live) {
+      int parts = 0;
+      for (int cc = c_lo; cc <= c_hi; ++cc) parts += holds(cc) ? 1 : 0;
+      if (wait_count(p, c, cnt, (uint32_t)(parts - 1), gu ? 4u : 6u)) *cnt = 0u;   // ready for the next step
+    }
+    bar_sync(kBarEpi, 4 * 32);
+    // this CTA's own part first (it is c_lo), then the others in CTA order,
+    // four in flight at a time: the additions of the general path below
+    for (int cb = c_lo + 1; cb <= c_hi; cb += 4) {
+      float4 ld[4][4];
+      bool use[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int cc = cb + j;
+        use[j] = live && cc <= c_hi && holds(cc);
+        const float4* src =
+            reinterpret_cast<const float4*>((gu ? p.gpart : p.dpart) + (((size_t)cc * nsl + slot_of(cc, sl0)) * 128 + i) * 16);
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        ld[j][0] = use[j] ? __ldcg(src) : z;
+        ld[j][1] = use[j] && q1 ? __ldcg(src + 1) : z;
+        ld[j][2] = use[j] && gu ? __ldcg(src + 2) : z;
+        ld[j][3] = use[j] && gu && q1 ? __ldcg(src + 3) : z;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!use[j]) continue;
+        a[0] += ld[j][0].x; a[1] += ld[j][0].y; a[2] += ld[j][0].z; a[3] += ld[j][0].w;
+        a[4] += ld[j][1].x; a[5] += ld[j][1].y; a[6] += ld[j][1].z; a[7] += ld[j][1].w;
+        b[0] += ld[j][2].x; b[1] += ld[j][2].y; b[2] += ld[j][2].z; b[3] += ld[j][2].w;
+        b[4] += ld[j][3].x; b[5] += ld[j][3].y; b[6] += ld[j][3].z; b[7] += ld[j][3].w;
+      }
+    }
+    if (!q1) {
+#pragma unroll
+      for (int r = 4; r < 8; ++r) a[r] = b[r] = 0.f;   // the general path adds zeros there
+    }
+    if (!gu) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) b[r] = 0.f;
+    }
+    return true;
+  }
   if (live) {
     __stcg(mine, make_float4(a[0], a[1], a[2], a[3]));
     if (q1) __stcg(mine + 1, make_float4(a[4], a[5], a[6], a[7]));
