@@ -303,7 +303,7 @@ int mono_ffn_debug_skip_arrival(mono_ffn_plan_t* plan, int cta, int stage);
 /* Race detection for tests: with max_ns > 0 (at most 100000) every thread
  * that publishes a grid-visible arrival (the stage counters, the split-block
  * arrivals of the tensor-core kernels, the per-expert activation counts)
- * first sleeps a pseudo-random hash(CTA, step epoch, point) % max_ns
+ * first sleeps a pseudo-random hash(CTA, step, point) % max_ns
  * nanoseconds, so the order in which CTAs arrive changes from step to step;
  * results must not change.  0 turns it off (the default). */
 int mono_ffn_debug_jitter(mono_ffn_plan_t* plan, unsigned max_ns);
