@@ -462,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_cc_kernel(const __grid_c
   bar_sync(kBarCons, kCW * 32);
   if (ctid == 0) {
     if (may_publish(p, c->epoch, 4, 4)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_act, 1u);
     }
     wait_count(p, c, &p.sync->cnt_act, ep1, 4u);

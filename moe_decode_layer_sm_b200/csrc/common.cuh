@@ -672,7 +672,6 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
       for (int i = ptid; i < p.n_xready_all; i += kPreThreads) p.xready[i] = 0u;
     bar_sync(kBarPre, kPreThreads);
     if (ptid == 0 && may_publish(p, c->epoch, 1, 0)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_mix, 1u);
     }
     trace(p, 1, ptid == 0);
@@ -724,7 +723,6 @@ __device__ void prologue_mix(const Params& p, Ctl* c, uint8_t* regA, uint32_t ep
     }
     bar_sync(kBarPre, kPreThreads);
     if (ptid == 0 && may_publish(p, c->epoch, 0, 10)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_mix2, 1u);
     }
     if (ptid == 0) wait_count(p, c, &p.sync->cnt_mix2, ep1, 1u);
@@ -914,7 +912,6 @@ __device__ void collapse_norm(const Params& p, Ctl* c, uint8_t* regA, uint32_t e
     }
     bar_sync(kBarCons, kCW * 32);
     if (ctid == 0 && may_publish(p, c->epoch, 7, 1)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_a, 1u);
     }
   }
@@ -1057,7 +1054,6 @@ __device__ __noinline__ void router_logits(const Params& p, Ctl* c, const uint8_
   }
   if (dry) return;
   if (ctid == 0 && may_publish(p, c->epoch, 2, 2)) {
-    __threadfence();
     red_release_add(&p.sync->cnt_logit, 1u);
   }
   trace(p, 4, ctid == 0);

@@ -187,7 +187,6 @@ __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo
         if (gu) __stcg(mine + 2, make_float4(b[0], b[1], b[2], b[3]));
         if (gu && q1) __stcg(mine + 3, make_float4(b[4], b[5], b[6], b[7]));
       }
-      __threadfence();
       bar_sync(kBarEpi, 4 * 32);
       if (tid == 0 && live && may_publish(p, c->epoch, 0, 5 + (uint32_t)sg.list)) red_release_add(cnt, 1u);
       return false;
@@ -684,7 +683,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tc_kernel(const __grid_c
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
     if (tid == 0 && may_publish(p, c->epoch, 6, 9)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_y, 1u);
     }
     tc_fence_before();

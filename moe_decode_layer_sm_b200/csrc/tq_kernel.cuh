@@ -879,7 +879,6 @@ __global__ void __launch_bounds__(kThreads, 1) mono_ffn_tq_kernel(const __grid_c
     trace(p, 9, tid == 0);
     bar_sync(kBarEpi, 4 * 32);
     if (tid == 0 && may_publish(p, c->epoch, 6, 9)) {
-      __threadfence();
       red_release_add(&p.sync->cnt_y, 1u);
     }
     tc_fence_before();
