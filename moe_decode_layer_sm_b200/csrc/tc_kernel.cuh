@@ -8,9 +8,9 @@
 // one contiguous TMA bulk copy, and one tcgen05.mma covers M = 128 rows x
 // K = 16 (4 KB of weights).  Work is cut in units of (block, 128 contraction
 // elements) and every CTA takes an equal contiguous range of units: inside a
-// range the blocks are whole, only the first and last may be partial; the
-// CTA that completes a split block last (an atomic per block) adds the parts
-// in CTA order, so results do not depend on timing.
+// range the blocks are whole, only the first and last may be partial; one
+// CTA adds a split block's parts in CTA order (epi_combine), so results do
+// not depend on timing.
 //
 //   producer (warp 8)   TMA bulk copies into the ring (the ring's depth is
 //                       what keeps enough bytes in flight: an L2 prefetch
@@ -146,9 +146,9 @@ __device__ __forceinline__ const uint8_t* seg_base(const Params& p, const Ctl* c
 
 // Epilogue, thread i (= row i of the 128-row tile) of warps 0-3, with this
 // CTA's part of a block in a[8] (gate, or the down output) and b[8] (up):
-// for a block split across CTAs, publish the part; the CTA that arrives last
-// adds every part in CTA order.  A part is [a0..a7 | b0..b7] of this row;
-// only the quarters the rows and the list need move.  Returns true in the
+// for a split block, publish the part; one CTA (the lowest holder, or on the
+// shared list the last to arrive) adds the parts in CTA order.  A part is
+// [a0..a7 | b0..b7] of this row, only the quarters in use.  Returns true in the
 // CTA that holds the complete block (then a and b hold its sums); the same
 // answer in every epilogue thread.
 __device__ __forceinline__ bool epi_combine(const Params& p, Ctl* c, const TcGeo& geo, const Seg& sg, int upb, bool gu,
