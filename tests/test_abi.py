@@ -43,6 +43,27 @@ def test_plan_refusal_lists_every_reason_without_a_gpu():
         assert frag in msg, (frag, msg)
 
 
+def test_plan_refuses_sizes_beyond_the_32_bit_work_partition():
+    """The kernels partition each work list in 32-bit arithmetic (units x
+    grid < 2^31); the plan refuses larger hidden x inter before any device
+    call, and takes the largest workload of the pages."""
+    from moe_decode_layer_sm_b200 import binding
+    L = binding.lib()
+    import ctypes
+
+    def reasons(hidden, inter):
+        cfg = binding.Config(hidden=hidden, hc=4, n_routed=256, top_k=16, inter=inter, max_rows=8, n_layers=1,
+                             hc_dtype=1, norm_dtype=1, expert_dtype=1, round_bf16=1, sinkhorn_iters=20, device=0)
+        h = ctypes.c_void_p()
+        if L.mono_ffn_plan(ctypes.byref(cfg), ctypes.byref(h)) == 0:   # a GPU box: the plan is made
+            L.mono_ffn_destroy(h)
+            return ""
+        return L.mono_ffn_last_error(None).decode()
+
+    assert "work partition" in reasons(65536, 65536)
+    assert "work partition" not in reasons(5120, 2048)
+
+
 def test_build_is_keyed_on_the_source_hash(tmp_path, monkeypatch):
     """build() trusts the library only when the stamp beside it holds the
     hash of the current sources and nvcc command; a later modification time
