@@ -204,13 +204,30 @@ def parallelism(world):
 
 
 def run_reference(args):
+    """The oracle, as it stands, on the host cores: W untimed steps, then
+    exactly K timed steps, each one layer step of the bounded sample
+    (_oracle_case: the whole step at one row, else row 0 scaled to the
+    rows).  Rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    from oracle import oracle as O
     wl = workload(args.config)
-    # bounded: the whole --steps K --warmup W run stays within a few minutes
-    budget = min(20.0, max(5.0, 60.0 / max(1, args.steps + args.warmup)))
-    cb = cpu_oracle_sample(wl, budget_s=budget)
+    w1, lw, hc, scale, what = _oracle_case(wl)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    _omp_threads(cores)
+    O.layer(w1, lw, hc)   # first touch of the weights
+    for _ in range(args.warmup):
+        O.layer(w1, lw, hc)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.layer(w1, lw, hc)
+        times.append(time.perf_counter() - t0)
+    us = sum(times) / len(times) * 1e6 * scale
+    cb = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+          "sample": f"{what}; {args.warmup} warm-up and {args.steps} timed steps, mean; touched experts generated "
+                    f"before timing"}
     line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": cb["value"] / 1000.0, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
