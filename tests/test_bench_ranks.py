@@ -61,3 +61,30 @@ def test_two_ranks_take_the_max_and_count_every_rank():
     # one rank: no collective, the value is its own time per layer-step
     assert b.job_times(3.0, 4.0, 1, "cpu") == (3.0, 4.0)
     assert b.job_value(400.0, 100, 4, 1) == pytest.approx(1000.0)
+
+
+def test_reference_arm_times_exactly_k_steps_after_w(monkeypatch, capsys):
+    """`bench.py --impl reference` runs the oracle W untimed steps, then
+    exactly K timed steps, and prints one JSON line on the metric's unit
+    with the reference-arm keys (on a small workload, on the CPU)."""
+    import json
+    import types
+    b = _bench()
+    from oracle import oracle as O
+    calls = []
+    real = O.layer
+
+    def counting(*a, **k):
+        calls.append(1)
+        return real(*a, **k)
+
+    monkeypatch.setattr(O, "layer", counting)
+    monkeypatch.setenv("RANK", "0")
+    args = types.SimpleNamespace(config="tiny-fp32-r1", steps=4, warmup=2, gpus=1)
+    b.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert len(calls) == 1 + 2 + 4   # first touch, W warm-up, K timed
+    assert line["impl"] == "reference" and line["steps"] == 4 and line["warmup"] == 2
+    assert line["unit"] == b.UNIT and line["higher_is_better"] is False and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and "2 warm-up and 4 timed steps" in line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": b.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
